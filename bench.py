@@ -1,0 +1,414 @@
+#!/usr/bin/env python
+"""Throughput of blockwise packed causal RoPE attention on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+the forward (RoPE table, block metadata, longest-first order, attention
+kernel) and, for workloads with a backward, the backward (delta, metadata,
+attention backward kernel, dQ conversion), all through the C ABI.
+
+Prints ONE JSON line (rank 0). `value` is mask-aware attention TFLOP/s of
+the whole job (forward 4*D*pairs*H, backward 10*D*pairs*H, pairs = exact
+count of visible (query, key) pairs of the generated segments); tokens/s
+and the forward / backward split ride along.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the fp64 CPU oracle, timed
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own
+independent copy of the workload (weak scaling, no data-path collective);
+timing is the max over ranks of CUDA-event time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_blockwise_causal_b200 import workloads as wl  # noqa: E402
+
+METRIC = ("attention TFLOP/s and tokens/s (fwd, fwd+bwd) at 1 B200; "
+          "% of bf16 tensor peak")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
+                  "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["source"] = "fallback"
+    return d
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.lines = []
+        self.sel = []
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.sel = ["-i", uuid if uuid.startswith("GPU-") else
+                        "GPU-" + uuid]
+        except Exception:
+            self.sel = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", *self.sel, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.th = threading.Thread(target=self._read, daemon=True)
+            self.th.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------ oracle sample
+
+def oracle_sample(w, t_host, budget_s, backward):
+    """Time the fp64 oracle on a prefix of the workload's first row (head 0),
+    sized so one run takes about budget_s. Returns (TFLOP/s, info)."""
+    import oracle
+    from threadpoolctl import threadpool_info
+
+    def run(L):
+        q = t_host["q"][:1, :L, :1]
+        k = t_host["k"][:1, :L, :1]
+        v = t_host["v"][:1, :L, :1]
+        seg = t_host["segment_ids"][:1, :L]
+        pos = t_host["positions"][:1, :L]
+        t0 = time.perf_counter()
+        if backward:
+            g = t_host["dout"][:1, :L, :1]
+            oracle.attn_bwd(q, k, v, g, seg, pos, w.theta)
+        else:
+            oracle.attn_fwd(q, k, v, seg, pos, w.theta)
+        dt = time.perf_counter() - t0
+        segn = seg[0].numpy()
+        runs = np.diff(np.r_[0, np.flatnonzero(np.diff(segn)) + 1, L])
+        pairs = int((runs * (runs + 1) // 2).sum())
+        flop = (14 if backward else 4) * w.D * pairs
+        return dt, flop
+
+    L = min(1024, w.N)
+    dt, _ = run(L)
+    scale = math.sqrt(max(budget_s, 0.1) / max(dt, 1e-3))
+    L = int(min(w.N, max(128, (L * scale) // 128 * 128)))
+    dt, flop = run(L)
+    threads = max((i.get("num_threads", 1) for i in threadpool_info()),
+                  default=1)
+    info = {"sample": f"oracle {'fwd+bwd' if backward else 'fwd'} (fp64, "
+                      f"dense row-blocked) on the first {L} tokens of batch "
+                      f"row 0, head 0 of {w.name}; mask-aware FLOP of that "
+                      f"prefix / wall time",
+            "cores": int(threads), "host_cores": os.cpu_count(),
+            "seconds": dt}
+    return flop / dt / 1e12, info
+
+
+# ------------------------------------------------------------------ main
+
+def init_dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=120),
+            device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, ws, dev):
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reference_arm(args, ws, rank):
+    """The oracle, timed as it stands on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    w = wl.WORKLOADS[args.workload]
+    t_host = wl.make_inputs(w, args.seed, device="cpu",
+                            with_dout=w.backward)
+    times, flops, info = [], [], None
+    for i in range(args.warmup + args.steps):
+        tf, info = oracle_sample(w, t_host, args.ref_budget, w.backward)
+        if i >= args.warmup:
+            times.append(info["seconds"])
+            flops.append(tf)
+    value = float(np.mean(flops))
+    line = {"impl": "reference", "metric": METRIC, "value": value,
+            "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": float(np.mean(times)) * 1e3,
+            "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H,
+                       "D": w.D, "theta": w.theta},
+            "cpu_baseline": {"kind": "oracle", "value": value,
+                             "unit": "TFLOP/s", "cores": info["cores"],
+                             "sample": info["sample"]},
+            "e2e": {"value": value, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="text32k",
+                    choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-budget", type=float, default=6.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    ws, rank, local = init_dist()
+    if args.impl == "reference":
+        reference_arm(args, ws, rank)
+        if ws > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    from long_context_blockwise_causal_b200 import ops
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = wl.WORKLOADS[args.workload]
+    qkp = "bf16x3" if w.scale == 1.0 else "bf16"
+    t = wl.make_inputs(w, args.seed + 1000 * rank, device=dev,
+                       with_dout=w.backward)
+    B, N, H, D = t["q"].shape
+    pairs_per_head = wl.visible_pairs(t["lengths"])
+    fwd_flop = 4.0 * D * pairs_per_head * H
+    bwd_flop = 10.0 * D * pairs_per_head * H if w.backward else 0.0
+    max_pos = int(t["positions"].max().item()) + 1
+    ws_bytes = max(ops.fwd_workspace_size(B, N, H, max_pos),
+                   ops.bwd_workspace_size(B, N, H, max_pos)
+                   if w.backward else 0)
+    workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    out = torch.empty_like(t["q"])
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    grads = [torch.empty_like(t["q"]) for _ in range(3)] if w.backward \
+        else None
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        ops.fwd(t["q"], t["k"], t["v"], t["segment_ids"], t["positions"],
+                w.theta, max_pos=max_pos, qk_precision=qkp, out=out, lse=lse,
+                workspace=workspace, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        if w.backward:
+            ops.bwd(t["q"], t["k"], t["v"], out, t["dout"], lse,
+                    t["segment_ids"], t["positions"], w.theta,
+                    max_pos=max_pos, qk_precision=qkp, dq=grads[0],
+                    dk=grads[1], dv=grads[2], workspace=workspace,
+                    stream=stream)
+            if ev is not None:
+                ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if ops.last_status() != ops.OK:
+        raise SystemExit("device status not OK after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)]
+           for _ in range(args.steps)]
+    clocks = ClockSampler(dev) if rank == 0 else None
+    barrier(ws)
+    torch.cuda.synchronize(dev)
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    launches0 = ops.kernel_launches()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = ops.kernel_launches() - launches0
+    barrier(ws)
+    clk = clocks.stop() if clocks else None
+    status = ops.last_status()
+    ms = start.elapsed_time(end) / args.steps
+    ms = max_over_ranks(ms, ws, dev)
+    fwd_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    bwd_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs])) \
+        if w.backward else 0.0
+
+    # end to end through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        names = ["q", "k", "v", "segment_ids", "positions"] + \
+            (["dout"] if w.backward else [])
+        hin = {n: t[n].cpu().pin_memory() for n in names}
+        hout = [torch.empty(out.shape, dtype=out.dtype).pin_memory(),
+                torch.empty(lse.shape, dtype=lse.dtype).pin_memory()]
+        if w.backward:
+            hout += [torch.empty(out.shape, dtype=out.dtype).pin_memory()
+                     for _ in range(3)]
+        h2d = sum(x.numel() * x.element_size() for x in hin.values())
+        d2h = sum(x.numel() * x.element_size() for x in hout)
+
+        def e2e_step():
+            for n in names:
+                t[n].copy_(hin[n], non_blocking=True)
+            step()
+            res = [out, lse] + (grads if w.backward else [])
+            for hb, db in zip(hout, res):
+                hb.copy_(db, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier(ws)
+        s2 = torch.cuda.Event(enable_timing=True)
+        e2 = torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        ksteps = max(1, min(args.steps, 5))
+        for _ in range(ksteps):
+            e2e_step()
+        e2.record(stream)
+        torch.cuda.synchronize(dev)
+        ems = max_over_ranks(s2.elapsed_time(e2) / ksteps, ws, dev)
+        e2e = {"value": (fwd_flop + bwd_flop) * ws / (ems / 1e3) / 1e12,
+               "unit": "TFLOP/s", "ms_per_step": ems,
+               "tokens_per_s": B * N * ws / (ems / 1e3),
+               "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h)}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        t_host = {k_: (v_.cpu() if torch.is_tensor(v_) else v_)
+                  for k_, v_ in t.items()}
+        tf, info = oracle_sample(w, t_host, args.cpu_budget, w.backward)
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": info["cores"],
+               "kind": "oracle", "sample": info["sample"],
+               "seconds": info["seconds"], "host_cores": info["host_cores"]}
+
+    if rank == 0:
+        pk = peaks()
+        total_flop = (fwd_flop + bwd_flop) * ws
+        value = total_flop / (ms / 1e3) / 1e12
+        peak_burst = pk["bf16_tflops"]
+        peak_sus = pk.get("bf16_tflops_sustained", peak_burst)
+        fwd_tf = fwd_flop / (fwd_ms / 1e3) / 1e12
+        bwd_tf = bwd_flop / (bwd_ms / 1e3) / 1e12 if w.backward else None
+        dom = "bwd" if w.backward and bwd_ms > fwd_ms else "fwd"
+        ach = bwd_tf if dom == "bwd" else fwd_tf
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": B, "N": N, "H": H, "D": D,
+                       "theta": w.theta, "qk_precision": qkp,
+                       "segments": w.segments,
+                       "visible_pairs_per_head": pairs_per_head,
+                       "l2": "inputs larger than L2 (no flush)"
+                       if 3 * t["q"].numel() * 2 > 126e6 else
+                       "inputs smaller than L2 (re-read from L2)",
+                       "parallelism": f"replicas x{ws}"},
+            "tokens_per_s": B * N * ws / (ms / 1e3),
+            "fwd": {"ms": fwd_ms, "tflops": fwd_tf,
+                    "frac_of_burst_peak": fwd_tf / peak_burst},
+            "bwd": ({"ms": bwd_ms, "tflops": bwd_tf,
+                     "frac_of_burst_peak": bwd_tf / peak_burst}
+                    if w.backward else None),
+            "roofline": {"bound": "tensor", "kernel": f"{dom} attention",
+                         "achieved": ach, "peak": peak_sus,
+                         "peak_kind": f"bf16 sustained ({pk['source']})",
+                         "unit": "TFLOP/s", "frac": ach / peak_sus,
+                         "traffic": None},
+            "gpu_launches": int(launches),
+            "device_status": status,
+            "clocks": clk,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

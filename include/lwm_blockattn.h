@@ -1,0 +1,185 @@
+/*
+ * lwm_blockattn.h -- C ABI of liblwm_blockattn.so: blockwise packed causal
+ * RoPE self-attention (forward and backward) on one NVIDIA B200 (sm_100a).
+ *
+ * What is computed (for every batch row b, head h and query token i):
+ *   q~_i = R(pos_i) q_i,  k~_j = R(pos_j) k_j      RoPE, interleaved pairs
+ *   A(i) = { j : seg_j == seg_i and j <= i }         packing + causal mask
+ *   s_ij = (q~_i . k~_j) / sqrt(D)                   for j in A(i)
+ *   lse_i = log sum_{j in A(i)} exp(s_ij)            natural log
+ *   out_i = sum_{j in A(i)} exp(s_ij - lse_i) v_j
+ * and, for the backward, the chain rule of the above with respect to the
+ * un-rotated q and k and to v.
+ *
+ * Where the pages define it:
+ *   - blockwise attention over query/key chunks (scan_query_chunk_size,
+ *     scan_key_chunk_size = block_q, block_k): "LWM：突破 100 万 Token 的
+ *     开源大模型", 配置参数 and 脚本运行说明;
+ *   - masked sequence packing (a token attends only inside its example):
+ *     same page, 概述 contribution (b); "[论文解读] World Model on
+ *     Million-Length Video And Language With Blockwise RingAttention",
+ *     提出的方法;
+ *   - RoPE with a context-scaled theta: same review, 提出的方法;
+ *   - the ring sweep of key/value blocks and the FlashAttention-style
+ *     online softmax: "开源巨兽LWM：如何用RingAttention撬动百万Token多模态
+ *     世界", 3.1 and 3.2; "Inside Large World Model", Stage I.
+ * Readings where the pages are silent: scale 1/sqrt(D); pair k of a head
+ * vector is (x[2k], x[2k+1]) with frequency theta^(-2k/D); angles in fp64;
+ * the causal rule compares token indices (positions drive RoPE only).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the
+ *     library never allocates device memory and never frees anything.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Every call
+ *     except lwm_blockattn_check_inputs and lwm_blockattn_last_status is
+ *     asynchronous on `stream`.
+ *   - Arguments are validated on the host before any launch; on error a
+ *     status code is returned and nothing is launched. Nothing aborts.
+ *   - Layouts (row-major, contiguous):
+ *       q, k, v, out, dout, dq, dk, dv : [B][N][H][D]
+ *       segment_ids, positions         : [B][N] int32
+ *       lse                            : [B][H][N] float32
+ *   - dtype LWM_DTYPE_BF16: q/k/v/out/dout/dq/dk/dv are bfloat16 and the
+ *     tensor-core path runs (tcgen05, fp32 accumulate).
+ *     dtype LWM_DTYPE_FP32: those tensors are float32 and an fp32 CUDA-core
+ *     path runs (accuracy mode; not a performance target).
+ *   - qk_precision LWM_QK_BF16: rotated q and k are rounded to bf16 before
+ *     Q K^T. LWM_QK_BF16X3: they are split as hi + lo (both bf16) and
+ *     Q K^T = hi.hi + hi.lo + lo.hi, for inputs whose scores are large
+ *     enough that bf16 rounding of rotated q/k would move the logsumexp by
+ *     more than ~1e-3. Ignored for LWM_DTYPE_FP32.
+ *   - Preconditions the kernels trust (lwm_blockattn_check_inputs verifies
+ *     them): segment_ids non-decreasing along each batch row (packed
+ *     examples are contiguous runs); 0 <= positions < max_pos.
+ *   - Supported shapes: D == 128; block_q == block_k == 128; any N >= 0
+ *     (a ragged last block is masked); B, H >= 0 (0 => no work); every
+ *     tensor pointer 16-byte aligned.
+ */
+#ifndef LWM_BLOCKATTN_H
+#define LWM_BLOCKATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LWM_BLOCKATTN_VERSION 1
+
+#if defined(__GNUC__)
+#define LWM_API __attribute__((visibility("default")))
+#else
+#define LWM_API
+#endif
+
+typedef enum {
+  LWM_OK = 0,
+  LWM_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, negative size ... */
+  LWM_ERR_UNSUPPORTED = 2,   /* valid but not implemented (D != 128 ...)    */
+  LWM_ERR_WORKSPACE = 3,     /* workspace null or smaller than required     */
+  LWM_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed           */
+  LWM_ERR_TIMEOUT = 5,       /* a device-side bounded wait gave up          */
+  LWM_ERR_PRECONDITION = 6   /* check_inputs: ids decrease / pos range     */
+} lwm_status;
+
+typedef enum { LWM_DTYPE_BF16 = 0, LWM_DTYPE_FP32 = 1 } lwm_dtype;
+typedef enum { LWM_QK_BF16 = 0, LWM_QK_BF16X3 = 1 } lwm_qk_precision;
+
+/* Tile classes written by lwm_blockattn_classify. */
+enum { LWM_TILE_EMPTY = 0, LWM_TILE_PARTIAL = 1, LWM_TILE_FULL = 2 };
+
+/* Bytes of device workspace lwm_blockattn_fwd needs for these sizes
+ * (RoPE cos/sin table of max_pos x D/2 float pairs, per-block segment
+ * ranges, the work list). Returns 0 for invalid sizes. */
+LWM_API size_t lwm_blockattn_fwd_workspace_size(int B, int N, int H, int D,
+                                        int block_q, int block_k,
+                                        int max_pos);
+
+/* Same for lwm_blockattn_bwd: additionally an fp32 dQ accumulator of
+ * B*N*H*D floats and the per-row dot(dO, O) of B*H*N floats. */
+LWM_API size_t lwm_blockattn_bwd_workspace_size(int B, int N, int H, int D,
+                                        int block_q, int block_k,
+                                        int max_pos);
+
+/* Forward. Writes out [B][N][H][D] (dtype) and lse [B][H][N] (fp32,
+ * natural log of the softmax denominator of the scaled scores).
+ * theta > 0 is the RoPE base; positions must lie in [0, max_pos).
+ * The workspace is scratch owned by the caller (>= the size above, 256-byte
+ * aligned); its content on entry does not matter and is clobbered.
+ * Returns LWM_OK or an error status (nothing launched on error). */
+LWM_API int lwm_blockattn_fwd(const void* q, const void* k, const void* v,
+                      const int32_t* segment_ids, const int32_t* positions,
+                      double theta, int block_q, int block_k, int max_pos,
+                      int B, int N, int H, int D, int dtype, int qk_precision,
+                      void* out, float* lse,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward. Given the forward's inputs, its out and lse, and dout (the
+ * gradient of the loss with respect to out), writes dq, dk, dv (dtype,
+ * [B][N][H][D]): gradients with respect to the un-rotated q and k and v.
+ * P is recomputed from lse; dq is accumulated in fp32 in the workspace
+ * (its summation order is not fixed, so dq is not bit-reproducible). */
+LWM_API int lwm_blockattn_bwd(const void* q, const void* k, const void* v,
+                      const void* out, const void* dout, const float* lse,
+                      const int32_t* segment_ids, const int32_t* positions,
+                      double theta, int block_q, int block_k, int max_pos,
+                      int B, int N, int H, int D, int dtype, int qk_precision,
+                      void* dq, void* dk, void* dv,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* Tile classifier (exported so it can be checked bit-exactly). For each
+ * batch row b and query block t (Tq = ceil(N/block_q) blocks), key blocks
+ * j (Tk = ceil(N/block_k)):
+ *   kv_lo[b][t] = (start of the packed example holding row t*block_q)
+ *                 / block_k,
+ *   kv_hi[b][t] = (last valid row of block t) / block_k,
+ *   tile_class[b][t][j] = EMPTY outside [kv_lo, kv_hi]; inside it FULL if
+ *   key block j ends before query block t starts, both blocks lie inside
+ *   [0, N) and the first key and last query share one segment id;
+ *   PARTIAL otherwise.
+ * With non-decreasing ids this equals "EMPTY: no allowed pair, FULL: all
+ * pairs allowed (indices >= N never allowed), PARTIAL: some".
+ * block_k must divide block_q; both in [16, 1024]. tile_class may be NULL
+ * (then only kv_lo/kv_hi are written). Async on stream. */
+LWM_API int lwm_blockattn_classify(const int32_t* segment_ids, int B, int N,
+                           int block_q, int block_k, int32_t* kv_lo,
+                           int32_t* kv_hi, uint8_t* tile_class,
+                           void* stream);
+
+/* RoPE table the kernels use: table[p][k] = (cos a, sin a) as float32 with
+ * a = p * theta^(-2k/D) evaluated in fp64, p in [0, max_pos),
+ * k in [0, D/2). table holds max_pos * D floats. Async on stream. */
+LWM_API int lwm_blockattn_rope_table(double theta, int D, int max_pos, float* table,
+                             void* stream);
+
+/* Synchronous precondition check: returns LWM_OK if segment_ids are
+ * non-decreasing along every row and all positions lie in [0, max_pos),
+ * LWM_ERR_PRECONDITION otherwise. If max_pos_out is non-NULL it receives
+ * 1 + the largest position seen (a valid max_pos for these inputs).
+ * Uses a few bytes of the library's own device memory; synchronises
+ * `stream`. */
+LWM_API int lwm_blockattn_check_inputs(const int32_t* segment_ids,
+                               const int32_t* positions, int B, int N,
+                               int max_pos, int* max_pos_out, void* stream);
+
+/* Synchronises `stream`, then returns and clears the device status word
+ * that the kernels set when a bounded wait gives up (LWM_ERR_TIMEOUT) or
+ * LWM_OK. Also reports a sticky CUDA error as LWM_ERR_CUDA. */
+LWM_API int lwm_blockattn_last_status(void* stream);
+
+/* Static string naming a status code. */
+LWM_API const char* lwm_status_string(int status);
+
+/* LWM_BLOCKATTN_VERSION of the built library. */
+LWM_API int lwm_blockattn_version(void);
+
+/* Number of CUDA kernels this library has launched in this process (all
+ * devices, all streams), counted on the host at each successful launch. */
+LWM_API uint64_t lwm_blockattn_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LWM_BLOCKATTN_H */

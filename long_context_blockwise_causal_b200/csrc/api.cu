@@ -1,0 +1,348 @@
+// C ABI of liblwm_blockattn.so (declared in include/lwm_blockattn.h):
+// host-side validation, workspace carving and the launch sequence of the
+// forward and backward passes.
+#include <atomic>
+#include <cmath>
+#include <cstring>
+
+#include "aux_kernels.cuh"
+#include "tc_kernels.cuh"
+
+namespace lwm {
+
+// Device status word set by bounded waits that give up; read and cleared
+// by lwm_blockattn_last_status.
+__device__ int g_status_word;
+// Result words of lwm_blockattn_check_inputs: [0] violation bits, [1] max
+// position seen.
+__device__ int g_check_words[2];
+
+static std::atomic<uint64_t> g_launches{0};
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Carve {
+  char* base;
+  size_t off = 0;
+  template <typename T>
+  T* take(size_t count) {
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += align_up(count * sizeof(T));
+    return p;
+  }
+};
+
+// Workspace regions shared by forward and backward.
+struct Workspace {
+  float* table;          // [max_pos][D/2] float2
+  int32_t* kv_lo;        // [B][Tq]
+  int32_t* kv_hi;        // [B][Tq]
+  uint64_t* sort_keys;   // [max(B*Uq, B*Uk)]
+  int32_t* order_fwd;    // [B*Uq] units of kFwdRowsPerCta rows, longest first
+  // backward only
+  int32_t* q_lo;         // [B][Tk]
+  int32_t* q_hi;         // [B][Tk]
+  int32_t* order_bwd;    // [B*Uk]
+  float* delta;          // [B][H][N]
+  float* dq_acc;         // [B][N][H][D]
+  size_t bytes;
+};
+
+Workspace carve(void* base, int B, int N, int H, int D, int max_pos,
+                bool backward) {
+  Carve c{static_cast<char*>(base)};
+  Workspace w{};
+  int Tq = (N + kBlock - 1) / kBlock;
+  int Tk = Tq;
+  int Uq = (Tq + kFwdBlocksPerUnit - 1) / kFwdBlocksPerUnit;
+  int Uk = (Tk + kBwdBlocksPerUnit - 1) / kBwdBlocksPerUnit;
+  w.table = c.take<float>(size_t(max_pos) * D);
+  w.kv_lo = c.take<int32_t>(size_t(B) * Tq);
+  w.kv_hi = c.take<int32_t>(size_t(B) * Tq);
+  w.sort_keys = c.take<uint64_t>(size_t(B) * (Uq > Uk ? Uq : Uk));
+  w.order_fwd = c.take<int32_t>(size_t(B) * Uq);
+  if (backward) {
+    w.q_lo = c.take<int32_t>(size_t(B) * Tk);
+    w.q_hi = c.take<int32_t>(size_t(B) * Tk);
+    w.order_bwd = c.take<int32_t>(size_t(B) * Uk);
+    w.delta = c.take<float>(size_t(B) * H * N);
+    w.dq_acc = c.take<float>(size_t(B) * N * H * D);
+  }
+  w.bytes = c.off;
+  return w;
+}
+
+bool sizes_ok(int B, int N, int H, int D, int block_q, int block_k,
+              int max_pos) {
+  return B >= 0 && N >= 0 && H >= 0 && D > 0 && block_q > 0 && block_k > 0 &&
+         max_pos >= 0 && (int64_t(B) * N) < (int64_t(1) << 31);
+}
+
+int shape_status(int D, int block_q, int block_k) {
+  if (D != kHeadDim || block_q != kBlock || block_k != kBlock)
+    return LWM_ERR_UNSUPPORTED;
+  return LWM_OK;
+}
+
+inline bool aligned16(const void* p) {
+  return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? LWM_OK : LWM_ERR_CUDA; }
+
+#define LWM_TRY(expr)                                  \
+  do {                                                 \
+    cudaError_t e_ = (expr);                           \
+    if (e_ != cudaSuccess) return LWM_ERR_CUDA;        \
+  } while (0)
+
+int* status_word() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+  return static_cast<int*>(p);
+}
+
+// Common front half of both passes: RoPE table and block metadata.
+int prepare(const int32_t* seg, double theta, int B, int N, int D,
+            int max_pos, const Workspace& w, cudaStream_t st) {
+  LWM_TRY(launch_rope_table(theta, D, max_pos, w.table, st));
+  LWM_TRY(launch_block_meta(seg, B, N, kBlock, kBlock, w.kv_lo, w.kv_hi, st));
+  return LWM_OK;
+}
+
+}  // namespace
+}  // namespace lwm
+
+using namespace lwm;
+
+extern "C" {
+
+const char* lwm_status_string(int status) {
+  switch (status) {
+    case LWM_OK: return "ok";
+    case LWM_ERR_INVALID_ARG: return "invalid argument";
+    case LWM_ERR_UNSUPPORTED: return "unsupported configuration";
+    case LWM_ERR_WORKSPACE: return "workspace missing or too small";
+    case LWM_ERR_CUDA: return "CUDA error";
+    case LWM_ERR_TIMEOUT: return "device-side wait timed out";
+    case LWM_ERR_PRECONDITION: return "input precondition violated";
+    default: return "unknown status";
+  }
+}
+
+int lwm_blockattn_version(void) { return LWM_BLOCKATTN_VERSION; }
+
+uint64_t lwm_blockattn_kernel_launches(void) {
+  return g_launches.load(std::memory_order_relaxed);
+}
+
+size_t lwm_blockattn_fwd_workspace_size(int B, int N, int H, int D,
+                                        int block_q, int block_k,
+                                        int max_pos) {
+  if (!sizes_ok(B, N, H, D, block_q, block_k, max_pos)) return 0;
+  return carve(nullptr, B, N, H, D, max_pos, false).bytes;
+}
+
+size_t lwm_blockattn_bwd_workspace_size(int B, int N, int H, int D,
+                                        int block_q, int block_k,
+                                        int max_pos) {
+  if (!sizes_ok(B, N, H, D, block_q, block_k, max_pos)) return 0;
+  return carve(nullptr, B, N, H, D, max_pos, true).bytes;
+}
+
+int lwm_blockattn_fwd(const void* q, const void* k, const void* v,
+                      const int32_t* segment_ids, const int32_t* positions,
+                      double theta, int block_q, int block_k, int max_pos,
+                      int B, int N, int H, int D, int dtype, int qk_precision,
+                      void* out, float* lse, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  if (!sizes_ok(B, N, H, D, block_q, block_k, max_pos))
+    return LWM_ERR_INVALID_ARG;
+  if (!(theta > 0.0) || !std::isfinite(theta)) return LWM_ERR_INVALID_ARG;
+  if (dtype != LWM_DTYPE_BF16 && dtype != LWM_DTYPE_FP32)
+    return LWM_ERR_INVALID_ARG;
+  if (qk_precision != LWM_QK_BF16 && qk_precision != LWM_QK_BF16X3)
+    return LWM_ERR_INVALID_ARG;
+  int s = shape_status(D, block_q, block_k);
+  if (s != LWM_OK) return s;
+  if (int64_t(B) * N * H == 0) return LWM_OK;
+  if (max_pos < 1) return LWM_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, segment_ids, positions, out, lse, workspace};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return LWM_ERR_INVALID_ARG;
+  Workspace w = carve(workspace, B, N, H, D, max_pos, false);
+  if (workspace_bytes < w.bytes) return LWM_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = prepare(segment_ids, theta, B, N, D, max_pos, w, st);
+  if (s != LWM_OK) return s;
+  if (dtype == LWM_DTYPE_FP32) {
+    return cuda_status(launch_fwd_simt<float>(
+        static_cast<const float*>(q), static_cast<const float*>(k),
+        static_cast<const float*>(v), segment_ids, positions, w.table,
+        w.kv_lo, B, N, H, static_cast<float*>(out), lse, st));
+  }
+  FwdArgs a{};
+  a.q = q; a.k = k; a.v = v; a.out = out; a.lse = lse;
+  a.seg = segment_ids; a.pos = positions; a.table = w.table;
+  a.kv_lo = w.kv_lo; a.kv_hi = w.kv_hi; a.order = w.order_fwd;
+  a.B = B; a.N = N; a.H = H;
+  a.qk_x3 = qk_precision == LWM_QK_BF16X3;
+  a.status = status_word();
+  if (!a.status) return LWM_ERR_CUDA;
+  LWM_TRY(launch_lpt_order(B, (N + kBlock - 1) / kBlock, kFwdBlocksPerUnit,
+                           w.kv_lo, w.kv_hi, w.sort_keys, w.order_fwd, st));
+  return cuda_status(launch_fwd_tc(a, st));
+}
+
+int lwm_blockattn_bwd(const void* q, const void* k, const void* v,
+                      const void* out, const void* dout, const float* lse,
+                      const int32_t* segment_ids, const int32_t* positions,
+                      double theta, int block_q, int block_k, int max_pos,
+                      int B, int N, int H, int D, int dtype, int qk_precision,
+                      void* dq, void* dk, void* dv, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  if (!sizes_ok(B, N, H, D, block_q, block_k, max_pos))
+    return LWM_ERR_INVALID_ARG;
+  if (!(theta > 0.0) || !std::isfinite(theta)) return LWM_ERR_INVALID_ARG;
+  if (dtype != LWM_DTYPE_BF16 && dtype != LWM_DTYPE_FP32)
+    return LWM_ERR_INVALID_ARG;
+  if (qk_precision != LWM_QK_BF16 && qk_precision != LWM_QK_BF16X3)
+    return LWM_ERR_INVALID_ARG;
+  int s = shape_status(D, block_q, block_k);
+  if (s != LWM_OK) return s;
+  if (int64_t(B) * N * H == 0) return LWM_OK;
+  if (max_pos < 1) return LWM_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, out, dout, lse, segment_ids, positions,
+                        dq, dk, dv, workspace};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return LWM_ERR_INVALID_ARG;
+  Workspace w = carve(workspace, B, N, H, D, max_pos, true);
+  if (workspace_bytes < w.bytes) return LWM_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = prepare(segment_ids, theta, B, N, D, max_pos, w, st);
+  if (s != LWM_OK) return s;
+  const float scale = 1.f / std::sqrt(float(D));
+  LWM_TRY(cudaMemsetAsync(w.dq_acc, 0, sizeof(float) * size_t(B) * N * H * D,
+                          st));
+  if (dtype == LWM_DTYPE_FP32) {
+    using T = float;
+    LWM_TRY(launch_bwd_delta<T>(static_cast<const T*>(out),
+                                static_cast<const T*>(dout), B, N, H, w.delta,
+                                st));
+    LWM_TRY(launch_bwd_simt<T>(
+        static_cast<const T*>(q), static_cast<const T*>(k),
+        static_cast<const T*>(v), static_cast<const T*>(dout), lse, w.delta,
+        segment_ids, positions, w.table, B, N, H, w.dq_acc,
+        static_cast<T*>(dk), static_cast<T*>(dv), st));
+    return cuda_status(launch_dq_convert<T>(w.dq_acc, positions, w.table, B,
+                                            N, H, scale, static_cast<T*>(dq),
+                                            st));
+  }
+  using T = __nv_bfloat16;
+  LWM_TRY(launch_bwd_delta<T>(static_cast<const T*>(out),
+                              static_cast<const T*>(dout), B, N, H, w.delta,
+                              st));
+  if (qk_precision == LWM_QK_BF16X3) {
+    // fp32 CUDA-core backward: at least the precision of the split product
+    LWM_TRY(launch_bwd_simt<T>(
+        static_cast<const T*>(q), static_cast<const T*>(k),
+        static_cast<const T*>(v), static_cast<const T*>(dout), lse, w.delta,
+        segment_ids, positions, w.table, B, N, H, w.dq_acc,
+        static_cast<T*>(dk), static_cast<T*>(dv), st));
+  } else {
+    LWM_TRY(launch_kv_meta(B, (N + kBlock - 1) / kBlock,
+                           (N + kBlock - 1) / kBlock, w.kv_lo, w.kv_hi, w.q_lo,
+                           w.q_hi, st));
+    LWM_TRY(launch_lpt_order(B, (N + kBlock - 1) / kBlock, kBwdBlocksPerUnit,
+                             w.q_lo, w.q_hi, w.sort_keys, w.order_bwd, st));
+    BwdArgs a{};
+    a.q = q; a.k = k; a.v = v; a.dout = dout; a.lse = lse; a.delta = w.delta;
+    a.seg = segment_ids; a.pos = positions; a.table = w.table;
+    a.q_lo = w.q_lo; a.q_hi = w.q_hi; a.order = w.order_bwd;
+    a.dq_acc = w.dq_acc; a.dk = dk; a.dv = dv;
+    a.B = B; a.N = N; a.H = H;
+    a.status = status_word();
+    if (!a.status) return LWM_ERR_CUDA;
+    LWM_TRY(launch_bwd_tc(a, st));
+  }
+  return cuda_status(launch_dq_convert<T>(w.dq_acc, positions, w.table, B, N,
+                                          H, scale, static_cast<T*>(dq), st));
+}
+
+int lwm_blockattn_classify(const int32_t* segment_ids, int B, int N,
+                           int block_q, int block_k, int32_t* kv_lo,
+                           int32_t* kv_hi, uint8_t* tile_class,
+                           void* stream) {
+  if (B < 0 || N < 0 || (int64_t(B) * N) >= (int64_t(1) << 31))
+    return LWM_ERR_INVALID_ARG;
+  if (block_q < 16 || block_q > 1024 || block_k < 16 || block_k > 1024 ||
+      block_q % block_k != 0)
+    return LWM_ERR_UNSUPPORTED;
+  if (int64_t(B) * N == 0) return LWM_OK;
+  if (!segment_ids || !kv_lo || !kv_hi) return LWM_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  LWM_TRY(launch_block_meta(segment_ids, B, N, block_q, block_k, kv_lo, kv_hi,
+                            st));
+  if (tile_class)
+    LWM_TRY(launch_tile_class(segment_ids, B, N, block_q, block_k, kv_lo,
+                              kv_hi, tile_class, st));
+  return LWM_OK;
+}
+
+int lwm_blockattn_rope_table(double theta, int D, int max_pos, float* table,
+                             void* stream) {
+  if (!(theta > 0.0) || !std::isfinite(theta) || D <= 0 || D % 2 ||
+      max_pos < 0)
+    return LWM_ERR_INVALID_ARG;
+  if (max_pos == 0) return LWM_OK;
+  if (!table) return LWM_ERR_INVALID_ARG;
+  return cuda_status(launch_rope_table(theta, D, max_pos, table,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+int lwm_blockattn_check_inputs(const int32_t* segment_ids,
+                               const int32_t* positions, int B, int N,
+                               int max_pos, int* max_pos_out, void* stream) {
+  if (B < 0 || N < 0 || max_pos < 0) return LWM_ERR_INVALID_ARG;
+  if (int64_t(B) * N == 0) {
+    if (max_pos_out) *max_pos_out = 0;
+    return LWM_OK;
+  }
+  if (!segment_ids || !positions) return LWM_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void* words = nullptr;
+  LWM_TRY(cudaGetSymbolAddress(&words, g_check_words));
+  int init[2] = {0, -1};
+  LWM_TRY(cudaMemcpyAsync(words, init, sizeof(init), cudaMemcpyHostToDevice,
+                          st));
+  LWM_TRY(launch_check_inputs(segment_ids, positions, B, N, max_pos,
+                              static_cast<int*>(words), st));
+  int res[2];
+  LWM_TRY(cudaMemcpyAsync(res, words, sizeof(res), cudaMemcpyDeviceToHost, st));
+  LWM_TRY(cudaStreamSynchronize(st));
+  if (max_pos_out) *max_pos_out = res[1] + 1;
+  return res[0] ? LWM_ERR_PRECONDITION : LWM_OK;
+}
+
+int lwm_blockattn_last_status(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return LWM_ERR_CUDA;
+  void* word = nullptr;
+  if (cudaGetSymbolAddress(&word, g_status_word) != cudaSuccess)
+    return LWM_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, word, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return LWM_ERR_CUDA;
+  int zero = 0;
+  if (cudaMemcpy(word, &zero, sizeof(int), cudaMemcpyHostToDevice) !=
+      cudaSuccess)
+    return LWM_ERR_CUDA;
+  return v;
+}
+
+}  // extern "C"

@@ -1,0 +1,358 @@
+// Auxiliary kernels of the blockwise attention path: RoPE table, tile
+// classification and block metadata, the longest-first work order, the
+// precondition check, the backward preprocess and the dQ conversion.
+#include "aux_kernels.cuh"
+
+namespace lwm {
+
+// table[p][k] = (cos a, sin a), a = p * theta^(-2k/D) in fp64 ("[论文解读]
+// World Model on Million-Length Video And Language With Blockwise
+// RingAttention", 提出的方法: RoPE with a context-scaled theta).
+__global__ void rope_table_kernel(double theta, int half_d, int max_pos,
+                                  float2* __restrict__ table) {
+  int64_t n = int64_t(max_pos) * half_d;
+  for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < n;
+       e += int64_t(gridDim.x) * blockDim.x) {
+    int p = int(e / half_d);
+    int k = int(e - int64_t(p) * half_d);
+    double inv_freq = pow(theta, -2.0 * double(k) / double(2 * half_d));
+    double a = double(p) * inv_freq;
+    double s, c;
+    sincos(a, &s, &c);
+    table[e] = make_float2(float(c), float(s));
+  }
+}
+
+// First index of the contiguous run holding row i (ids non-decreasing).
+__device__ __forceinline__ int run_start(const int32_t* __restrict__ seg,
+                                         int i) {
+  int v = seg[i];
+  int lo = 0, hi = i;  // answer in [0, i]
+  while (lo < hi) {
+    int mid = (lo + hi) >> 1;
+    if (seg[mid] < v) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
+__global__ void block_meta_kernel(const int32_t* __restrict__ seg, int B,
+                                  int N, int bq, int bk, int Tq,
+                                  int32_t* __restrict__ kv_lo,
+                                  int32_t* __restrict__ kv_hi) {
+  int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= B * Tq) return;
+  int b = e / Tq, t = e - b * Tq;
+  const int32_t* s = seg + int64_t(b) * N;
+  int qs = t * bq;
+  int qe = min(qs + bq, N) - 1;
+  kv_lo[e] = run_start(s, qs) / bk;
+  kv_hi[e] = qe / bk;
+}
+
+__global__ void tile_class_kernel(const int32_t* __restrict__ seg, int B,
+                                  int N, int bq, int bk, int Tq, int Tk,
+                                  const int32_t* __restrict__ kv_lo,
+                                  const int32_t* __restrict__ kv_hi,
+                                  uint8_t* __restrict__ cls) {
+  int64_t total = int64_t(B) * Tq * Tk;
+  for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+       e < total; e += int64_t(gridDim.x) * blockDim.x) {
+    int j = int(e % Tk);
+    int64_t bt = e / Tk;
+    int t = int(bt % Tq);
+    int b = int(bt / Tq);
+    uint8_t c = LWM_TILE_EMPTY;
+    if (j >= kv_lo[bt] && j <= kv_hi[bt]) {
+      const int32_t* s = seg + int64_t(b) * N;
+      int qs = t * bq, qe = qs + bq - 1;
+      int ks = j * bk, ke = ks + bk - 1;
+      bool full = ke < qs && qe < N && s[ks] == s[qe];
+      c = full ? LWM_TILE_FULL : LWM_TILE_PARTIAL;
+    }
+    cls[e] = c;
+  }
+}
+
+// Key-block view for the backward: query blocks that see key block j form
+// the contiguous range [q_lo, q_hi] (kv_lo and kv_hi are non-decreasing).
+__global__ void kv_meta_kernel(int B, int Tq, int Tk,
+                               const int32_t* __restrict__ kv_lo,
+                               const int32_t* __restrict__ kv_hi,
+                               int32_t* __restrict__ q_lo,
+                               int32_t* __restrict__ q_hi) {
+  int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= B * Tk) return;
+  int b = e / Tk, j = e - b * Tk;
+  const int32_t* lo = kv_lo + int64_t(b) * Tq;
+  const int32_t* hi = kv_hi + int64_t(b) * Tq;
+  // first t with hi[t] >= j
+  int a = 0, z = Tq;
+  while (a < z) { int m = (a + z) >> 1; if (hi[m] < j) a = m + 1; else z = m; }
+  int first = a;
+  // last t with lo[t] <= j
+  a = 0; z = Tq;
+  while (a < z) { int m = (a + z) >> 1; if (lo[m] <= j) a = m + 1; else z = m; }
+  int last = a - 1;
+  q_lo[e] = first;
+  q_hi[e] = last;
+}
+
+// Cost of each unit (b, u): units are groups of `rows_per_unit` blocks of
+// the "outer" dimension whose inner ranges [lo, hi] are unioned.
+__global__ void unit_cost_kernel(int B, int T, int group,
+                                 const int32_t* __restrict__ lo,
+                                 const int32_t* __restrict__ hi, int U,
+                                 uint64_t* __restrict__ keys) {
+  int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= B * U) return;
+  int b = e / U, u = e - b * U;
+  int t0 = u * group, t1 = min(t0 + group, T) - 1;
+  int l = lo[b * T + t0], h = hi[b * T + t0];
+  for (int t = t0 + 1; t <= t1; ++t) {
+    l = min(l, lo[b * T + t]);
+    h = max(h, hi[b * T + t]);
+  }
+  int cost = max(0, h - l + 1);
+  // ascending key order == descending cost, then ascending unit id
+  keys[e] = (uint64_t(0x7FFFFFFF - cost) << 32) | uint32_t(e);
+}
+
+// Longest-first order: one CTA bitonic-sorts up to kSortMax keys in shared
+// memory; the sorted unit ids are written to order[].
+__global__ void __launch_bounds__(1024)
+lpt_sort_kernel(const uint64_t* __restrict__ keys, int n,
+                int32_t* __restrict__ order) {
+  extern __shared__ uint64_t sk[];
+  int p2 = 1;
+  while (p2 < n) p2 <<= 1;
+  for (int i = threadIdx.x; i < p2; i += blockDim.x)
+    sk[i] = i < n ? keys[i] : ~0ull;
+  __syncthreads();
+  for (int size = 2; size <= p2; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < p2; i += blockDim.x) {
+        int j = i ^ stride;
+        if (j > i) {
+          bool up = (i & size) == 0;
+          uint64_t a = sk[i], c = sk[j];
+          if ((a > c) == up) { sk[i] = c; sk[j] = a; }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = threadIdx.x; i < n; i += blockDim.x)
+    order[i] = int32_t(sk[i] & 0xFFFFFFFFu);
+}
+
+// Fallback order for more units than one CTA can sort: per batch row, the
+// units from last to first (longest first for a causal row).
+__global__ void reverse_order_kernel(int B, int U, int32_t* __restrict__ order) {
+  int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= B * U) return;
+  int b = e / U, u = e - b * U;
+  order[e] = b * U + (U - 1 - u);
+}
+
+__global__ void check_inputs_kernel(const int32_t* __restrict__ seg,
+                                    const int32_t* __restrict__ pos, int B,
+                                    int N, int max_pos, int* __restrict__ res) {
+  int64_t total = int64_t(B) * N;
+  int bad = 0, mx = -1;
+  for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+       e < total; e += int64_t(gridDim.x) * blockDim.x) {
+    int i = int(e % N);
+    int p = pos[e];
+    if (p < 0 || p >= max_pos) bad |= 2;
+    mx = max(mx, p);
+    if (i + 1 < N && seg[e + 1] < seg[e]) bad |= 1;
+  }
+  if (bad) atomicOr(&res[0], bad);
+  atomicMax(&res[1], mx);
+}
+
+// D_i = sum_d dO_i[d] * O_i[d] (fp32), stored [B][H][N]; one warp per row.
+template <typename T>
+__global__ void bwd_delta_kernel(const T* __restrict__ out,
+                                 const T* __restrict__ dout, int B, int N,
+                                 int H, float* __restrict__ delta) {
+  int64_t rows = int64_t(B) * N * H;
+  int64_t warp = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5;
+  int lane = threadIdx.x & 31;
+  if (warp >= rows) return;
+  const T* o = out + warp * kHeadDim;
+  const T* g = dout + warp * kHeadDim;
+  float acc = 0.f;
+#pragma unroll
+  for (int i = 0; i < kHeadDim / 32; ++i) {
+    int d = lane + 32 * i;
+    acc += float(o[d]) * float(g[d]);
+  }
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+  if (lane == 0) {
+    int h = int(warp % H);
+    int64_t bn = warp / H;
+    int n = int(bn % N);
+    int b = int(bn / N);
+    delta[(int64_t(b) * H + h) * N + n] = acc;
+  }
+}
+
+// dq = R(-pos) * dq_acc, rounded to T; one thread per (row, pair).
+template <typename T>
+__global__ void dq_convert_kernel(const float* __restrict__ acc,
+                                  const int32_t* __restrict__ pos,
+                                  const float2* __restrict__ table, int B,
+                                  int N, int H, float scale,
+                                  T* __restrict__ dq) {
+  int64_t total = int64_t(B) * N * H * (kHeadDim / 2);
+  for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+       e < total; e += int64_t(gridDim.x) * blockDim.x) {
+    int k = int(e % (kHeadDim / 2));
+    int64_t bnh = e / (kHeadDim / 2);
+    int64_t bn = bnh / H;
+    float2 cs = table[int64_t(pos[bn]) * (kHeadDim / 2) + k];
+    float2 x = reinterpret_cast<const float2*>(acc)[e];
+    x.x *= scale;
+    x.y *= scale;
+    // inverse rotation: (a, b) -> (a c + b s, -a s + b c)
+    float a = x.x * cs.x + x.y * cs.y;
+    float c = x.y * cs.x - x.x * cs.y;
+    dq[2 * e] = T(a);
+    dq[2 * e + 1] = T(c);
+  }
+}
+
+// ------------------------------------------------------------ launchers
+static inline int grid_for(int64_t n, int threads, int cap = 148 * 16) {
+  int64_t g = (n + threads - 1) / threads;
+  return int(g < 1 ? 1 : (g > cap ? cap : g));
+}
+
+cudaError_t launch_rope_table(double theta, int D, int max_pos, float* table,
+                              cudaStream_t st) {
+  if (max_pos <= 0) return cudaSuccess;
+  int64_t n = int64_t(max_pos) * (D / 2);
+  rope_table_kernel<<<grid_for(n, 256, 148 * 32), 256, 0, st>>>(
+      theta, D / 2, max_pos, reinterpret_cast<float2*>(table));
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_block_meta(const int32_t* seg, int B, int N, int bq, int bk,
+                              int32_t* kv_lo, int32_t* kv_hi,
+                              cudaStream_t st) {
+  int Tq = (N + bq - 1) / bq;
+  int n = B * Tq;
+  if (n == 0) return cudaSuccess;
+  block_meta_kernel<<<(n + 255) / 256, 256, 0, st>>>(seg, B, N, bq, bk, Tq,
+                                                      kv_lo, kv_hi);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tile_class(const int32_t* seg, int B, int N, int bq,
+                              int bk, const int32_t* kv_lo,
+                              const int32_t* kv_hi, uint8_t* cls,
+                              cudaStream_t st) {
+  int Tq = (N + bq - 1) / bq, Tk = (N + bk - 1) / bk;
+  int64_t n = int64_t(B) * Tq * Tk;
+  if (n == 0) return cudaSuccess;
+  tile_class_kernel<<<grid_for(n, 256, 148 * 32), 256, 0, st>>>(
+      seg, B, N, bq, bk, Tq, Tk, kv_lo, kv_hi, cls);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_kv_meta(int B, int Tq, int Tk, const int32_t* kv_lo,
+                           const int32_t* kv_hi, int32_t* q_lo, int32_t* q_hi,
+                           cudaStream_t st) {
+  int n = B * Tk;
+  if (n == 0) return cudaSuccess;
+  kv_meta_kernel<<<(n + 255) / 256, 256, 0, st>>>(B, Tq, Tk, kv_lo, kv_hi,
+                                                   q_lo, q_hi);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lpt_order(int B, int T, int group, const int32_t* lo,
+                             const int32_t* hi, uint64_t* keys,
+                             int32_t* order, cudaStream_t st) {
+  int U = (T + group - 1) / group;
+  int n = B * U;
+  if (n == 0) return cudaSuccess;
+  if (n <= kSortMax) {
+    unit_cost_kernel<<<(n + 255) / 256, 256, 0, st>>>(B, T, group, lo, hi, U,
+                                                       keys);
+    note_launch();
+    int p2 = 1;
+    while (p2 < n) p2 <<= 1;
+    size_t smem = size_t(p2) * sizeof(uint64_t);
+    if (smem > 48 * 1024) {
+      cudaError_t e = cudaFuncSetAttribute(
+          lpt_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+          int(smem));
+      if (e != cudaSuccess) return e;
+    }
+    lpt_sort_kernel<<<1, 1024, smem, st>>>(keys, n, order);
+    note_launch();
+  } else {
+    reverse_order_kernel<<<(n + 255) / 256, 256, 0, st>>>(B, U, order);
+    note_launch();
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_check_inputs(const int32_t* seg, const int32_t* pos, int B,
+                                int N, int max_pos, int* res,
+                                cudaStream_t st) {
+  int64_t n = int64_t(B) * N;
+  if (n == 0) return cudaSuccess;
+  check_inputs_kernel<<<grid_for(n, 256), 256, 0, st>>>(seg, pos, B, N,
+                                                         max_pos, res);
+  note_launch();
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_bwd_delta(const T* out, const T* dout, int B, int N, int H,
+                             float* delta, cudaStream_t st) {
+  int64_t rows = int64_t(B) * N * H;
+  if (rows == 0) return cudaSuccess;
+  int64_t threads = rows * 32;
+  bwd_delta_kernel<T><<<int((threads + 255) / 256), 256, 0, st>>>(
+      out, dout, B, N, H, delta);
+  note_launch();
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_dq_convert(const float* acc, const int32_t* pos,
+                              const float* table, int B, int N, int H,
+                              float scale, T* dq, cudaStream_t st) {
+  int64_t n = int64_t(B) * N * H * (kHeadDim / 2);
+  if (n == 0) return cudaSuccess;
+  dq_convert_kernel<T><<<grid_for(n, 256, 148 * 32), 256, 0, st>>>(
+      acc, pos, reinterpret_cast<const float2*>(table), B, N, H, scale, dq);
+  note_launch();
+  return cudaGetLastError();
+}
+
+template cudaError_t launch_bwd_delta<__nv_bfloat16>(const __nv_bfloat16*,
+                                                     const __nv_bfloat16*, int,
+                                                     int, int, float*,
+                                                     cudaStream_t);
+template cudaError_t launch_bwd_delta<float>(const float*, const float*, int,
+                                             int, int, float*, cudaStream_t);
+template cudaError_t launch_dq_convert<__nv_bfloat16>(const float*,
+                                                      const int32_t*,
+                                                      const float*, int, int,
+                                                      int, float,
+                                                      __nv_bfloat16*,
+                                                      cudaStream_t);
+template cudaError_t launch_dq_convert<float>(const float*, const int32_t*,
+                                              const float*, int, int, int,
+                                              float, float*, cudaStream_t);
+
+}  // namespace lwm

@@ -1,0 +1,48 @@
+// Launchers of the auxiliary kernels (see aux_kernels.cu).
+#pragma once
+
+#include "common.cuh"
+
+namespace lwm {
+
+constexpr int kSortMax = 16384;  // units one CTA sorts in shared memory
+
+cudaError_t launch_rope_table(double theta, int D, int max_pos, float* table,
+                              cudaStream_t st);
+cudaError_t launch_block_meta(const int32_t* seg, int B, int N, int bq, int bk,
+                              int32_t* kv_lo, int32_t* kv_hi, cudaStream_t st);
+cudaError_t launch_tile_class(const int32_t* seg, int B, int N, int bq, int bk,
+                              const int32_t* kv_lo, const int32_t* kv_hi,
+                              uint8_t* cls, cudaStream_t st);
+cudaError_t launch_kv_meta(int B, int Tq, int Tk, const int32_t* kv_lo,
+                           const int32_t* kv_hi, int32_t* q_lo, int32_t* q_hi,
+                           cudaStream_t st);
+// Orders the units (b, u), u covering `group` consecutive blocks, by the
+// size of the union of their [lo, hi] ranges, longest first.
+cudaError_t launch_lpt_order(int B, int T, int group, const int32_t* lo,
+                             const int32_t* hi, uint64_t* keys, int32_t* order,
+                             cudaStream_t st);
+cudaError_t launch_check_inputs(const int32_t* seg, const int32_t* pos, int B,
+                                int N, int max_pos, int* res, cudaStream_t st);
+template <typename T>
+cudaError_t launch_bwd_delta(const T* out, const T* dout, int B, int N, int H,
+                             float* delta, cudaStream_t st);
+template <typename T>
+cudaError_t launch_dq_convert(const float* acc, const int32_t* pos,
+                              const float* table, int B, int N, int H,
+                              float scale, T* dq, cudaStream_t st);
+
+// CUDA-core kernels (fp32 arithmetic), any I/O type.
+template <typename T>
+cudaError_t launch_fwd_simt(const T* q, const T* k, const T* v,
+                            const int32_t* seg, const int32_t* pos,
+                            const float* table, const int32_t* kv_lo, int B,
+                            int N, int H, T* out, float* lse, cudaStream_t st);
+template <typename T>
+cudaError_t launch_bwd_simt(const T* q, const T* k, const T* v, const T* dout,
+                            const float* lse, const float* delta,
+                            const int32_t* seg, const int32_t* pos,
+                            const float* table, int B, int N, int H,
+                            float* dq_acc, T* dk, T* dv, cudaStream_t st);
+
+}  // namespace lwm

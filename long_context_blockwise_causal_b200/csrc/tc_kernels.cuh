@@ -1,0 +1,53 @@
+// Tensor-core (tcgen05) kernels of the blockwise attention path.
+#pragma once
+
+#include "common.cuh"
+
+namespace lwm {
+
+// A forward CTA owns this many consecutive 128-row query blocks of one
+// (batch row, head); a backward CTA this many 128-key blocks.
+constexpr int kFwdBlocksPerUnit = 2;
+constexpr int kBwdBlocksPerUnit = 1;
+
+struct FwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;
+  float* lse;
+  const int32_t* seg;
+  const int32_t* pos;
+  const float* table;
+  const int32_t* kv_lo;
+  const int32_t* kv_hi;
+  const int32_t* order;
+  int B, N, H;
+  bool qk_x3;
+  int* status;
+};
+
+struct BwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* dout;
+  const float* lse;
+  const float* delta;
+  const int32_t* seg;
+  const int32_t* pos;
+  const float* table;
+  const int32_t* q_lo;
+  const int32_t* q_hi;
+  const int32_t* order;
+  float* dq_acc;
+  void* dk;
+  void* dv;
+  int B, N, H;
+  int* status;
+};
+
+cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t st);
+cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t st);
+
+}  // namespace lwm

@@ -1,0 +1,236 @@
+"""ctypes binding of liblwm_blockattn.so (argument marshalling only).
+
+Every step of the attention path runs in the library's CUDA kernels; this
+module turns torch tensors into device pointers, sizes and the current
+stream, and turns status codes into exceptions. It never computes
+anything itself and has no fallback: without the built library (or on a
+tensor that is not on a CUDA device) it raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                         "liblwm_blockattn.so")
+_lib = None
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, \
+    ERR_TIMEOUT, ERR_PRECONDITION = range(7)
+DTYPE_BF16, DTYPE_FP32 = 0, 1
+QK_BF16, QK_BF16X3 = 0, 1
+TILE_EMPTY, TILE_PARTIAL, TILE_FULL = 0, 1, 2
+BLOCK = 128
+HEAD_DIM = 128
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_sz = ctypes.c_size_t
+_d = ctypes.c_double
+
+_SIGS = {
+    "lwm_blockattn_fwd_workspace_size": (_sz, [_i] * 7),
+    "lwm_blockattn_bwd_workspace_size": (_sz, [_i] * 7),
+    "lwm_blockattn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _d, _i, _i, _i,
+                               _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _sz,
+                               _vp]),
+    "lwm_blockattn_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _d,
+                               _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp,
+                               _vp, _vp, _sz, _vp]),
+    "lwm_blockattn_classify": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp,
+                                    _vp]),
+    "lwm_blockattn_rope_table": (_i, [_d, _i, _i, _vp, _vp]),
+    "lwm_blockattn_check_inputs": (_i, [_vp, _vp, _i, _i, _i,
+                                        ctypes.POINTER(_i), _vp]),
+    "lwm_blockattn_last_status": (_i, [_vp]),
+    "lwm_status_string": (ctypes.c_char_p, [_i]),
+    "lwm_blockattn_version": (_i, []),
+    "lwm_blockattn_kernel_launches": (ctypes.c_uint64, []),
+}
+
+
+class LwmError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+def lib() -> ctypes.CDLL:
+    """Load the shared library once; raise if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(
+                f"{_LIB_PATH} is missing; build it with "
+                "`python -m long_context_blockwise_causal_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def exported_symbols():
+    return list(_SIGS)
+
+
+def status_string(status: int) -> str:
+    return lib().lwm_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        raise LwmError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return DTYPE_BF16
+    if t.dtype == torch.float32:
+        return DTYPE_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _qk_code(qk_precision) -> int:
+    if qk_precision in (QK_BF16, "bf16"):
+        return QK_BF16
+    if qk_precision in (QK_BF16X3, "bf16x3"):
+        return QK_BF16X3
+    raise ValueError(f"qk_precision {qk_precision!r}")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def fwd_workspace_size(B, N, H, max_pos, D=HEAD_DIM, block_q=BLOCK,
+                       block_k=BLOCK) -> int:
+    return int(lib().lwm_blockattn_fwd_workspace_size(B, N, H, D, block_q,
+                                                      block_k, max_pos))
+
+
+def bwd_workspace_size(B, N, H, max_pos, D=HEAD_DIM, block_q=BLOCK,
+                       block_k=BLOCK) -> int:
+    return int(lib().lwm_blockattn_bwd_workspace_size(B, N, H, D, block_q,
+                                                      block_k, max_pos))
+
+
+def _workspace(nbytes, device, workspace):
+    if workspace is None:
+        return torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
+    if workspace.numel() * workspace.element_size() < nbytes:
+        raise LwmError(ERR_WORKSPACE, "workspace")
+    return workspace
+
+
+def fwd(q, k, v, segment_ids, positions, theta, max_pos=None,
+        qk_precision="bf16", out=None, lse=None, workspace=None,
+        stream=None, block_q=BLOCK, block_k=BLOCK):
+    """Forward pass. Returns (out [B,N,H,D] in q's dtype, lse [B,H,N] fp32)."""
+    _need_cuda(q, k, v, segment_ids, positions, out, lse, workspace)
+    B, N, H, D = q.shape
+    if max_pos is None:
+        max_pos = int(positions.max().item()) + 1 if positions.numel() else 1
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    ws = _workspace(fwd_workspace_size(B, N, H, max_pos, D, block_q, block_k),
+                    q.device, workspace)
+    st = lib().lwm_blockattn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(segment_ids), _ptr(positions),
+        float(theta), block_q, block_k, int(max_pos), B, N, H, D,
+        _dtype_code(q), _qk_code(qk_precision), _ptr(out), _ptr(lse),
+        _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "lwm_blockattn_fwd")
+    return out, lse
+
+
+def bwd(q, k, v, out, dout, lse, segment_ids, positions, theta,
+        max_pos=None, qk_precision="bf16", dq=None, dk=None, dv=None,
+        workspace=None, stream=None, block_q=BLOCK, block_k=BLOCK):
+    """Backward pass. Returns (dq, dk, dv) in q's dtype."""
+    _need_cuda(q, k, v, out, dout, lse, segment_ids, positions, dq, dk, dv,
+               workspace)
+    B, N, H, D = q.shape
+    if max_pos is None:
+        max_pos = int(positions.max().item()) + 1 if positions.numel() else 1
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    ws = _workspace(bwd_workspace_size(B, N, H, max_pos, D, block_q, block_k),
+                    q.device, workspace)
+    st = lib().lwm_blockattn_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
+        _ptr(segment_ids), _ptr(positions), float(theta), block_q, block_k,
+        int(max_pos), B, N, H, D, _dtype_code(q), _qk_code(qk_precision),
+        _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "lwm_blockattn_bwd")
+    return dq, dk, dv
+
+
+def classify(segment_ids, block_q=BLOCK, block_k=BLOCK, with_class=True,
+             stream=None):
+    """Returns kv_lo, kv_hi [B,Tq] int32 and tile_class [B,Tq,Tk] uint8."""
+    _need_cuda(segment_ids)
+    B, N = segment_ids.shape
+    tq = -(-N // block_q)
+    tk = -(-N // block_k)
+    dev = segment_ids.device
+    lo = torch.empty((B, tq), dtype=torch.int32, device=dev)
+    hi = torch.empty((B, tq), dtype=torch.int32, device=dev)
+    cls = torch.empty((B, tq, tk), dtype=torch.uint8, device=dev) \
+        if with_class else None
+    st = lib().lwm_blockattn_classify(_ptr(segment_ids), B, N, block_q,
+                                      block_k, _ptr(lo), _ptr(hi), _ptr(cls),
+                                      _stream(stream))
+    _check(st, "lwm_blockattn_classify")
+    return lo, hi, cls
+
+
+def rope_table(theta, max_pos, D=HEAD_DIM, device="cuda", stream=None):
+    """The fp32 (cos, sin) table [max_pos, D/2, 2] the kernels use."""
+    t = torch.empty((max_pos, D // 2, 2), dtype=torch.float32, device=device)
+    st = lib().lwm_blockattn_rope_table(float(theta), D, max_pos, _ptr(t),
+                                        _stream(stream))
+    _check(st, "lwm_blockattn_rope_table")
+    return t
+
+
+def check_inputs(segment_ids, positions, max_pos, stream=None):
+    """(ok, 1 + largest position). Synchronous."""
+    _need_cuda(segment_ids, positions)
+    B, N = segment_ids.shape
+    mp = ctypes.c_int(0)
+    st = lib().lwm_blockattn_check_inputs(_ptr(segment_ids), _ptr(positions),
+                                          B, N, int(max_pos),
+                                          ctypes.byref(mp), _stream(stream))
+    if st not in (OK, ERR_PRECONDITION):
+        _check(st, "lwm_blockattn_check_inputs")
+    return st == OK, mp.value
+
+
+def kernel_launches() -> int:
+    """Kernels the library has launched in this process so far."""
+    return int(lib().lwm_blockattn_kernel_launches())
+
+
+def last_status(stream=None) -> int:
+    return int(lib().lwm_blockattn_last_status(_stream(stream)))

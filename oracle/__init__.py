@@ -38,7 +38,8 @@ Modules:
 
 from .rope import rope_inv_freq, rope_angles, rope_rotate  # noqa: F401
 from .attention import (  # noqa: F401
-    allowed_mask, attn_fwd, attn_fwd_rows, attn_bwd, SOFTMAX_SCALE_RULE,
+    allowed_mask, attn_fwd, attn_fwd_rows, attn_bwd, attn_bwd_rows,
+    attn_bwd_cols, SOFTMAX_SCALE_RULE,
 )
 from .blockwise import blockwise_fwd  # noqa: F401
 from .classify import (  # noqa: F401

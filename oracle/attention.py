@@ -174,3 +174,73 @@ def attn_bwd(q, k, v, dout, segment_ids, positions, theta, heads=None,
             out[b, :, h, :] = o
             lse[b, h, :] = ls
     return {"dq": dq, "dk": dk, "dv": dv, "out": out, "lse": lse}
+
+
+def attn_bwd_rows(q, k, v, dout, segment_ids, positions, theta, b, h, rows,
+                  row_block=256):
+    """dq at query rows ``rows`` of (b, h), fp64 [len(rows), D].
+
+    Only row i's own softmax enters dq_i: dq~_i = sum_j dS_ij k~_j / sqrt(D)
+    with dS_ij = P_ij (dP_ij - dO_i . O_i), so the rows can be computed one
+    by one at any sequence length.
+    """
+    seg = _i64(segment_ids)[b]
+    pos = _i64(positions)[b]
+    rows = np.asarray(rows, dtype=np.int64)
+    kb = _f64(k[b, :, h, :])
+    vb = _f64(v[b, :, h, :])
+    n, d = kb.shape
+    scale = 1.0 / np.sqrt(d)
+    kr = rope_rotate(kb, pos, theta)
+    cols = np.arange(n)
+    dq = np.empty((len(rows), d))
+    for s0 in range(0, len(rows), row_block):
+        r = rows[s0:s0 + row_block]
+        qr = rope_rotate(_f64(q[b, r, h, :]), pos[r], theta)
+        s = _scores(qr, kr, scale, allowed_mask(seg, r, cols))
+        mx = s.max(axis=1, keepdims=True)
+        l_ = np.log(np.exp(s - mx).sum(axis=1, keepdims=True)) + mx
+        p = np.exp(s - l_)
+        o = p @ vb
+        dob = _f64(dout[b, r, h, :])
+        delta = (dob * o).sum(axis=1, keepdims=True)
+        ds = p * (dob @ vb.T - delta)
+        dq[s0:s0 + len(r)] = rope_rotate((ds @ kr) * scale, pos[r], theta,
+                                         sign=-1)
+    return dq
+
+
+def attn_bwd_cols(q, k, v, dout, segment_ids, positions, theta, b, h, cols,
+                  row_block=256):
+    """dk, dv at key columns ``cols`` of (b, h), fp64 [len(cols), D] each.
+
+    Key j collects from every query i that sees it, so the forward of the
+    whole head (lse_i, O_i for all i) is computed first.
+    """
+    seg = _i64(segment_ids)[b]
+    pos = _i64(positions)[b]
+    cols = np.asarray(cols, dtype=np.int64)
+    qb = _f64(q[b, :, h, :])
+    kb = _f64(k[b, :, h, :])
+    vb = _f64(v[b, :, h, :])
+    dob = _f64(dout[b, :, h, :])
+    n, d = kb.shape
+    scale = 1.0 / np.sqrt(d)
+    qr = rope_rotate(qb, pos, theta)
+    kr = rope_rotate(kb, pos, theta)
+    allc = np.arange(n)
+    dk_r = np.zeros((len(cols), d))
+    dv_ = np.zeros((len(cols), d))
+    for s0 in range(0, n, row_block):
+        r = allc[s0:s0 + row_block]
+        s = _scores(qr[r], kr, scale, allowed_mask(seg, r, allc))
+        mx = s.max(axis=1, keepdims=True)
+        l_ = np.log(np.exp(s - mx).sum(axis=1, keepdims=True)) + mx
+        p_all = np.exp(s - l_)
+        o = p_all @ vb
+        delta = (dob[r] * o).sum(axis=1, keepdims=True)
+        p = p_all[:, cols]
+        ds = p * (dob[r] @ vb[cols].T - delta)
+        dv_ += p.T @ dob[r]
+        dk_r += (ds.T @ qr[r]) * scale
+    return rope_rotate(dk_r, pos[cols], theta, sign=-1), dv_

@@ -1,0 +1,114 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point the header declares, sizes workspaces, and rejects bad
+arguments with status codes before touching the device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from long_context_blockwise_causal_b200 import ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    names = []
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", f)).read()
+            names += re.findall(r"LWM_API\s+[\w\s\*]+?\b(lwm_\w+)\s*\(", txt)
+    return names
+
+
+def test_header_declares_the_bound_entry_points():
+    declared = set(header_functions())
+    assert declared, "no LWM_API declarations found"
+    assert declared == set(ops.exported_symbols())
+
+
+def test_library_exports_every_declared_symbol():
+    L = ops.lib()
+    for name in header_functions():
+        assert hasattr(L, name), name
+    assert L.lwm_blockattn_version() == 1
+
+
+def test_status_strings():
+    assert ops.status_string(ops.OK) == "ok"
+    assert "workspace" in ops.status_string(ops.ERR_WORKSPACE)
+    assert ops.status_string(99) == "unknown status"
+
+
+def test_workspace_sizes_grow_with_inputs():
+    a = ops.fwd_workspace_size(1, 2048, 4, 2048)
+    b = ops.fwd_workspace_size(1, 65536, 4, 2048)
+    c = ops.fwd_workspace_size(1, 2048, 4, 4096)
+    assert 0 < a < b and a < c
+    # table dominates: max_pos * D floats
+    assert c - a >= (4096 - 2048) * 128 * 4
+    bw = ops.bwd_workspace_size(1, 2048, 4, 2048)
+    assert bw >= a + 2048 * 4 * 128 * 4  # + fp32 dq accumulator
+    assert ops.fwd_workspace_size(-1, 2048, 4, 2048) == 0
+    assert ops.bwd_workspace_size(1, -5, 4, 2048) == 0
+
+
+def _fwd_raw(**kw):
+    args = dict(q=1 << 20, k=1 << 20, v=1 << 20, seg=1 << 20, pos=1 << 20,
+                theta=1e4, bq=128, bk=128, max_pos=16, B=1, N=16, H=1, D=128,
+                dtype=0, qkp=0, out=1 << 20, lse=1 << 20, ws=1 << 20,
+                wsb=1 << 40, stream=None)
+    args.update(kw)
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    return ops.lib().lwm_blockattn_fwd(
+        v(args["q"]), v(args["k"]), v(args["v"]), v(args["seg"]),
+        v(args["pos"]), args["theta"], args["bq"], args["bk"],
+        args["max_pos"], args["B"], args["N"], args["H"], args["D"],
+        args["dtype"], args["qkp"], v(args["out"]), v(args["lse"]),
+        v(args["ws"]), args["wsb"], v(args["stream"]))
+
+
+@pytest.mark.parametrize("kw,status", [
+    ({"q": None}, ops.ERR_INVALID_ARG),
+    ({"lse": None}, ops.ERR_INVALID_ARG),
+    ({"ws": None}, ops.ERR_INVALID_ARG),
+    ({"k": (1 << 20) + 2}, ops.ERR_INVALID_ARG),     # misaligned
+    ({"theta": -1.0}, ops.ERR_INVALID_ARG),
+    ({"theta": float("nan")}, ops.ERR_INVALID_ARG),
+    ({"dtype": 7}, ops.ERR_INVALID_ARG),
+    ({"qkp": 5}, ops.ERR_INVALID_ARG),
+    ({"N": -1}, ops.ERR_INVALID_ARG),
+    ({"max_pos": 0}, ops.ERR_INVALID_ARG),
+    ({"D": 64}, ops.ERR_UNSUPPORTED),
+    ({"bq": 64}, ops.ERR_UNSUPPORTED),
+    ({"bk": 64}, ops.ERR_UNSUPPORTED),
+    ({"wsb": 100}, ops.ERR_WORKSPACE),
+    ({"N": 0, "q": None}, ops.OK),                    # empty: no work
+    ({"H": 0}, ops.OK),
+    ({"B": 0}, ops.OK),
+])
+def test_fwd_rejects_bad_arguments_before_launch(kw, status):
+    assert _fwd_raw(**kw) == status
+
+
+def test_bwd_and_classify_reject_bad_arguments():
+    L = ops.lib()
+    v = ctypes.c_void_p
+    p = v(1 << 20)
+    st = L.lwm_blockattn_bwd(p, p, p, p, p, p, p, p, 1e4, 128, 128, 16, 1, 16,
+                             1, 128, 0, 0, p, p, None, p, 1 << 40, None)
+    assert st == ops.ERR_INVALID_ARG  # dv is NULL
+    st = L.lwm_blockattn_bwd(p, p, p, p, p, p, p, p, 1e4, 128, 128, 16, 1, 16,
+                             1, 128, 0, 0, p, p, p, p, 10, None)
+    assert st == ops.ERR_WORKSPACE
+    assert L.lwm_blockattn_classify(p, 1, 16, 128, 48, p, p, None,
+                                    None) == ops.ERR_UNSUPPORTED
+    assert L.lwm_blockattn_classify(None, 1, 16, 128, 128, p, p, None,
+                                    None) == ops.ERR_INVALID_ARG
+    assert L.lwm_blockattn_classify(None, 0, 16, 128, 128, None, None, None,
+                                    None) == ops.OK
+    assert L.lwm_blockattn_rope_table(0.0, 128, 10, p, None) == \
+        ops.ERR_INVALID_ARG
+    assert L.lwm_blockattn_rope_table(1e4, 127, 10, p, None) == \
+        ops.ERR_INVALID_ARG

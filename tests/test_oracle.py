@@ -391,3 +391,17 @@ def test_segment_generators_shapes():
     video = L[L % wl.TOKENS_PER_FRAME == 0]
     assert len(video) > 0
     assert wl.visible_pairs([np.array([3, 1])]) == 7
+
+
+def test_sampled_backward_rows_and_cols_equal_full_backward():
+    q, k, v, seg, pos = rand_case(17, N=90, H=2, D=16, lo=1, hi=40)
+    g = np.random.default_rng(18).standard_normal(q.shape)
+    full = oracle.attn_bwd(q, k, v, g, seg, pos, 1e5)
+    rows = np.array([0, 3, 44, 89])
+    dq = oracle.attn_bwd_rows(q, k, v, g, seg, pos, 1e5, 0, 1, rows,
+                              row_block=3)
+    np.testing.assert_allclose(dq, full["dq"][0, rows, 1], atol=1e-12)
+    dk, dv = oracle.attn_bwd_cols(q, k, v, g, seg, pos, 1e5, 0, 0, rows,
+                                  row_block=7)
+    np.testing.assert_allclose(dk, full["dk"][0, rows, 0], atol=1e-12)
+    np.testing.assert_allclose(dv, full["dv"][0, rows, 0], atol=1e-12)
