@@ -71,7 +71,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Bounded wait for the phase with the given parity to complete. Returns
 // false (after recording a timeout in *status and raising *abort) if it did
-// not complete within limit_ns, or if another role already aborted.
+// not complete within limit_ns, or if another role already aborted. With
+// abort == nullptr the wait ignores other roles (used to drain copies that
+// are still in flight before the CTA exits).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           volatile int* abort, int* status,
                                           uint64_t limit_ns) {
@@ -80,9 +82,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63) == 0) {
-      if (*abort) return false;
+      if (abort && *abort) return false;
       if (globaltimer_ns() - t0 > limit_ns) {
-        *abort = 1;
+        if (abort) *abort = 1;
         atomicMax(status, kStatusTimeout);
         return false;
       }

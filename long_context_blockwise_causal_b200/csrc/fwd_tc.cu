@@ -1,0 +1,690 @@
+// Forward blockwise packed causal RoPE attention on tcgen05 (sm_100a).
+//
+// Method ("开源巨兽LWM：如何用RingAttention撬动百万Token多模态世界", 3.1-3.2;
+// "LWM：突破 100 万 Token 的开源大模型", 配置参数 and 概述 (b)): the query
+// blocks of one (batch row, head) sweep the key/value blocks from the block
+// holding their diagonal down to the start of their packed example, keeping
+// a running max, a running sum and an output accumulator (online softmax);
+// RoPE ("[论文解读] World Model on Million-Length Video And Language With
+// Blockwise RingAttention", 提出的方法) is applied to the Q and K tiles in
+// shared memory right after they land.
+//
+// CTA = persistent worker over units of 2 x 128 query rows of one (b, h):
+//   warps 0-3   softmax for query sub-tile 0 (TMEM lanes 0-127)
+//   warps 4-7   softmax for query sub-tile 1
+//   warps 8-11  RoPE: rotate each landed Q / K tile in place (fp32 math,
+//               bf16 round to nearest even; hi/lo split in the x3 mode)
+//   warp 12     TMA producer (Q per unit, K and V per key block)
+//   warp 13     tcgen05 issuer (one elected lane) + TMEM owner
+// TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; P (bf16)
+// is written over the first 64 columns of S and read from there by the
+// P.V MMA. O is rescaled in TMEM only when a row max grows by more than
+// 2^8 (the result is exact either way: max and sum stay consistent).
+#include <cuda.h>
+
+#include "aux_kernels.cuh"
+#include "tc_kernels.cuh"
+
+namespace lwm {
+namespace {
+
+constexpr int kThreadsFwd = 14 * 32;
+constexpr int kTileBytes = kBlock * kHeadDim * 2;       // 32 KB bf16 tile
+constexpr int kHalfTileBytes = kTileBytes / 2;          // one 64-wide d chunk
+constexpr uint64_t kWaitLimitNs = 4000000000ull;        // 4 s per wait
+constexpr float kRescaleThreshold = 8.0f;               // log2 units
+
+template <bool X3>
+struct FwdCfg {
+  static constexpr int KS = X3 ? 1 : 2;   // K stages
+  static constexpr int VS = X3 ? 1 : 2;   // V stages
+  static constexpr int kQ = 0;
+  static constexpr int kQlo = kQ + 2 * kTileBytes;
+  static constexpr int kK = kQlo + (X3 ? 2 * kTileBytes : 0);
+  static constexpr int kKlo = kK + KS * kTileBytes;
+  static constexpr int kV = kKlo + (X3 ? KS * kTileBytes : 0);
+  static constexpr int kBars = kV + VS * kTileBytes;
+  // barrier slots
+  static constexpr int bQFull = 0, bQReady = 2, bQEmpty = 4, bSFull = 6,
+                       bPFull = 8, bOFull = 10, bOEmpty = 12, bEpi = 14,
+                       bDone = 16, bKFull = 17,
+                       bKReady = bKFull + KS, bKEmpty = bKReady + KS,
+                       bVFull = bKEmpty + KS, bVEmpty = bVFull + VS,
+                       kNumBars = bVEmpty + VS;
+  static constexpr int kMisc = kBars + kNumBars * 8;
+  static constexpr int kSmem = kMisc + 16 + 1024;  // + alignment slack
+};
+
+struct FwdParams {
+  const int32_t* seg;
+  const int32_t* pos;
+  const float2* table;
+  const int32_t* kv_lo;
+  const int32_t* kv_hi;
+  const int32_t* order;
+  float* lse;
+  int* status;
+  int B, N, H, Tq, U, G;
+  int total_items;
+  float scale_log2;
+};
+
+struct Item {
+  int b, h, t[2];
+  int lo[2], hi[2];
+  int jlo, jhi;
+  bool present[2];
+};
+
+__device__ __forceinline__ Item get_item(const FwdParams& p, int it) {
+  Item m;
+  int per_group = p.G * p.B * p.U;
+  int hg = it / per_group;
+  int rem = it - hg * per_group;
+  int r = rem / p.G;
+  int hh = rem - r * p.G;
+  m.h = hg * p.G + hh;
+  int unit = p.order[r];
+  m.b = unit / p.U;
+  int u = unit - m.b * p.U;
+  m.jlo = 1 << 30;
+  m.jhi = -1;
+#pragma unroll
+  for (int s = 0; s < 2; ++s) {
+    m.t[s] = 2 * u + s;
+    m.present[s] = m.t[s] < p.Tq;
+    if (m.present[s]) {
+      m.lo[s] = p.kv_lo[m.b * p.Tq + m.t[s]];
+      m.hi[s] = p.kv_hi[m.b * p.Tq + m.t[s]];
+      m.jlo = min(m.jlo, m.lo[s]);
+      m.jhi = max(m.jhi, m.hi[s]);
+    } else {
+      m.lo[s] = 1;
+      m.hi[s] = 0;
+    }
+  }
+  return m;
+}
+
+__device__ __forceinline__ bool active(const Item& m, int s, int j) {
+  return j >= m.lo[s] && j <= m.hi[s];
+}
+
+// Rotate one landed 128x128 bf16 tile (two SW128 64-wide chunks) in place.
+// rows: global row index of tile row 0; lo_dst (x3 mode) receives the
+// bf16 residual of each rotated value.
+template <bool X3>
+__device__ __forceinline__ void rope_tile(uint8_t* tile, uint8_t* lo_dst,
+                                          const int32_t* __restrict__ pos,
+                                          const float2* __restrict__ table,
+                                          int64_t rowbase, int row0, int N,
+                                          int tid) {
+#pragma unroll 4
+  for (int it = 0; it < 16; ++it) {
+    int q = it * 128 + tid;
+    int r = q >> 4;
+    int cc = q & 15;
+    int sub = cc >> 3, lc = cc & 7;
+    int off = sub * kHalfTileBytes + r * 128 + ((lc ^ (r & 7)) << 4);
+    int grow = row0 + r;
+    if (grow >= N) {
+      if (X3) *reinterpret_cast<uint4*>(lo_dst + off) = make_uint4(0, 0, 0, 0);
+      continue;  // zero-filled by TMA; nothing to rotate
+    }
+    int p = pos[rowbase + grow];
+    const float4* cs = reinterpret_cast<const float4*>(
+        table + int64_t(p) * (kHeadDim / 2) + sub * 32 + lc * 4);
+    float4 c01 = __ldg(cs);
+    float4 c23 = __ldg(cs + 1);
+    uint4 w = *reinterpret_cast<uint4*>(tile + off);
+    float cc4[4] = {c01.x, c01.z, c23.x, c23.z};
+    float ss4[4] = {c01.y, c01.w, c23.y, c23.w};
+    uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    uint32_t hi_out[4], lo_out[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float a = bf16lo_to_f32(ws[e]);
+      float b = bf16hi_to_f32(ws[e]);
+      float ra = a * cc4[e] - b * ss4[e];
+      float rb = a * ss4[e] + b * cc4[e];
+      uint32_t h = pack_bf16x2(ra, rb);
+      hi_out[e] = h;
+      if (X3)
+        lo_out[e] = pack_bf16x2(ra - bf16lo_to_f32(h), rb - bf16hi_to_f32(h));
+    }
+    *reinterpret_cast<uint4*>(tile + off) =
+        make_uint4(hi_out[0], hi_out[1], hi_out[2], hi_out[3]);
+    if (X3)
+      *reinterpret_cast<uint4*>(lo_dst + off) =
+          make_uint4(lo_out[0], lo_out[1], lo_out[2], lo_out[3]);
+  }
+}
+
+template <bool X3>
+__global__ void __launch_bounds__(kThreadsFwd, 1)
+fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+              const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v,
+              const __grid_constant__ CUtensorMap tm_o,
+              const FwdParams p) {
+  using C = FwdCfg<X3>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bars = sbase + C::kBars;
+  auto bar = [&](int i) { return bars + 8u * i; };
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(C::bQFull + s), 1);
+      mbar_init(bar(C::bQReady + s), 4);
+      mbar_init(bar(C::bQEmpty + s), 1);
+      mbar_init(bar(C::bSFull + s), 1);
+      mbar_init(bar(C::bPFull + s), 4);
+      mbar_init(bar(C::bOFull + s), 1);
+      mbar_init(bar(C::bOEmpty + s), 4);
+      mbar_init(bar(C::bEpi + s), 128);
+    }
+    mbar_init(bar(C::bDone), 1);
+    for (int i = 0; i < C::KS; ++i) {
+      mbar_init(bar(C::bKFull + i), 1);
+      mbar_init(bar(C::bKReady + i), 4);
+      mbar_init(bar(C::bKEmpty + i), 1);
+    }
+    for (int i = 0; i < C::VS; ++i) {
+      mbar_init(bar(C::bVFull + i), 1);
+      mbar_init(bar(C::bVEmpty + i), 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 13) {
+    tmem_alloc(smem_u32(tmem_holder), 512);
+    tmem_relinquish();
+  }
+  if (warp == 12 && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_o);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int nitems = p.total_items;
+
+  if (warp == 12) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int qfill[2] = {0, 0};
+      int kfill = 0, vfill = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+        Item m = get_item(p, it);
+        for (int s = 0; s < 2 && ok; ++s) {
+          if (!m.present[s]) continue;
+          if (qfill[s] > 0)
+            ok = mbar_wait(bar(C::bQEmpty + s), (qfill[s] - 1) & 1,
+                           abort_flag, p.status, kWaitLimitNs);
+          if (!ok) break;
+          uint32_t dst = sbase + C::kQ + s * kTileBytes;
+          mbar_arrive_expect_tx(bar(C::bQFull + s), kTileBytes);
+          tma_load_4d(dst, &tm_q, bar(C::bQFull + s), 0, m.h,
+                      m.t[s] * kBlock, m.b);
+          tma_load_4d(dst + kHalfTileBytes, &tm_q, bar(C::bQFull + s), 64,
+                      m.h, m.t[s] * kBlock, m.b);
+          qfill[s]++;
+        }
+        for (int j = m.jhi; j >= m.jlo && ok; --j) {
+          int ks = kfill % C::KS;
+          if (kfill >= C::KS)
+            ok = mbar_wait(bar(C::bKEmpty + ks), ((kfill / C::KS) - 1) & 1,
+                           abort_flag, p.status, kWaitLimitNs);
+          if (!ok) break;
+          uint32_t kd = sbase + C::kK + ks * kTileBytes;
+          mbar_arrive_expect_tx(bar(C::bKFull + ks), kTileBytes);
+          tma_load_4d(kd, &tm_k, bar(C::bKFull + ks), 0, m.h, j * kBlock,
+                      m.b);
+          tma_load_4d(kd + kHalfTileBytes, &tm_k, bar(C::bKFull + ks), 64,
+                      m.h, j * kBlock, m.b);
+          kfill++;
+          int vs = vfill % C::VS;
+          if (vfill >= C::VS)
+            ok = mbar_wait(bar(C::bVEmpty + vs), ((vfill / C::VS) - 1) & 1,
+                           abort_flag, p.status, kWaitLimitNs);
+          if (!ok) break;
+          uint32_t vd = sbase + C::kV + vs * kTileBytes;
+          mbar_arrive_expect_tx(bar(C::bVFull + vs), kTileBytes);
+          tma_load_4d(vd, &tm_v, bar(C::bVFull + vs), 0, m.h, j * kBlock,
+                      m.b);
+          tma_load_4d(vd + kHalfTileBytes, &tm_v, bar(C::bVFull + vs), 64,
+                      m.h, j * kBlock, m.b);
+          vfill++;
+        }
+      }
+      // Drain: every armed load must land before the CTA may exit (on the
+      // normal path these phases have completed already).
+      for (int s = 0; s < 2; ++s)
+        if (qfill[s] > 0)
+          mbar_wait(bar(C::bQFull + s), (qfill[s] - 1) & 1, nullptr,
+                    p.status, kWaitLimitNs);
+      for (int f = kfill - 1; f >= 0 && f >= kfill - C::KS; --f)
+        mbar_wait(bar(C::bKFull + f % C::KS), (f / C::KS) & 1, nullptr,
+                  p.status, kWaitLimitNs);
+      for (int f = vfill - 1; f >= 0 && f >= vfill - C::VS; --f)
+        mbar_wait(bar(C::bVFull + f % C::VS), (f / C::VS) & 1, nullptr,
+                  p.status, kWaitLimitNs);
+    }
+  } else if (warp >= 8 && warp < 12) {
+    // ------------------------------------------------ RoPE rotation
+    const int tid = threadIdx.x - 8 * 32;
+    int qcount[2] = {0, 0};
+    int kcount = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+      Item m = get_item(p, it);
+      const int64_t rowbase = int64_t(m.b) * p.N;
+      for (int s = 0; s < 2 && ok; ++s) {
+        if (!m.present[s]) continue;
+        ok = mbar_wait(bar(C::bQFull + s), qcount[s] & 1, abort_flag,
+                       p.status, kWaitLimitNs);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        qcount[s]++;
+        rope_tile<X3>(smem + C::kQ + s * kTileBytes,
+                      smem + C::kQlo + s * kTileBytes, p.pos, p.table,
+                      rowbase, m.t[s] * kBlock, p.N, tid);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::bQReady + s));
+      }
+      for (int j = m.jhi; j >= m.jlo && ok; --j) {
+        int ks = kcount % C::KS;
+        ok = mbar_wait(bar(C::bKFull + ks), (kcount / C::KS) & 1, abort_flag,
+                       p.status, kWaitLimitNs);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        kcount++;
+        rope_tile<X3>(smem + C::kK + ks * kTileBytes,
+                      smem + C::kKlo + ks * kTileBytes, p.pos, p.table,
+                      rowbase, j * kBlock, p.N, tid);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::bKReady + ks));
+      }
+    }
+  } else if (warp == 13) {
+    // ------------------------------------------------ tcgen05 issuer
+    if (lane == 0) {
+      const uint32_t idS = idesc_bf16(128, 128, 0, 0);
+      const uint32_t idPV = idesc_bf16(128, 128, 0, 1);
+      int kc = 0, vc = 0;
+      int qc[2] = {0, 0}, pc[2] = {0, 0}, oc[2] = {0, 0};
+      bool ok = true;
+      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+        Item m = get_item(p, it);
+        bool qwaited[2] = {false, false};
+        bool pv_started[2] = {false, false};
+        int prev = -1;
+        for (int j = m.jhi; j >= m.jlo - 1 && ok; --j) {
+          const bool has_j = j >= m.jlo;
+          int ks = kc % C::KS;
+          if (has_j) {
+            ok = mbar_wait(bar(C::bKReady + ks), (kc / C::KS) & 1, abort_flag,
+                           p.status, kWaitLimitNs);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          int vs = vc % C::VS;
+          if (prev >= 0) {
+            ok = mbar_wait(bar(C::bVFull + vs), (vc / C::VS) & 1, abort_flag,
+                           p.status, kWaitLimitNs);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          for (int s = 0; s < 2 && ok; ++s) {
+            if (prev >= 0 && active(m, s, prev)) {
+              ok = mbar_wait(bar(C::bPFull + s), pc[s] & 1, abort_flag,
+                             p.status, kWaitLimitNs);
+              if (!ok) break;
+              pc[s]++;
+              if (!pv_started[s] && oc[s] > 0) {
+                ok = mbar_wait(bar(C::bOEmpty + s), (oc[s] - 1) & 1,
+                               abort_flag, p.status, kWaitLimitNs);
+                if (!ok) break;
+              }
+              tc_fence_after();
+              const uint32_t vbase = sbase + C::kV + vs * kTileBytes;
+              const uint32_t a_tm = tmem + s * 128;        // P over S_s
+              const uint32_t d_tm = tmem + 256 + s * 128;  // O_s
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                uint64_t bd = sdesc_sw128(vbase + k * 2048, kHalfTileBytes,
+                                          1024);
+                mma_ts(d_tm, a_tm + k * 8, bd, idPV,
+                       (pv_started[s] || k > 0) ? 1u : 0u);
+              }
+              pv_started[s] = true;
+            }
+            if (has_j && active(m, s, j)) {
+              if (!qwaited[s]) {
+                ok = mbar_wait(bar(C::bQReady + s), qc[s] & 1, abort_flag,
+                               p.status, kWaitLimitNs);
+                if (!ok) break;
+                qc[s]++;
+                qwaited[s] = true;
+                tc_fence_after();
+              }
+              const uint32_t qb = sbase + C::kQ + s * kTileBytes;
+              const uint32_t kb = sbase + C::kK + ks * kTileBytes;
+              const uint32_t d_tm = tmem + s * 128;
+              int step = 0;
+              const int npass = X3 ? 3 : 1;
+              for (int pass = 0; pass < npass; ++pass) {
+                // pass 0: hi.hi, 1: hi(Q).lo(K), 2: lo(Q).hi(K)
+                uint32_t qa = qb + (pass == 2 ? (C::kQlo - C::kQ) : 0);
+                uint32_t kbb = kb + (pass == 1 ? (C::kKlo - C::kK) : 0);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                  uint32_t off = (k >> 2) * kHalfTileBytes + (k & 3) * 32;
+                  uint64_t ad = sdesc_sw128(qa + off, 16, 1024);
+                  uint64_t bd = sdesc_sw128(kbb + off, 16, 1024);
+                  mma_ss(d_tm, ad, bd, idS, step > 0 ? 1u : 0u);
+                  ++step;
+                }
+              }
+              mma_commit(bar(C::bSFull + s));
+            }
+          }
+          if (!ok) break;
+          if (has_j) {
+            mma_commit(bar(C::bKEmpty + ks));
+            kc++;
+          }
+          if (prev >= 0) {
+            mma_commit(bar(C::bVEmpty + vs));
+            vc++;
+          }
+          prev = has_j ? j : -1;
+        }
+        if (!ok) break;
+        for (int s = 0; s < 2; ++s)
+          if (m.present[s]) {
+            mma_commit(bar(C::bOFull + s));
+            oc[s]++;
+          }
+      }
+      // every issued MMA must be complete before TMEM is released
+      mma_commit(bar(C::bDone));
+      mbar_wait(bar(C::bDone), 0, nullptr, p.status, kWaitLimitNs);
+    }
+  } else {
+    // ------------------------------------------------ softmax (warps 0-7)
+    const int s = warp >> 2;                 // query sub-tile
+    const int r = (warp & 3) * 32 + lane;    // row in the sub-tile = TMEM lane
+    const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + s * 128;
+    const uint32_t tO = tmem + lane_off + 256 + s * 128;
+    int sc = 0, oc = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+      Item m = get_item(p, it);
+      if (!m.present[s]) continue;
+      const int64_t rowbase = int64_t(m.b) * p.N;
+      const int q0 = m.t[s] * kBlock;
+      const int i = q0 + r;
+      const bool valid = i < p.N;
+      const int seg_i = valid ? __ldg(p.seg + rowbase + i) : 0;
+      const int q_last = q0 + kBlock - 1;
+      const int seg_qlast = q_last < p.N ? __ldg(p.seg + rowbase + q_last) : 0;
+      float m_used = -INFINITY, l = 0.f;
+      bool first = true;
+      for (int j = m.hi[s]; j >= m.lo[s] && ok; --j) {
+        ok = mbar_wait(bar(C::bSFull + s), sc & 1, abort_flag, p.status,
+                       kWaitLimitNs);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        sc++;
+        tc_fence_after();
+        const int k0 = j * kBlock;
+        const bool full = (k0 + kBlock - 1 < q0) && (q_last < p.N) &&
+                          (__ldg(p.seg + rowbase + k0) == seg_qlast);
+        // pass 1: row max of the raw scores
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tS + c * 32, v);
+          tmem_wait_ld();
+          if (full) {
+#pragma unroll
+            for (int x = 0; x < 32; ++x) mx = fmaxf(mx, __uint_as_float(v[x]));
+          } else {
+#pragma unroll 8
+            for (int x = 0; x < 32; ++x) {
+              int kj = k0 + c * 32 + x;
+              bool okk = valid && kj <= i && kj < p.N &&
+                         __ldg(p.seg + rowbase + kj) == seg_i;
+              if (okk) mx = fmaxf(mx, __uint_as_float(v[x]));
+            }
+          }
+        }
+        const float m_tile = mx * p.scale_log2;
+        float m_new = m_used;
+        bool rescale = false;
+        if (m_tile > m_used + kRescaleThreshold) {
+          m_new = m_tile;
+          rescale = true;
+        }
+        const float alpha = rescale ? ex2(m_used - m_new) : 1.f;
+        if (!first && __any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tO + c * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int x = 0; x < 32; ++x)
+              v[x] = __float_as_uint(__uint_as_float(v[x]) * alpha);
+            tmem_st32(tO + c * 32, v);
+          }
+        }
+        l *= alpha;
+        const float sub = m_new == -INFINITY ? 0.f : m_new;
+        // pass 2: P = 2^(S*c - m), row sum, bf16 P over S columns [0, 64)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tS + c * 32, v);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int x = 0; x < 32; x += 2) {
+            float s0 = __uint_as_float(v[x]) * p.scale_log2 - sub;
+            float s1 = __uint_as_float(v[x + 1]) * p.scale_log2 - sub;
+            if (!full) {
+              int kj = k0 + c * 32 + x;
+              bool ok0 = valid && kj <= i && kj < p.N &&
+                         __ldg(p.seg + rowbase + kj) == seg_i;
+              bool ok1 = valid && kj + 1 <= i && kj + 1 < p.N &&
+                         __ldg(p.seg + rowbase + kj + 1) == seg_i;
+              s0 = ok0 ? s0 : -INFINITY;
+              s1 = ok1 ? s1 : -INFINITY;
+            }
+            float p0 = ex2(s0), p1 = ex2(s1);
+            l += p0 + p1;
+            pk[x >> 1] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(tS + c * 16, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::bPFull + s));
+        m_used = m_new;
+        first = false;
+      }
+      if (!ok) break;
+      // ---------------------------------------------- epilogue
+      ok = mbar_wait(bar(C::bOFull + s), oc & 1, abort_flag, p.status,
+                     kWaitLimitNs);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      oc++;
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      uint8_t* stage = smem + C::kQ + s * kTileBytes;  // Q_s is free now
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tO + c * 32, v);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int x = 0; x < 32; x += 2)
+          pk[x >> 1] = pack_bf16x2(__uint_as_float(v[x]) * inv,
+                                   __uint_as_float(v[x + 1]) * inv);
+        // columns c*32 .. c*32+31 = d chunk (c>>1), 16-byte chunks
+        // (c&1)*4 .. +3 of that 128-byte row
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          int lc = (c & 1) * 4 + e;
+          int off = (c >> 1) * kHalfTileBytes + r * 128 + ((lc ^ (r & 7)) << 4);
+          *reinterpret_cast<uint4*>(stage + off) =
+              make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::bOEmpty + s));
+      fence_proxy_async_smem();
+      mbar_arrive(bar(C::bEpi + s));
+      if (r == 0 &&
+          mbar_wait(bar(C::bEpi + s), (oc - 1) & 1, abort_flag, p.status,
+                    kWaitLimitNs)) {
+        uint32_t src = sbase + C::kQ + s * kTileBytes;
+        tma_store_4d(&tm_o, src, 0, m.h, q0, m.b);
+        tma_store_4d(&tm_o, src + kHalfTileBytes, 64, m.h, q0, m.b);
+        bulk_commit();
+        bulk_wait_read0();
+        mbar_arrive(bar(C::bQEmpty + s));
+      }
+      if (valid)
+        p.lse[(int64_t(m.b) * p.H + m.h) * p.N + i] =
+            (m_used + __log2f(l)) * kLn2;
+    }
+    if (threadIdx.x == 0 || threadIdx.x == 128) bulk_wait0();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 13) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------ host side
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType,
+                                   cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f,
+                                cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+
+}  // namespace
+
+// [B][N][H][D] bf16 tensor as a 4-D map {D, H, N, B}; box 64 x 1 x 128 x 1
+// with the 128-byte swizzle (one 64-wide d chunk of 128 rows per copy).
+bool make_bnhd_map(CUtensorMap* m, const void* base, int B, int N, int H) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {cuuint64_t(kHeadDim), cuuint64_t(H), cuuint64_t(N),
+                        cuuint64_t(B)};
+  cuuint64_t strides[3] = {cuuint64_t(kHeadDim) * 2,
+                           cuuint64_t(H) * kHeadDim * 2,
+                           cuuint64_t(N) * H * kHeadDim * 2};
+  cuuint32_t box[4] = {64, 1, cuuint32_t(kBlock), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                   const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) !=
+      cudaSuccess)
+    return 148;
+  return n;
+}
+
+template <bool X3>
+static cudaError_t launch_fwd_impl(const FwdArgs& a, cudaStream_t st) {
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_bnhd_map(&mq, a.q, a.B, a.N, a.H) ||
+      !make_bnhd_map(&mk, a.k, a.B, a.N, a.H) ||
+      !make_bnhd_map(&mv, a.v, a.B, a.N, a.H) ||
+      !make_bnhd_map(&mo, a.out, a.B, a.N, a.H))
+    return cudaErrorInvalidValue;
+  FwdParams p{};
+  p.seg = a.seg;
+  p.pos = a.pos;
+  p.table = reinterpret_cast<const float2*>(a.table);
+  p.kv_lo = a.kv_lo;
+  p.kv_hi = a.kv_hi;
+  p.order = a.order;
+  p.lse = a.lse;
+  p.status = a.status;
+  p.B = a.B;
+  p.N = a.N;
+  p.H = a.H;
+  p.Tq = (a.N + kBlock - 1) / kBlock;
+  p.U = (p.Tq + kFwdBlocksPerUnit - 1) / kFwdBlocksPerUnit;
+  p.G = 1;
+  for (int g = 4; g >= 1; --g)
+    if (a.H % g == 0) { p.G = g; break; }
+  p.total_items = a.B * p.U * a.H;
+  p.scale_log2 = kLog2e / sqrtf(float(kHeadDim));
+  constexpr int smem = FwdCfg<X3>::kSmem;
+  cudaError_t e = cudaFuncSetAttribute(
+      fwd_tc_kernel<X3>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  int grid = std::min(sm_count(), p.total_items);
+  fwd_tc_kernel<X3><<<grid, kThreadsFwd, smem, st>>>(mq, mk, mv, mo, p);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t st) {
+  if (a.B == 0 || a.N == 0 || a.H == 0) return cudaSuccess;
+  return a.qk_x3 ? launch_fwd_impl<true>(a, st) : launch_fwd_impl<false>(a, st);
+}
+
+}  // namespace lwm
