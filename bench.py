@@ -257,8 +257,10 @@ def main():
     fwd_flop = 4.0 * D * pairs_per_head * H
     bwd_flop = 10.0 * D * pairs_per_head * H if w.backward else 0.0
     max_pos = int(t["positions"].max().item()) + 1
-    ws_bytes = max(ops.fwd_workspace_size(B, N, H, max_pos),
-                   ops.bwd_workspace_size(B, N, H, max_pos)
+    ws_bytes = max(ops.fwd_workspace_size(B, N, H, max_pos,
+                                          qk_precision=qkp),
+                   ops.bwd_workspace_size(B, N, H, max_pos,
+                                          qk_precision=qkp)
                    if w.backward else 0)
     workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     out = torch.empty_like(t["q"])

@@ -89,18 +89,24 @@ typedef enum { LWM_QK_BF16 = 0, LWM_QK_BF16X3 = 1 } lwm_qk_precision;
 /* Tile classes written by lwm_blockattn_classify. */
 enum { LWM_TILE_EMPTY = 0, LWM_TILE_PARTIAL = 1, LWM_TILE_FULL = 2 };
 
-/* Bytes of device workspace lwm_blockattn_fwd needs for these sizes
- * (RoPE cos/sin table of max_pos x D/2 float pairs, per-block segment
- * ranges, the work list). Returns 0 for invalid sizes. */
+/* Bytes of device workspace lwm_blockattn_fwd needs for these sizes,
+ * dtype and qk_precision: the RoPE cos/sin table (max_pos x D/2 float
+ * pairs), per-block and per-row segment metadata, the work order and, for
+ * LWM_DTYPE_BF16, the rotated keys R(pos) k (B*N*H*D bf16; twice that for
+ * LWM_QK_BF16X3, which keeps the bf16 residual too). Returns 0 for invalid
+ * sizes. */
 LWM_API size_t lwm_blockattn_fwd_workspace_size(int B, int N, int H, int D,
                                         int block_q, int block_k,
-                                        int max_pos);
+                                        int max_pos, int dtype,
+                                        int qk_precision);
 
 /* Same for lwm_blockattn_bwd: additionally an fp32 dQ accumulator of
- * B*N*H*D floats and the per-row dot(dO, O) of B*H*N floats. */
+ * B*N*H*D floats, the per-row dot(dO, O) of B*H*N floats and, for
+ * LWM_DTYPE_BF16, the rotated queries as well as keys. */
 LWM_API size_t lwm_blockattn_bwd_workspace_size(int B, int N, int H, int D,
                                         int block_q, int block_k,
-                                        int max_pos);
+                                        int max_pos, int dtype,
+                                        int qk_precision);
 
 /* Forward. Writes out [B][N][H][D] (dtype) and lse [B][H][N] (fp32,
  * natural log of the softmax denominator of the scaled scores).

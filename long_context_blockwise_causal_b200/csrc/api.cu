@@ -42,6 +42,7 @@ struct Workspace {
   float* table;          // [max_pos][D/2] float2
   int32_t* kv_lo;        // [B][Tq]
   int32_t* kv_hi;        // [B][Tq]
+  int32_t* row_start;    // [B][N] first row of each row's packed example
   uint64_t* sort_keys;   // [max(B*Uq, B*Uk)]
   int32_t* order_fwd;    // [B*Uq] units of kFwdRowsPerCta rows, longest first
   // backward only
@@ -50,11 +51,15 @@ struct Workspace {
   int32_t* order_bwd;    // [B*Uk]
   float* delta;          // [B][H][N]
   float* dq_acc;         // [B][N][H][D]
+  // bf16 path: rotated keys (and queries for the backward), [B][N][H][D]
+  void* k_rot;
+  void* k_rot_lo;        // split-QK mode only
+  void* q_rot;           // backward only
   size_t bytes;
 };
 
 Workspace carve(void* base, int B, int N, int H, int D, int max_pos,
-                bool backward) {
+                bool backward, int dtype, int qkp) {
   Carve c{static_cast<char*>(base)};
   Workspace w{};
   int Tq = (N + kBlock - 1) / kBlock;
@@ -64,6 +69,7 @@ Workspace carve(void* base, int B, int N, int H, int D, int max_pos,
   w.table = c.take<float>(size_t(max_pos) * D);
   w.kv_lo = c.take<int32_t>(size_t(B) * Tq);
   w.kv_hi = c.take<int32_t>(size_t(B) * Tq);
+  w.row_start = c.take<int32_t>(size_t(B) * N);
   w.sort_keys = c.take<uint64_t>(size_t(B) * (Uq > Uk ? Uq : Uk));
   w.order_fwd = c.take<int32_t>(size_t(B) * Uq);
   if (backward) {
@@ -72,6 +78,13 @@ Workspace carve(void* base, int B, int N, int H, int D, int max_pos,
     w.order_bwd = c.take<int32_t>(size_t(B) * Uk);
     w.delta = c.take<float>(size_t(B) * H * N);
     w.dq_acc = c.take<float>(size_t(B) * N * H * D);
+  }
+  if (dtype == LWM_DTYPE_BF16) {
+    const size_t elems = size_t(B) * N * H * D;
+    w.k_rot = c.take<uint16_t>(elems);
+    if (qkp == LWM_QK_BF16X3 && !backward)
+      w.k_rot_lo = c.take<uint16_t>(elems);
+    if (backward) w.q_rot = c.take<uint16_t>(elems);
   }
   w.bytes = c.off;
   return w;
@@ -112,6 +125,7 @@ int prepare(const int32_t* seg, double theta, int B, int N, int D,
             int max_pos, const Workspace& w, cudaStream_t st) {
   LWM_TRY(launch_rope_table(theta, D, max_pos, w.table, st));
   LWM_TRY(launch_block_meta(seg, B, N, kBlock, kBlock, w.kv_lo, w.kv_hi, st));
+  LWM_TRY(launch_row_start(seg, B, N, w.row_start, st));
   return LWM_OK;
 }
 
@@ -143,16 +157,20 @@ uint64_t lwm_blockattn_kernel_launches(void) {
 
 size_t lwm_blockattn_fwd_workspace_size(int B, int N, int H, int D,
                                         int block_q, int block_k,
-                                        int max_pos) {
+                                        int max_pos, int dtype,
+                                        int qk_precision) {
   if (!sizes_ok(B, N, H, D, block_q, block_k, max_pos)) return 0;
-  return carve(nullptr, B, N, H, D, max_pos, false).bytes;
+  return carve(nullptr, B, N, H, D, max_pos, false, dtype, qk_precision)
+      .bytes;
 }
 
 size_t lwm_blockattn_bwd_workspace_size(int B, int N, int H, int D,
                                         int block_q, int block_k,
-                                        int max_pos) {
+                                        int max_pos, int dtype,
+                                        int qk_precision) {
   if (!sizes_ok(B, N, H, D, block_q, block_k, max_pos)) return 0;
-  return carve(nullptr, B, N, H, D, max_pos, true).bytes;
+  return carve(nullptr, B, N, H, D, max_pos, true, dtype, qk_precision)
+      .bytes;
 }
 
 int lwm_blockattn_fwd(const void* q, const void* k, const void* v,
@@ -175,7 +193,8 @@ int lwm_blockattn_fwd(const void* q, const void* k, const void* v,
   const void* ptrs[] = {q, k, v, segment_ids, positions, out, lse, workspace};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return LWM_ERR_INVALID_ARG;
-  Workspace w = carve(workspace, B, N, H, D, max_pos, false);
+  Workspace w = carve(workspace, B, N, H, D, max_pos, false, dtype,
+                      qk_precision);
   if (workspace_bytes < w.bytes) return LWM_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   s = prepare(segment_ids, theta, B, N, D, max_pos, w, st);
@@ -190,8 +209,13 @@ int lwm_blockattn_fwd(const void* q, const void* k, const void* v,
   a.q = q; a.k = k; a.v = v; a.out = out; a.lse = lse;
   a.seg = segment_ids; a.pos = positions; a.table = w.table;
   a.kv_lo = w.kv_lo; a.kv_hi = w.kv_hi; a.order = w.order_fwd;
+  a.row_start = w.row_start;
+  a.k_rot = w.k_rot; a.k_rot_lo = w.k_rot_lo;
   a.B = B; a.N = N; a.H = H;
   a.qk_x3 = qk_precision == LWM_QK_BF16X3;
+  // keys are reused by every query block that sees them: rotate them once
+  LWM_TRY(launch_rope_apply(k, positions, w.table, B, N, H, w.k_rot,
+                            w.k_rot_lo, st));
   a.status = status_word();
   if (!a.status) return LWM_ERR_CUDA;
   LWM_TRY(launch_lpt_order(B, (N + kBlock - 1) / kBlock, kFwdBlocksPerUnit,
@@ -221,7 +245,8 @@ int lwm_blockattn_bwd(const void* q, const void* k, const void* v,
                         dq, dk, dv, workspace};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return LWM_ERR_INVALID_ARG;
-  Workspace w = carve(workspace, B, N, H, D, max_pos, true);
+  Workspace w = carve(workspace, B, N, H, D, max_pos, true, dtype,
+                      qk_precision);
   if (workspace_bytes < w.bytes) return LWM_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   s = prepare(segment_ids, theta, B, N, D, max_pos, w, st);
@@ -264,7 +289,9 @@ int lwm_blockattn_bwd(const void* q, const void* k, const void* v,
     a.q = q; a.k = k; a.v = v; a.dout = dout; a.lse = lse; a.delta = w.delta;
     a.seg = segment_ids; a.pos = positions; a.table = w.table;
     a.q_lo = w.q_lo; a.q_hi = w.q_hi; a.order = w.order_bwd;
+    a.row_start = w.row_start;
     a.dq_acc = w.dq_acc; a.dk = dk; a.dv = dv;
+    a.q_rot = w.q_rot; a.k_rot = w.k_rot;
     a.B = B; a.N = N; a.H = H;
     a.status = status_word();
     if (!a.status) return LWM_ERR_CUDA;

@@ -23,6 +23,42 @@ __global__ void rope_table_kernel(double theta, int half_d, int max_pos,
   }
 }
 
+// hi = R(pos) x rounded to bf16 (RNE); lo (when given) = the bf16 rounding
+// of what hi misses, so hi + lo carries the rotated value to ~2^-16. One
+// thread per 16-byte chunk (4 interleaved pairs) of a [B][N][H][D] tensor.
+__global__ void rope_apply_kernel(const __nv_bfloat16* __restrict__ x,
+                                  const int32_t* __restrict__ pos,
+                                  const float2* __restrict__ table,
+                                  int64_t chunks, int H,
+                                  __nv_bfloat16* __restrict__ hi,
+                                  __nv_bfloat16* __restrict__ lo) {
+  constexpr int kChunksPerRow = kHeadDim / 8;
+  for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+       e < chunks; e += int64_t(gridDim.x) * blockDim.x) {
+    const int c = int(e % kChunksPerRow);
+    const int64_t bn = (e / kChunksPerRow) / H;
+    const int p = pos[bn];
+    const float4* t = reinterpret_cast<const float4*>(
+        table + int64_t(p) * (kHeadDim / 2) + c * 4);
+    const float4 cs01 = __ldg(t), cs23 = __ldg(t + 1);
+    const uint4 w = reinterpret_cast<const uint4*>(x)[e];
+    const float cc[4] = {cs01.x, cs01.z, cs23.x, cs23.z};
+    const float ss[4] = {cs01.y, cs01.w, cs23.y, cs23.w};
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float a = bf16lo_to_f32(ws[k]), b = bf16hi_to_f32(ws[k]);
+      const float ra = fmaf(a, cc[k], -b * ss[k]);
+      const float rb = fmaf(a, ss[k], b * cc[k]);
+      h[k] = pack_bf16x2(ra, rb);
+      l[k] = pack_bf16x2(ra - bf16lo_to_f32(h[k]), rb - bf16hi_to_f32(h[k]));
+    }
+    reinterpret_cast<uint4*>(hi)[e] = make_uint4(h[0], h[1], h[2], h[3]);
+    if (lo) reinterpret_cast<uint4*>(lo)[e] = make_uint4(l[0], l[1], l[2], l[3]);
+  }
+}
+
 // First index of the contiguous run holding row i (ids non-decreasing).
 __device__ __forceinline__ int run_start(const int32_t* __restrict__ seg,
                                          int i) {
@@ -33,6 +69,19 @@ __device__ __forceinline__ int run_start(const int32_t* __restrict__ seg,
     if (seg[mid] < v) lo = mid + 1; else hi = mid;
   }
   return lo;
+}
+
+// rs[b][i] = first index of the packed example holding row i. With
+// non-decreasing ids, "seg_j == seg_i and j <= i" is "rs[i] <= j <= i".
+__global__ void row_start_kernel(const int32_t* __restrict__ seg, int B, int N,
+                                 int32_t* __restrict__ rs) {
+  int64_t total = int64_t(B) * N;
+  for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < total;
+       e += int64_t(gridDim.x) * blockDim.x) {
+    int b = int(e / N);
+    int i = int(e - int64_t(b) * N);
+    rs[e] = run_start(seg + int64_t(b) * N, i);
+  }
 }
 
 __global__ void block_meta_kernel(const int32_t* __restrict__ seg, int B,
@@ -248,6 +297,28 @@ cudaError_t launch_block_meta(const int32_t* seg, int B, int N, int bq, int bk,
   if (n == 0) return cudaSuccess;
   block_meta_kernel<<<(n + 255) / 256, 256, 0, st>>>(seg, B, N, bq, bk, Tq,
                                                       kv_lo, kv_hi);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_apply(const void* x, const int32_t* pos,
+                              const float* table, int B, int N, int H,
+                              void* hi, void* lo, cudaStream_t st) {
+  int64_t chunks = int64_t(B) * N * H * (kHeadDim / 8);
+  if (chunks == 0) return cudaSuccess;
+  rope_apply_kernel<<<grid_for(chunks, 256, 148 * 16), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(x), pos,
+      reinterpret_cast<const float2*>(table), chunks, H,
+      static_cast<__nv_bfloat16*>(hi), static_cast<__nv_bfloat16*>(lo));
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_row_start(const int32_t* seg, int B, int N, int32_t* rs,
+                             cudaStream_t st) {
+  int64_t n = int64_t(B) * N;
+  if (n == 0) return cudaSuccess;
+  row_start_kernel<<<grid_for(n, 256, 148 * 16), 256, 0, st>>>(seg, B, N, rs);
   note_launch();
   return cudaGetLastError();
 }

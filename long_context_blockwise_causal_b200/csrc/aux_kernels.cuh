@@ -11,6 +11,12 @@ cudaError_t launch_rope_table(double theta, int D, int max_pos, float* table,
                               cudaStream_t st);
 cudaError_t launch_block_meta(const int32_t* seg, int B, int N, int bq, int bk,
                               int32_t* kv_lo, int32_t* kv_hi, cudaStream_t st);
+// hi = R(pos) x in bf16, lo = residual (skipped when lo == nullptr).
+cudaError_t launch_rope_apply(const void* x, const int32_t* pos,
+                              const float* table, int B, int N, int H,
+                              void* hi, void* lo, cudaStream_t st);
+cudaError_t launch_row_start(const int32_t* seg, int B, int N, int32_t* rs,
+                             cudaStream_t st);
 cudaError_t launch_tile_class(const int32_t* seg, int B, int N, int bq, int bk,
                               const int32_t* kv_lo, const int32_t* kv_hi,
                               uint8_t* cls, cudaStream_t st);

@@ -6,16 +6,20 @@
 // holding their diagonal down to the start of their packed example, keeping
 // a running max, a running sum and an output accumulator (online softmax);
 // RoPE ("[论文解读] World Model on Million-Length Video And Language With
-// Blockwise RingAttention", 提出的方法) is applied to the Q and K tiles in
-// shared memory right after they land.
+// Blockwise RingAttention", 提出的方法) is applied to each Q tile in shared
+// memory right after it lands. Keys are rotated once per token by a
+// separate pass (each key block is read by every query block that sees it,
+// so rotating it in the loader would repeat the work O(N/128) times).
 //
 // CTA = persistent worker over units of 2 x 128 query rows of one (b, h):
 //   warps 0-3   softmax for query sub-tile 0 (TMEM lanes 0-127)
 //   warps 4-7   softmax for query sub-tile 1
-//   warps 8-11  RoPE: rotate each landed Q / K tile in place (fp32 math,
+//   warps 8-11  RoPE: rotate each landed Q tile in place (fp32 math,
 //               bf16 round to nearest even; hi/lo split in the x3 mode)
-//   warp 12     TMA producer (Q per unit, K and V per key block)
+//   warp 12     TMA producer (Q per unit, rotated K and V per key block)
 //   warp 13     tcgen05 issuer (one elected lane) + TMEM owner
+//   warps 14-15 idle (they complete the fourth warpgroup, which setmaxnreg
+//               needs; their registers go to the softmax warps)
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; P (bf16)
 // is written over the first 64 columns of S and read from there by the
 // P.V MMA. O is rescaled in TMEM only when a row max grows by more than
@@ -28,7 +32,12 @@
 namespace lwm {
 namespace {
 
-constexpr int kThreadsFwd = 14 * 32;
+constexpr int kThreadsFwd = 16 * 32;
+// Register budget per warpgroup after setmaxnreg (launch: 128 each). The
+// four groups share each SM sub-partition, so the sum must stay 4 x 128.
+constexpr int kRegsSoftmax = 176, kRegsRope = 96, kRegsMisc = 64;
+static_assert(2 * kRegsSoftmax + kRegsRope + kRegsMisc == 4 * 128,
+              "register split must equal the launch allocation");
 constexpr int kTileBytes = kBlock * kHeadDim * 2;       // 32 KB bf16 tile
 constexpr int kHalfTileBytes = kTileBytes / 2;          // one 64-wide d chunk
 constexpr uint64_t kWaitLimitNs = 4000000000ull;        // 4 s per wait
@@ -47,8 +56,7 @@ struct FwdCfg {
   // barrier slots
   static constexpr int bQFull = 0, bQReady = 2, bQEmpty = 4, bSFull = 6,
                        bPFull = 8, bOFull = 10, bOEmpty = 12, bEpi = 14,
-                       bDone = 16, bKFull = 17,
-                       bKReady = bKFull + KS, bKEmpty = bKReady + KS,
+                       bDone = 16, bKFull = 17, bKEmpty = bKFull + KS,
                        bVFull = bKEmpty + KS, bVEmpty = bVFull + VS,
                        kNumBars = bVEmpty + VS;
   static constexpr int kMisc = kBars + kNumBars * 8;
@@ -57,6 +65,7 @@ struct FwdCfg {
 
 struct FwdParams {
   const int32_t* seg;
+  const int32_t* row_start;
   const int32_t* pos;
   const float2* table;
   const int32_t* kv_lo;
@@ -110,54 +119,78 @@ __device__ __forceinline__ bool active(const Item& m, int s, int j) {
   return j >= m.lo[s] && j <= m.hi[s];
 }
 
-// Rotate one landed 128x128 bf16 tile (two SW128 64-wide chunks) in place.
-// rows: global row index of tile row 0; lo_dst (x3 mode) receives the
-// bf16 residual of each rotated value.
+// RoPE of one row of a landed 128x128 bf16 tile (two SW128 64-wide d
+// chunks), in place. Thread r owns row r: its 16 chunks sit at distinct
+// swizzled 16-byte slots of its 128-byte rows, so a quarter-warp touches
+// 8 different slots (no bank conflicts). The row's 64 (cos, sin) pairs are
+// read in quarters of 16 pairs; cs holds the first quarter, loaded by the
+// caller ahead of the barrier wait. lo_dst (x3 mode) receives the bf16
+// residual of each rotated value.
 template <bool X3>
-__device__ __forceinline__ void rope_tile(uint8_t* tile, uint8_t* lo_dst,
-                                          const int32_t* __restrict__ pos,
-                                          const float2* __restrict__ table,
-                                          int64_t rowbase, int row0, int N,
-                                          int tid) {
-#pragma unroll 4
-  for (int it = 0; it < 16; ++it) {
-    int q = it * 128 + tid;
-    int r = q >> 4;
-    int cc = q & 15;
-    int sub = cc >> 3, lc = cc & 7;
-    int off = sub * kHalfTileBytes + r * 128 + ((lc ^ (r & 7)) << 4);
-    int grow = row0 + r;
-    if (grow >= N) {
-      if (X3) *reinterpret_cast<uint4*>(lo_dst + off) = make_uint4(0, 0, 0, 0);
-      continue;  // zero-filled by TMA; nothing to rotate
-    }
-    int p = pos[rowbase + grow];
-    const float4* cs = reinterpret_cast<const float4*>(
-        table + int64_t(p) * (kHeadDim / 2) + sub * 32 + lc * 4);
-    float4 c01 = __ldg(cs);
-    float4 c23 = __ldg(cs + 1);
-    uint4 w = *reinterpret_cast<uint4*>(tile + off);
-    float cc4[4] = {c01.x, c01.z, c23.x, c23.z};
-    float ss4[4] = {c01.y, c01.w, c23.y, c23.w};
-    uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-    uint32_t hi_out[4], lo_out[4];
+__device__ __forceinline__ void rope_row(uint8_t* tile, uint8_t* lo_dst,
+                                         const float4* __restrict__ trow,
+                                         float4 (&cs)[8], int r, bool valid) {
+  if (!valid) {
+    if (X3) {
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      float a = bf16lo_to_f32(ws[e]);
-      float b = bf16hi_to_f32(ws[e]);
-      float ra = a * cc4[e] - b * ss4[e];
-      float rb = a * ss4[e] + b * cc4[e];
-      uint32_t h = pack_bf16x2(ra, rb);
-      hi_out[e] = h;
-      if (X3)
-        lo_out[e] = pack_bf16x2(ra - bf16lo_to_f32(h), rb - bf16hi_to_f32(h));
+      for (int c = 0; c < 16; ++c)
+        *reinterpret_cast<uint4*>(lo_dst + (c >> 3) * kHalfTileBytes +
+                                  r * 128 + (((c & 7) ^ (r & 7)) << 4)) =
+            make_uint4(0, 0, 0, 0);
     }
-    *reinterpret_cast<uint4*>(tile + off) =
-        make_uint4(hi_out[0], hi_out[1], hi_out[2], hi_out[3]);
-    if (X3)
-      *reinterpret_cast<uint4*>(lo_dst + off) =
-          make_uint4(lo_out[0], lo_out[1], lo_out[2], lo_out[3]);
+    return;  // zero-filled by TMA; nothing to rotate
   }
+#pragma unroll
+  for (int qt = 0; qt < 4; ++qt) {
+    if (qt > 0) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) cs[e] = __ldg(trow + qt * 8 + e);
+    }
+#pragma unroll
+    for (int cl = 0; cl < 4; ++cl) {
+      const int lc = (qt & 1) * 4 + cl;
+      const int off =
+          (qt >> 1) * kHalfTileBytes + r * 128 + ((lc ^ (r & 7)) << 4);
+      uint4 w = *reinterpret_cast<uint4*>(tile + off);
+      const float c4[4] = {cs[2 * cl].x, cs[2 * cl].z, cs[2 * cl + 1].x,
+                           cs[2 * cl + 1].z};
+      const float s4[4] = {cs[2 * cl].y, cs[2 * cl].w, cs[2 * cl + 1].y,
+                           cs[2 * cl + 1].w};
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+      uint32_t hi_out[4], lo_out[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float a = bf16lo_to_f32(ws[e]);
+        const float b = bf16hi_to_f32(ws[e]);
+        const float ra = fmaf(a, c4[e], -b * s4[e]);
+        const float rb = fmaf(a, s4[e], b * c4[e]);
+        const uint32_t h = pack_bf16x2(ra, rb);
+        hi_out[e] = h;
+        if (X3)
+          lo_out[e] = pack_bf16x2(ra - bf16lo_to_f32(h), rb - bf16hi_to_f32(h));
+      }
+      *reinterpret_cast<uint4*>(tile + off) =
+          make_uint4(hi_out[0], hi_out[1], hi_out[2], hi_out[3]);
+      if (X3)
+        *reinterpret_cast<uint4*>(lo_dst + off) =
+            make_uint4(lo_out[0], lo_out[1], lo_out[2], lo_out[3]);
+    }
+  }
+}
+
+// Loads (position, first quarter of cos/sin) of tile row r before the wait.
+__device__ __forceinline__ const float4* rope_prefetch(
+    const int32_t* __restrict__ pos, const float2* __restrict__ table,
+    int64_t rowbase, int grow, int N, float4 (&cs)[8], bool& valid) {
+  valid = grow < N;
+  const float4* trow = nullptr;
+  if (valid) {
+    const int pp = __ldg(pos + rowbase + grow);
+    trow = reinterpret_cast<const float4*>(table + int64_t(pp) * (kHeadDim / 2));
+#pragma unroll
+    for (int e = 0; e < 8; ++e) cs[e] = __ldg(trow + e);
+  }
+  return trow;
 }
 
 template <bool X3>
@@ -166,6 +199,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
               const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v,
               const __grid_constant__ CUtensorMap tm_o,
+              const __grid_constant__ CUtensorMap tm_klo,
               const FwdParams p) {
   using C = FwdCfg<X3>;
   extern __shared__ uint8_t smem_raw[];
@@ -194,7 +228,6 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(bar(C::bDone), 1);
     for (int i = 0; i < C::KS; ++i) {
       mbar_init(bar(C::bKFull + i), 1);
-      mbar_init(bar(C::bKReady + i), 4);
       mbar_init(bar(C::bKEmpty + i), 1);
     }
     for (int i = 0; i < C::VS; ++i) {
@@ -213,6 +246,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
     prefetch_tmap(&tm_o);
+    if (X3) prefetch_tmap(&tm_klo);
   }
   tc_fence_before();
   __syncthreads();
@@ -222,6 +256,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   if (warp == 12) {
     // ------------------------------------------------ TMA producer
+    regs_dec<kRegsMisc>();
     if (lane == 0) {
       int qfill[2] = {0, 0};
       int kfill = 0, vfill = 0;
@@ -249,11 +284,19 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                            abort_flag, p.status, kWaitLimitNs);
           if (!ok) break;
           uint32_t kd = sbase + C::kK + ks * kTileBytes;
-          mbar_arrive_expect_tx(bar(C::bKFull + ks), kTileBytes);
+          mbar_arrive_expect_tx(bar(C::bKFull + ks),
+                                X3 ? 2 * kTileBytes : kTileBytes);
           tma_load_4d(kd, &tm_k, bar(C::bKFull + ks), 0, m.h, j * kBlock,
                       m.b);
           tma_load_4d(kd + kHalfTileBytes, &tm_k, bar(C::bKFull + ks), 64,
                       m.h, j * kBlock, m.b);
+          if (X3) {
+            uint32_t kl = sbase + C::kKlo + ks * kTileBytes;
+            tma_load_4d(kl, &tm_klo, bar(C::bKFull + ks), 0, m.h,
+                        j * kBlock, m.b);
+            tma_load_4d(kl + kHalfTileBytes, &tm_klo, bar(C::bKFull + ks),
+                        64, m.h, j * kBlock, m.b);
+          }
           kfill++;
           int vs = vfill % C::VS;
           if (vfill >= C::VS)
@@ -284,44 +327,35 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
   } else if (warp >= 8 && warp < 12) {
     // ------------------------------------------------ RoPE rotation
-    const int tid = threadIdx.x - 8 * 32;
+    regs_dec<kRegsRope>();
+    const int r = threadIdx.x - 8 * 32;  // tile row owned by this thread
     int qcount[2] = {0, 0};
-    int kcount = 0;
     bool ok = true;
     for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
       Item m = get_item(p, it);
       const int64_t rowbase = int64_t(m.b) * p.N;
       for (int s = 0; s < 2 && ok; ++s) {
         if (!m.present[s]) continue;
+        float4 cs0[8];
+        bool valid;
+        const float4* trow = rope_prefetch(p.pos, p.table, rowbase,
+                                           m.t[s] * kBlock + r, p.N, cs0,
+                                           valid);
         ok = mbar_wait(bar(C::bQFull + s), qcount[s] & 1, abort_flag,
                        p.status, kWaitLimitNs);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         qcount[s]++;
-        rope_tile<X3>(smem + C::kQ + s * kTileBytes,
-                      smem + C::kQlo + s * kTileBytes, p.pos, p.table,
-                      rowbase, m.t[s] * kBlock, p.N, tid);
+        rope_row<X3>(smem + C::kQ + s * kTileBytes,
+                     smem + C::kQlo + s * kTileBytes, trow, cs0, r, valid);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(C::bQReady + s));
       }
-      for (int j = m.jhi; j >= m.jlo && ok; --j) {
-        int ks = kcount % C::KS;
-        ok = mbar_wait(bar(C::bKFull + ks), (kcount / C::KS) & 1, abort_flag,
-                       p.status, kWaitLimitNs);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        kcount++;
-        rope_tile<X3>(smem + C::kK + ks * kTileBytes,
-                      smem + C::kKlo + ks * kTileBytes, p.pos, p.table,
-                      rowbase, j * kBlock, p.N, tid);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(C::bKReady + ks));
-      }
     }
   } else if (warp == 13) {
     // ------------------------------------------------ tcgen05 issuer
+    regs_dec<kRegsMisc>();
     if (lane == 0) {
       const uint32_t idS = idesc_bf16(128, 128, 0, 0);
       const uint32_t idPV = idesc_bf16(128, 128, 0, 1);
@@ -337,7 +371,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           const bool has_j = j >= m.jlo;
           int ks = kc % C::KS;
           if (has_j) {
-            ok = mbar_wait(bar(C::bKReady + ks), (kc / C::KS) & 1, abort_flag,
+            ok = mbar_wait(bar(C::bKFull + ks), (kc / C::KS) & 1, abort_flag,
                            p.status, kWaitLimitNs);
             if (!ok) break;
             tc_fence_after();
@@ -425,8 +459,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       mma_commit(bar(C::bDone));
       mbar_wait(bar(C::bDone), 0, nullptr, p.status, kWaitLimitNs);
     }
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------ softmax (warps 0-7)
+    regs_inc<kRegsSoftmax>();
     const int s = warp >> 2;                 // query sub-tile
     const int r = (warp & 3) * 32 + lane;    // row in the sub-tile = TMEM lane
     const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
@@ -441,9 +476,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       const int q0 = m.t[s] * kBlock;
       const int i = q0 + r;
       const bool valid = i < p.N;
-      const int seg_i = valid ? __ldg(p.seg + rowbase + i) : 0;
+      // allowed keys of row i: rs_i <= kj <= hi_i (empty for rows >= N)
+      const int rs_i = valid ? __ldg(p.row_start + rowbase + i) : 0;
+      const int hi_i = valid ? i : -1;
       const int q_last = q0 + kBlock - 1;
-      const int seg_qlast = q_last < p.N ? __ldg(p.seg + rowbase + q_last) : 0;
+      const int rs_last = q_last < p.N ? __ldg(p.row_start + rowbase + q_last)
+                                       : 0x7fffffff;
       float m_used = -INFINITY, l = 0.f;
       bool first = true;
       for (int j = m.hi[s]; j >= m.lo[s] && ok; --j) {
@@ -454,28 +492,35 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         sc++;
         tc_fence_after();
         const int k0 = j * kBlock;
-        const bool full = (k0 + kBlock - 1 < q0) && (q_last < p.N) &&
-                          (__ldg(p.seg + rowbase + k0) == seg_qlast);
-        // pass 1: row max of the raw scores
-        float mx = -INFINITY;
+        // every pair of the tile allowed: keys end before the first query,
+        // all queries valid, and the last query's example starts at or
+        // before the first key
+        const bool full = (k0 + kBlock - 1 < q0) && (k0 >= rs_last);
+        // the whole 128-column S row of this thread in registers
+        uint32_t v[4][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tS + c * 32, v);
-          tmem_wait_ld();
-          if (full) {
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, v[c]);
+        tmem_wait_ld();
+        if (!full) {  // mask: keep rs_i <= key <= hi_i
 #pragma unroll
-            for (int x = 0; x < 32; ++x) mx = fmaxf(mx, __uint_as_float(v[x]));
-          } else {
-#pragma unroll 8
-            for (int x = 0; x < 32; ++x) {
-              int kj = k0 + c * 32 + x;
-              bool okk = valid && kj <= i && kj < p.N &&
-                         __ldg(p.seg + rowbase + kj) == seg_i;
-              if (okk) mx = fmaxf(mx, __uint_as_float(v[x]));
-            }
+          for (int c = 0; c < 4; ++c) {
+            const int lo = rs_i - (k0 + c * 32), hi = hi_i - (k0 + c * 32);
+#pragma unroll
+            for (int x = 0; x < 32; ++x)
+              v[c][x] = (x >= lo && x <= hi) ? v[c][x] : 0xff800000u;
           }
         }
+        float mc[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          mc[c] = __uint_as_float(v[c][0]);
+#pragma unroll
+          for (int x = 1; x < 31; x += 2)
+            mc[c] = max3(mc[c], __uint_as_float(v[c][x]),
+                         __uint_as_float(v[c][x + 1]));
+          mc[c] = fmaxf(mc[c], __uint_as_float(v[c][31]));
+        }
+        const float mx = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
         const float m_tile = mx * p.scale_log2;
         float m_new = m_used;
         bool rescale = false;
@@ -484,45 +529,41 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           rescale = true;
         }
         const float alpha = rescale ? ex2(m_used - m_new) : 1.f;
-        if (!first && __any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t v[32];
-            tmem_ld32(tO + c * 32, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int x = 0; x < 32; ++x)
-              v[x] = __float_as_uint(__uint_as_float(v[x]) * alpha);
-            tmem_st32(tO + c * 32, v);
-          }
-        }
         l *= alpha;
         const float sub = m_new == -INFINITY ? 0.f : m_new;
-        // pass 2: P = 2^(S*c - m), row sum, bf16 P over S columns [0, 64)
+        // P = 2^(S*c - m) (bf16, over S columns [0, 64)), row sum in fp32
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+        const float2 nsub2 = make_float2(-sub, -sub);
+        float2 lsum = make_float2(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tS + c * 32, v);
-          tmem_wait_ld();
           uint32_t pk[16];
 #pragma unroll
           for (int x = 0; x < 32; x += 2) {
-            float s0 = __uint_as_float(v[x]) * p.scale_log2 - sub;
-            float s1 = __uint_as_float(v[x + 1]) * p.scale_log2 - sub;
-            if (!full) {
-              int kj = k0 + c * 32 + x;
-              bool ok0 = valid && kj <= i && kj < p.N &&
-                         __ldg(p.seg + rowbase + kj) == seg_i;
-              bool ok1 = valid && kj + 1 <= i && kj + 1 < p.N &&
-                         __ldg(p.seg + rowbase + kj + 1) == seg_i;
-              s0 = ok0 ? s0 : -INFINITY;
-              s1 = ok1 ? s1 : -INFINITY;
-            }
-            float p0 = ex2(s0), p1 = ex2(s1);
-            l += p0 + p1;
+            const float2 t = fma2(make_float2(__uint_as_float(v[c][x]),
+                                              __uint_as_float(v[c][x + 1])),
+                                  sc2, nsub2);
+            const float p0 = ex2(t.x), p1 = ex2(t.y);
+            lsum = add2(lsum, make_float2(p0, p1));
             pk[x >> 1] = pack_bf16x2(p0, p1);
           }
           tmem_st16(tS + c * 16, pk);
+        }
+        l += lsum.x + lsum.y;
+        // O holds every P.V issued so far for this row (the S MMA this
+        // tile waited on was issued after them); rescale it when the max
+        // moved past the threshold
+        if (!first && __any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + c * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int x = 0; x < 32; ++x)
+              o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+            tmem_st32(tO + c * 32, o);
+          }
         }
         tmem_wait_st();
         tc_fence_before();
@@ -581,6 +622,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             (m_used + __log2f(l)) * kLn2;
     }
     if (threadIdx.x == 0 || threadIdx.x == 128) bulk_wait0();
+  } else {
+    regs_dec<kRegsMisc>();  // warps 14-15: no role
   }
 
   tc_fence_before();
@@ -647,14 +690,16 @@ int sm_count() {
 
 template <bool X3>
 static cudaError_t launch_fwd_impl(const FwdArgs& a, cudaStream_t st) {
-  CUtensorMap mq, mk, mv, mo;
+  CUtensorMap mq, mk, mv, mo, mklo;
   if (!make_bnhd_map(&mq, a.q, a.B, a.N, a.H) ||
-      !make_bnhd_map(&mk, a.k, a.B, a.N, a.H) ||
+      !make_bnhd_map(&mk, a.k_rot, a.B, a.N, a.H) ||
       !make_bnhd_map(&mv, a.v, a.B, a.N, a.H) ||
-      !make_bnhd_map(&mo, a.out, a.B, a.N, a.H))
+      !make_bnhd_map(&mo, a.out, a.B, a.N, a.H) ||
+      !make_bnhd_map(&mklo, X3 ? a.k_rot_lo : a.k_rot, a.B, a.N, a.H))
     return cudaErrorInvalidValue;
   FwdParams p{};
   p.seg = a.seg;
+  p.row_start = a.row_start;
   p.pos = a.pos;
   p.table = reinterpret_cast<const float2*>(a.table);
   p.kv_lo = a.kv_lo;
@@ -673,11 +718,19 @@ static cudaError_t launch_fwd_impl(const FwdArgs& a, cudaStream_t st) {
   p.total_items = a.B * p.U * a.H;
   p.scale_log2 = kLog2e / sqrtf(float(kHeadDim));
   constexpr int smem = FwdCfg<X3>::kSmem;
-  cudaError_t e = cudaFuncSetAttribute(
+  // setmaxnreg hands out exactly the registers the block was launched with;
+  // refuse to launch a build whose allocation differs (it could wait
+  // forever for registers that do not exist).
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, fwd_tc_kernel<X3>);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != 128) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(
       fwd_tc_kernel<X3>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int grid = std::min(sm_count(), p.total_items);
-  fwd_tc_kernel<X3><<<grid, kThreadsFwd, smem, st>>>(mq, mk, mv, mo, p);
+  fwd_tc_kernel<X3><<<grid, kThreadsFwd, smem, st>>>(mq, mk, mv, mo, mklo,
+                                                      p);
   note_launch();
   return cudaGetLastError();
 }

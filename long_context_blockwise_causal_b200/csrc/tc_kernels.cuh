@@ -22,6 +22,9 @@ struct FwdArgs {
   const int32_t* kv_lo;
   const int32_t* kv_hi;
   const int32_t* order;
+  const int32_t* row_start;
+  const void* k_rot;       // R(pos) k, bf16 [B][N][H][D]
+  const void* k_rot_lo;    // bf16 residual of k_rot (split-QK mode)
   int B, N, H;
   bool qk_x3;
   int* status;
@@ -40,6 +43,9 @@ struct BwdArgs {
   const int32_t* q_lo;
   const int32_t* q_hi;
   const int32_t* order;
+  const int32_t* row_start;
+  void* q_rot;             // scratch for R(pos) q, bf16 [B][N][H][D]
+  void* k_rot;             // scratch for R(pos) k
   float* dq_acc;
   void* dk;
   void* dv;

@@ -32,8 +32,8 @@ _sz = ctypes.c_size_t
 _d = ctypes.c_double
 
 _SIGS = {
-    "lwm_blockattn_fwd_workspace_size": (_sz, [_i] * 7),
-    "lwm_blockattn_bwd_workspace_size": (_sz, [_i] * 7),
+    "lwm_blockattn_fwd_workspace_size": (_sz, [_i] * 9),
+    "lwm_blockattn_bwd_workspace_size": (_sz, [_i] * 9),
     "lwm_blockattn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _d, _i, _i, _i,
                                _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _sz,
                                _vp]),
@@ -98,12 +98,16 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _dtype_code(t: torch.Tensor) -> int:
-    if t.dtype == torch.bfloat16:
+def _dtype_code_of(dtype) -> int:
+    if dtype == torch.bfloat16:
         return DTYPE_BF16
-    if t.dtype == torch.float32:
+    if dtype == torch.float32:
         return DTYPE_FP32
-    raise TypeError(f"unsupported dtype {t.dtype}")
+    raise TypeError(f"unsupported dtype {dtype}")
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    return _dtype_code_of(t.dtype)
 
 
 def _qk_code(qk_precision) -> int:
@@ -120,16 +124,20 @@ def _need_cuda(*ts):
             raise ValueError("tensors must be contiguous CUDA tensors")
 
 
-def fwd_workspace_size(B, N, H, max_pos, D=HEAD_DIM, block_q=BLOCK,
+def fwd_workspace_size(B, N, H, max_pos, dtype=torch.bfloat16,
+                       qk_precision="bf16", D=HEAD_DIM, block_q=BLOCK,
                        block_k=BLOCK) -> int:
-    return int(lib().lwm_blockattn_fwd_workspace_size(B, N, H, D, block_q,
-                                                      block_k, max_pos))
+    return int(lib().lwm_blockattn_fwd_workspace_size(
+        B, N, H, D, block_q, block_k, max_pos, _dtype_code_of(dtype),
+        _qk_code(qk_precision)))
 
 
-def bwd_workspace_size(B, N, H, max_pos, D=HEAD_DIM, block_q=BLOCK,
+def bwd_workspace_size(B, N, H, max_pos, dtype=torch.bfloat16,
+                       qk_precision="bf16", D=HEAD_DIM, block_q=BLOCK,
                        block_k=BLOCK) -> int:
-    return int(lib().lwm_blockattn_bwd_workspace_size(B, N, H, D, block_q,
-                                                      block_k, max_pos))
+    return int(lib().lwm_blockattn_bwd_workspace_size(
+        B, N, H, D, block_q, block_k, max_pos, _dtype_code_of(dtype),
+        _qk_code(qk_precision)))
 
 
 def _workspace(nbytes, device, workspace):
@@ -152,7 +160,8 @@ def fwd(q, k, v, segment_ids, positions, theta, max_pos=None,
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    ws = _workspace(fwd_workspace_size(B, N, H, max_pos, D, block_q, block_k),
+    ws = _workspace(fwd_workspace_size(B, N, H, max_pos, q.dtype,
+                                       qk_precision, D, block_q, block_k),
                     q.device, workspace)
     st = lib().lwm_blockattn_fwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(segment_ids), _ptr(positions),
@@ -175,7 +184,8 @@ def bwd(q, k, v, out, dout, lse, segment_ids, positions, theta,
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    ws = _workspace(bwd_workspace_size(B, N, H, max_pos, D, block_q, block_k),
+    ws = _workspace(bwd_workspace_size(B, N, H, max_pos, q.dtype,
+                                       qk_precision, D, block_q, block_k),
                     q.device, workspace)
     st = lib().lwm_blockattn_bwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),

@@ -7,6 +7,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from long_context_blockwise_causal_b200 import ops
 
@@ -50,6 +51,12 @@ def test_workspace_sizes_grow_with_inputs():
     assert c - a >= (4096 - 2048) * 128 * 4
     bw = ops.bwd_workspace_size(1, 2048, 4, 2048)
     assert bw >= a + 2048 * 4 * 128 * 4  # + fp32 dq accumulator
+    # split-QK mode keeps the bf16 residual of the rotated keys
+    x3 = ops.fwd_workspace_size(1, 2048, 4, 2048, qk_precision="bf16x3")
+    assert x3 >= a + 2048 * 4 * 128 * 2
+    # fp32 I/O needs no rotated-key scratch
+    f32 = ops.fwd_workspace_size(1, 2048, 4, 2048, dtype=torch.float32)
+    assert f32 <= a - 2048 * 4 * 128 * 2
     assert ops.fwd_workspace_size(-1, 2048, 4, 2048) == 0
     assert ops.bwd_workspace_size(1, -5, 4, 2048) == 0
 
