@@ -184,6 +184,35 @@ LWM_API int lwm_blockattn_version(void);
  * devices, all streams), counted on the host at each successful launch. */
 LWM_API uint64_t lwm_blockattn_kernel_launches(void);
 
+/* Size of the library-owned scratch array used by
+ * lwm_blockattn_fwd_noalloc (64 MiB on every device that loads the
+ * library, held until the process exits). */
+#define LWM_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/* The forward pass for callers that cannot allocate device memory while
+ * they run (e.g. a latency-critical serving loop where cudaMalloc could
+ * synchronise the device, or a plain C host with no device allocator of
+ * its own). The pages have no counterpart to this entry point: it exists
+ * only for such callers.
+ * Arguments and results are those of lwm_blockattn_fwd without the
+ * workspace: the scratch lives in a fixed device array inside the library
+ * (LWM_NOALLOC_SCRATCH_BYTES). Sizes whose lwm_blockattn_fwd_workspace_size
+ * exceeds it return LWM_ERR_WORKSPACE and launch nothing. The call never
+ * allocates or frees memory.
+ * The first call on each device looks up that device's scratch address
+ * (cudaGetSymbolAddress with the device current); make it before any stream
+ * capture begins. All calls share the one array: calls that overlap on the
+ * GPU (other streams or threads without ordering) race on it, so serialise
+ * them. */
+LWM_API int lwm_blockattn_fwd_noalloc(const void* q, const void* k,
+                                      const void* v,
+                                      const int32_t* segment_ids,
+                                      const int32_t* positions, double theta,
+                                      int block_q, int block_k, int max_pos,
+                                      int B, int N, int H, int D, int dtype,
+                                      int qk_precision, void* out,
+                                      float* lse, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -49,6 +49,9 @@ _SIGS = {
     "lwm_status_string": (ctypes.c_char_p, [_i]),
     "lwm_blockattn_version": (_i, []),
     "lwm_blockattn_kernel_launches": (ctypes.c_uint64, []),
+    "lwm_blockattn_fwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _d, _i, _i,
+                                       _i, _i, _i, _i, _i, _i, _i, _vp, _vp,
+                                       _vp]),
 }
 
 
@@ -169,6 +172,27 @@ def fwd(q, k, v, segment_ids, positions, theta, max_pos=None,
         _dtype_code(q), _qk_code(qk_precision), _ptr(out), _ptr(lse),
         _ptr(ws), ws.numel(), _stream(stream))
     _check(st, "lwm_blockattn_fwd")
+    return out, lse
+
+
+def fwd_noalloc(q, k, v, segment_ids, positions, theta, max_pos,
+                qk_precision="bf16", out=None, lse=None, stream=None,
+                block_q=BLOCK, block_k=BLOCK):
+    """Forward through lwm_blockattn_fwd_noalloc: the library's own fixed
+    scratch array replaces the workspace (see the header for its limits).
+    ``out``/``lse`` are allocated here only if the caller passes none."""
+    _need_cuda(q, k, v, segment_ids, positions, out, lse)
+    B, N, H, D = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    st = lib().lwm_blockattn_fwd_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(segment_ids), _ptr(positions),
+        float(theta), block_q, block_k, int(max_pos), B, N, H, D,
+        _dtype_code(q), _qk_code(qk_precision), _ptr(out), _ptr(lse),
+        _stream(stream))
+    _check(st, "lwm_blockattn_fwd_noalloc")
     return out, lse
 
 
