@@ -43,6 +43,7 @@ struct Workspace {
   int32_t* kv_lo;        // [B][Tq]
   int32_t* kv_hi;        // [B][Tq]
   int32_t* row_start;    // [B][N] first row of each row's packed example
+  int32_t* row_end;      // [B][N] its last row (backward only)
   uint64_t* sort_keys;   // [max(B*Uq, B*Uk)]
   int32_t* order_fwd;    // [B*Uq] units of kFwdRowsPerCta rows, longest first
   // backward only
@@ -70,6 +71,7 @@ Workspace carve(void* base, int B, int N, int H, int D, int max_pos,
   w.kv_lo = c.take<int32_t>(size_t(B) * Tq);
   w.kv_hi = c.take<int32_t>(size_t(B) * Tq);
   w.row_start = c.take<int32_t>(size_t(B) * N);
+  if (backward) w.row_end = c.take<int32_t>(size_t(B) * N);
   w.sort_keys = c.take<uint64_t>(size_t(B) * (Uq > Uk ? Uq : Uk));
   w.order_fwd = c.take<int32_t>(size_t(B) * Uq);
   if (backward) {
@@ -125,7 +127,7 @@ int prepare(const int32_t* seg, double theta, int B, int N, int D,
             int max_pos, const Workspace& w, cudaStream_t st) {
   LWM_TRY(launch_rope_table(theta, D, max_pos, w.table, st));
   LWM_TRY(launch_block_meta(seg, B, N, kBlock, kBlock, w.kv_lo, w.kv_hi, st));
-  LWM_TRY(launch_row_start(seg, B, N, w.row_start, st));
+  LWM_TRY(launch_row_start(seg, B, N, w.row_start, w.row_end, st));
   return LWM_OK;
 }
 
@@ -291,7 +293,12 @@ int lwm_blockattn_bwd(const void* q, const void* k, const void* v,
     a.q_lo = w.q_lo; a.q_hi = w.q_hi; a.order = w.order_bwd;
     a.row_start = w.row_start;
     a.dq_acc = w.dq_acc; a.dk = dk; a.dv = dv;
-    a.q_rot = w.q_rot; a.k_rot = w.k_rot;
+    a.q_rot = w.q_rot; a.k_rot = w.k_rot; a.row_end = w.row_end;
+    // queries and keys are both re-read inside the key-major sweep
+    LWM_TRY(launch_rope_apply(q, positions, w.table, B, N, H, w.q_rot,
+                              nullptr, st));
+    LWM_TRY(launch_rope_apply(k, positions, w.table, B, N, H, w.k_rot,
+                              nullptr, st));
     a.B = B; a.N = N; a.H = H;
     a.status = status_word();
     if (!a.status) return LWM_ERR_CUDA;

@@ -73,14 +73,26 @@ __device__ __forceinline__ int run_start(const int32_t* __restrict__ seg,
 
 // rs[b][i] = first index of the packed example holding row i. With
 // non-decreasing ids, "seg_j == seg_i and j <= i" is "rs[i] <= j <= i".
+// re[b][i] = last index of that example, so key k is seen by rows
+// k .. re[k].
 __global__ void row_start_kernel(const int32_t* __restrict__ seg, int B, int N,
-                                 int32_t* __restrict__ rs) {
+                                 int32_t* __restrict__ rs,
+                                 int32_t* __restrict__ re) {
   int64_t total = int64_t(B) * N;
   for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < total;
        e += int64_t(gridDim.x) * blockDim.x) {
     int b = int(e / N);
     int i = int(e - int64_t(b) * N);
-    rs[e] = run_start(seg + int64_t(b) * N, i);
+    const int32_t* s = seg + int64_t(b) * N;
+    rs[e] = run_start(s, i);
+    if (re) {
+      int v = s[i], lo = i, hi = N - 1;  // last index with s == v
+      while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (s[mid] > v) hi = mid - 1; else lo = mid;
+      }
+      re[e] = lo;
+    }
   }
 }
 
@@ -315,10 +327,11 @@ cudaError_t launch_rope_apply(const void* x, const int32_t* pos,
 }
 
 cudaError_t launch_row_start(const int32_t* seg, int B, int N, int32_t* rs,
-                             cudaStream_t st) {
+                             int32_t* re, cudaStream_t st) {
   int64_t n = int64_t(B) * N;
   if (n == 0) return cudaSuccess;
-  row_start_kernel<<<grid_for(n, 256, 148 * 16), 256, 0, st>>>(seg, B, N, rs);
+  row_start_kernel<<<grid_for(n, 256, 148 * 16), 256, 0, st>>>(seg, B, N, rs,
+                                                                re);
   note_launch();
   return cudaGetLastError();
 }

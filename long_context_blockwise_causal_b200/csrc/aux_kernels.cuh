@@ -15,8 +15,10 @@ cudaError_t launch_block_meta(const int32_t* seg, int B, int N, int bq, int bk,
 cudaError_t launch_rope_apply(const void* x, const int32_t* pos,
                               const float* table, int B, int N, int H,
                               void* hi, void* lo, cudaStream_t st);
+// rs[i]: first row of row i's packed example; re[i] (if re != nullptr):
+// its last row.
 cudaError_t launch_row_start(const int32_t* seg, int B, int N, int32_t* rs,
-                             cudaStream_t st);
+                             int32_t* re, cudaStream_t st);
 cudaError_t launch_tile_class(const int32_t* seg, int B, int N, int bq, int bk,
                               const int32_t* kv_lo, const int32_t* kv_hi,
                               uint8_t* cls, cudaStream_t st);

@@ -1,14 +1,527 @@
-// Backward pass entry for the bf16 path. Interim: the CUDA-core backward
-// kernel; the tcgen05 key-major backward replaces it.
+// Backward blockwise packed causal RoPE attention on tcgen05 (sm_100a).
+//
+// The chain rule of the forward ("LWM：突破 100 万 Token 的开源大模型",
+// 配置参数 / 概述 (b); "开源巨兽LWM：如何用RingAttention撬动百万Token多模态
+// 世界", 3.1-3.2), organised key-major: a persistent CTA owns one 128-key
+// block of one (batch row, head), keeps its dK and dV accumulators in TMEM,
+// and visits every 128-query block that can see it (the queries of the same
+// packed example at or after the key). Per query block i, with P recomputed
+// from the forward's logsumexp (scores in log2 units):
+//   S^T  = K~ Q~_i^T            (tcgen05, TMEM cols   0..127)
+//   dP^T = V dO_i^T             (tcgen05, TMEM cols 128..255)
+//   P^T  = 2^(S^T c - lse_i log2 e) (masked), dS^T = P^T (dP^T - D_i)
+//          written back as bf16 over the first 64 columns of each region
+//   dV  += P^T dO_i, dK~ += dS^T Q~_i   (A operands read from TMEM)
+//   dQ~_i = dS K~               (A = dS, staged in shared memory; result in
+//          TMEM cols 0..127, added to an fp32 accumulator in global memory)
+// Queries and keys arrive pre-rotated (R(pos) q, R(pos) k); dK = R(-pos)
+// (dK~ / sqrt(D)) in the epilogue, dQ the same in the conversion kernel.
+//
+// Warps: 0-3 compute (thread = key row = TMEM lane), 4-7 dQ reduction and
+// per-block (lse, D) staging, 8 TMA producer, 9 tcgen05 issuer + TMEM
+// owner, 10-11 idle (complete the warpgroup for setmaxnreg).
+#include <cuda.h>
+
 #include "aux_kernels.cuh"
 #include "tc_kernels.cuh"
 
 namespace lwm {
-cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t st) {
-  using T = __nv_bfloat16;
-  return launch_bwd_simt<T>(static_cast<const T*>(a.q), static_cast<const T*>(a.k),
-                            static_cast<const T*>(a.v), static_cast<const T*>(a.dout),
-                            a.lse, a.delta, a.seg, a.pos, a.table, a.B, a.N, a.H,
-                            a.dq_acc, static_cast<T*>(a.dk), static_cast<T*>(a.dv), st);
+namespace {
+
+constexpr int kThreadsBwd = 12 * 32;
+constexpr int kLaunchRegsBwd = 168;   // 65536 / 384, rounded down to 8
+constexpr int kRegsCompute = 240, kRegsDq = 160, kRegsMiscBwd = 104;
+static_assert(kRegsCompute + kRegsDq + kRegsMiscBwd == 3 * kLaunchRegsBwd,
+              "register split must equal the launch allocation");
+constexpr int kTile = kBlock * kHeadDim * 2;   // 32 KB
+constexpr int kHalf = kTile / 2;
+constexpr uint64_t kWaitNs = 4000000000ull;
+
+// shared memory map (bytes); tiles 1024-aligned
+constexpr int kSK = 0, kSV = kTile, kSQ = 2 * kTile, kSDO = 4 * kTile,
+              kSDS = 6 * kTile, kSAux = 7 * kTile,  // lse2[2][128], D[2][128]
+              kSBars = kSAux + 4 * 128 * 4;
+enum {
+  bKVFull = 0, bKVEmpty, bQFull0, bQFull1, bQEmpty0, bQEmpty1, bAux0, bAux1,
+  bSFull, bPFull, bDqFull, bDqEmpty, bAccFull, bAccEmpty, bDoneB, kNumBarsB
+};
+constexpr int kSMisc = kSBars + kNumBarsB * 8;
+constexpr int kSmemBwd = kSMisc + 16;
+
+struct BwdParams {
+  const int32_t* row_end;
+  const int32_t* pos;
+  const float2* table;
+  const int32_t* q_lo;
+  const int32_t* q_hi;
+  const int32_t* order;
+  const float* lse;
+  const float* delta;
+  float* dq_acc;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  int* status;
+  int B, N, H, Tk, G, total_items;
+  float scale_log2, scale;
+};
+
+struct BItem {
+  int b, h, j, qlo, qhi;
+};
+
+__device__ __forceinline__ BItem get_bitem(const BwdParams& p, int it) {
+  BItem m;
+  const int per_group = p.G * p.B * p.Tk;
+  const int hg = it / per_group;
+  const int rem = it - hg * per_group;
+  const int r = rem / p.G;
+  m.h = hg * p.G + (rem - r * p.G);
+  const int unit = p.order[r];
+  m.b = unit / p.Tk;
+  m.j = unit - m.b * p.Tk;
+  m.qlo = p.q_lo[unit];
+  m.qhi = p.q_hi[unit];
+  return m;
 }
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b,
+                                           float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr),
+               "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+__global__ void __launch_bounds__(kThreadsBwd, 1)
+bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+              const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v,
+              const __grid_constant__ CUtensorMap tm_do,
+              const BwdParams p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sbase = smem_u32(smem);
+  auto bar = [&](int i) { return sbase + kSBars + 8u * i; };
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kSMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSMisc + 4);
+  float* aux_lse = reinterpret_cast<float*>(smem + kSAux);        // [2][128]
+  float* aux_del = aux_lse + 2 * 128;                             // [2][128]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (sbase & 1023) {  // the swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) atomicMax(p.status, LWM_ERR_TIMEOUT);
+    return;
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(bar(bKVFull), 1);
+    mbar_init(bar(bKVEmpty), 1);
+    mbar_init(bar(bQFull0), 1);
+    mbar_init(bar(bQFull1), 1);
+    mbar_init(bar(bQEmpty0), 1);
+    mbar_init(bar(bQEmpty1), 1);
+    mbar_init(bar(bAux0), 128);
+    mbar_init(bar(bAux1), 128);
+    mbar_init(bar(bSFull), 1);
+    mbar_init(bar(bPFull), 4);
+    mbar_init(bar(bDqFull), 1);
+    mbar_init(bar(bDqEmpty), 4);
+    mbar_init(bar(bAccFull), 1);
+    mbar_init(bar(bAccEmpty), 4);
+    mbar_init(bar(bDoneB), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_holder), 512);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_do);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const uint32_t tA = tmem, tB = tmem + 128, tC = tmem + 256, tD = tmem + 384;
+  const int nitems = p.total_items;
+
+  if (warp < 4) {
+    // ---------------------------------------------------- compute (keys)
+    regs_inc<kRegsCompute>();
+    const int r = warp * 32 + lane;  // key row of the block = TMEM lane
+    const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    int g = 0, n = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+      const BItem m = get_bitem(p, it);
+      const int64_t rowbase = int64_t(m.b) * p.N;
+      const int k0 = m.j * kBlock;
+      const int kj = k0 + r;
+      const bool valid_k = kj < p.N;
+      // key kj is seen by queries kj .. re_k (none for a key >= N)
+      const int re_k = valid_k ? __ldg(p.row_end + rowbase + kj) : -1;
+      const int re_k0 = __ldg(p.row_end + rowbase + k0);
+      for (int i = m.qlo; i <= m.qhi && ok; ++i) {
+        const int st = g & 1;
+        ok = mbar_wait(bar(bSFull), g & 1, abort_flag, p.status, kWaitNs);
+        if (ok)
+          ok = mbar_wait(bar(bAux0 + st), (g >> 1) & 1, abort_flag, p.status,
+                         kWaitNs);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        const int q0 = i * kBlock;
+        const bool full = (k0 + kBlock - 1 < q0) && (re_k0 >= q0 + kBlock - 1);
+        const float* ls = aux_lse + st * 128;
+        const float* dl = aux_del + st * 128;
+        uint8_t* dsrow = smem + kSDS + r * 128;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t sv[2][32], dv[2][32];
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            tmem_ld32(tA + lane_off + (2 * half + cc) * 32, sv[cc]);
+            tmem_ld32(tB + lane_off + (2 * half + cc) * 32, dv[cc]);
+          }
+          tmem_wait_ld();
+          if (!full) {
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+              const int qb = q0 + (2 * half + cc) * 32;
+              const int lo = kj - qb, hi = re_k - qb;
+#pragma unroll
+              for (int x = 0; x < 32; ++x)
+                sv[cc][x] = (x >= lo && x <= hi) ? sv[cc][x] : 0xff800000u;
+            }
+          }
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            const int c = 2 * half + cc;
+            uint32_t pp[16], pd[16];
+#pragma unroll
+            for (int x = 0; x < 32; x += 2) {
+              const float4 l4 = *reinterpret_cast<const float4*>(ls + c * 32 + (x & ~3));
+              const float4 d4 = *reinterpret_cast<const float4*>(dl + c * 32 + (x & ~3));
+              const float la = (x & 3) ? l4.z : l4.x, lb = (x & 3) ? l4.w : l4.y;
+              const float da = (x & 3) ? d4.z : d4.x, db = (x & 3) ? d4.w : d4.y;
+              const float2 t = fma2(make_float2(__uint_as_float(sv[cc][x]),
+                                                __uint_as_float(sv[cc][x + 1])),
+                                    make_float2(p.scale_log2, p.scale_log2),
+                                    make_float2(-la, -lb));
+              const float p0 = ex2(t.x), p1 = ex2(t.y);
+              const float ds0 = p0 * (__uint_as_float(dv[cc][x]) - da);
+              const float ds1 = p1 * (__uint_as_float(dv[cc][x + 1]) - db);
+              pp[x >> 1] = pack_bf16x2(p0, p1);
+              pd[x >> 1] = pack_bf16x2(ds0, ds1);
+            }
+            tmem_st16(tA + lane_off + c * 16, pp);
+            tmem_st16(tB + lane_off + c * 16, pd);
+            // dS row r, queries c*32 .. c*32+31: query half (c >> 1),
+            // 16-byte chunks (c & 1) * 4 .. +3 of that 128-byte row
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int lc = (c & 1) * 4 + e;
+              *reinterpret_cast<uint4*>(dsrow + (c >> 1) * kHalf +
+                                        ((lc ^ (r & 7)) << 4)) =
+                  make_uint4(pd[4 * e], pd[4 * e + 1], pd[4 * e + 2],
+                             pd[4 * e + 3]);
+            }
+          }
+        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(bPFull));
+        ++g;
+      }
+      if (!ok) break;
+      // ------------------------------------------------ item epilogue
+      ok = mbar_wait(bar(bAccFull), n & 1, abort_flag, p.status, kWaitNs);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const int64_t orow = ((rowbase + (valid_k ? kj : 0)) * p.H + m.h) * kHeadDim;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tC + lane_off + c * 32, v);
+        tmem_wait_ld();
+        if (valid_k) {
+          uint4* dst = reinterpret_cast<uint4*>(p.dv + orow + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(
+                pack_bf16x2(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
+                pack_bf16x2(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
+                pack_bf16x2(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
+                pack_bf16x2(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
+        }
+      }
+      const float4* trow = reinterpret_cast<const float4*>(
+          p.table + int64_t(valid_k ? __ldg(p.pos + rowbase + kj) : 0) *
+                        (kHeadDim / 2));
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tD + lane_off + c * 32, v);
+        tmem_wait_ld();
+        if (valid_k) {
+          uint32_t o[16];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {  // pairs c*16 + 2e, 2e+1
+            const float4 cs = __ldg(trow + c * 8 + e);
+            const float a0 = __uint_as_float(v[4 * e]) * p.scale;
+            const float b0 = __uint_as_float(v[4 * e + 1]) * p.scale;
+            const float a1 = __uint_as_float(v[4 * e + 2]) * p.scale;
+            const float b1 = __uint_as_float(v[4 * e + 3]) * p.scale;
+            // R(-pos): (a, b) -> (a c + b s, b c - a s)
+            o[2 * e] = pack_bf16x2(fmaf(a0, cs.x, b0 * cs.y),
+                                   fmaf(b0, cs.x, -a0 * cs.y));
+            o[2 * e + 1] = pack_bf16x2(fmaf(a1, cs.z, b1 * cs.w),
+                                       fmaf(b1, cs.z, -a1 * cs.w));
+          }
+          uint4* dst = reinterpret_cast<uint4*>(p.dk + orow + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(bAccEmpty));
+      ++n;
+    }
+  } else if (warp < 8) {
+    // ---------------------------------------------------- dQ + staging
+    regs_dec<kRegsDq>();
+    const int r = (warp - 4) * 32 + lane;  // query row = TMEM lane
+    const uint32_t lane_off = uint32_t((warp - 4) * 32) << 16;
+    int g = 0;
+    bool ok = true;
+    int pb = 0, ph = 0, pq0 = 0;  // the block whose dQ is pending
+    auto flush = [&](int t) -> bool {
+      bool w = mbar_wait(bar(bDqFull), t & 1, abort_flag, p.status, kWaitNs);
+      w = __all_sync(0xffffffffu, w);
+      if (!w) return false;
+      tc_fence_after();
+      const int q = pq0 + r;
+      float* dst = p.dq_acc + ((int64_t(pb) * p.N + (q < p.N ? q : 0)) * p.H + ph) *
+                                  kHeadDim;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tA + lane_off + c * 32, v);
+        tmem_wait_ld();
+        if (q < p.N) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            red_add_v4(dst + c * 32 + 4 * e, __uint_as_float(v[4 * e]),
+                       __uint_as_float(v[4 * e + 1]),
+                       __uint_as_float(v[4 * e + 2]),
+                       __uint_as_float(v[4 * e + 3]));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(bDqEmpty));
+      return true;
+    };
+    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+      const BItem m = get_bitem(p, it);
+      const float* lse_bh = p.lse + (int64_t(m.b) * p.H + m.h) * p.N;
+      const float* del_bh = p.delta + (int64_t(m.b) * p.H + m.h) * p.N;
+      for (int i = m.qlo; i <= m.qhi && ok; ++i) {
+        const int st = g & 1;
+        const int q = i * kBlock + r;
+        // stage (lse log2 e, D) of this block; the slot's previous user
+        // (block g-2) finished with it before its dQ, flushed last round
+        aux_lse[st * 128 + r] = q < p.N ? __ldg(lse_bh + q) * kLog2e : 0.f;
+        aux_del[st * 128 + r] = q < p.N ? __ldg(del_bh + q) : 0.f;
+        mbar_arrive(bar(bAux0 + st));
+        if (g > 0) ok = flush(g - 1);
+        pb = m.b;
+        ph = m.h;
+        pq0 = i * kBlock;
+        ++g;
+      }
+    }
+    if (ok && g > 0) flush(g - 1);
+  } else {
+    // warps 8-11 share one register budget, then split: 8 producer,
+    // 9 MMA, 10-11 idle
+    regs_dec<kRegsMiscBwd>();
+    if (warp == 8) {
+    // ---------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int g = 0, n = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+        const BItem m = get_bitem(p, it);
+        if (n > 0)
+          ok = mbar_wait(bar(bKVEmpty), (n - 1) & 1, abort_flag, p.status,
+                         kWaitNs);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar(bKVFull), 2 * kTile);
+        const int k0 = m.j * kBlock;
+        tma_load_4d(sbase + kSK, &tm_k, bar(bKVFull), 0, m.h, k0, m.b);
+        tma_load_4d(sbase + kSK + kHalf, &tm_k, bar(bKVFull), 64, m.h, k0,
+                    m.b);
+        tma_load_4d(sbase + kSV, &tm_v, bar(bKVFull), 0, m.h, k0, m.b);
+        tma_load_4d(sbase + kSV + kHalf, &tm_v, bar(bKVFull), 64, m.h, k0,
+                    m.b);
+        ++n;
+        for (int i = m.qlo; i <= m.qhi && ok; ++i) {
+          const int st = g & 1;
+          if (g >= 2)
+            ok = mbar_wait(bar(bQEmpty0 + st), ((g >> 1) - 1) & 1, abort_flag,
+                           p.status, kWaitNs);
+          if (!ok) break;
+          mbar_arrive_expect_tx(bar(bQFull0 + st), 2 * kTile);
+          const int q0 = i * kBlock;
+          const uint32_t qd = sbase + kSQ + st * kTile;
+          const uint32_t od = sbase + kSDO + st * kTile;
+          tma_load_4d(qd, &tm_q, bar(bQFull0 + st), 0, m.h, q0, m.b);
+          tma_load_4d(qd + kHalf, &tm_q, bar(bQFull0 + st), 64, m.h, q0, m.b);
+          tma_load_4d(od, &tm_do, bar(bQFull0 + st), 0, m.h, q0, m.b);
+          tma_load_4d(od + kHalf, &tm_do, bar(bQFull0 + st), 64, m.h, q0,
+                      m.b);
+          ++g;
+        }
+      }
+      // drain loads that may still be in flight
+      if (n > 0)
+        mbar_wait(bar(bKVFull), (n - 1) & 1, nullptr, p.status, kWaitNs);
+      for (int f = g - 1; f >= 0 && f >= g - 2; --f)
+        mbar_wait(bar(bQFull0 + (f & 1)), (f >> 1) & 1, nullptr, p.status,
+                  kWaitNs);
+    }
+    } else if (warp == 9) {
+    // ---------------------------------------------------- tcgen05 issuer
+    if (lane == 0) {
+      const uint32_t idKK = idesc_bf16(128, 128, 0, 0);  // A, B K-major
+      const uint32_t idKM = idesc_bf16(128, 128, 0, 1);  // B MN-major
+      const uint32_t idMM = idesc_bf16(128, 128, 1, 1);  // A, B MN-major
+      int g = 0, n = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+        const BItem m = get_bitem(p, it);
+        ok = mbar_wait(bar(bKVFull), n & 1, abort_flag, p.status, kWaitNs);
+        if (!ok) break;
+        bool first_q = true;
+        for (int i = m.qlo; i <= m.qhi && ok; ++i) {
+          const int st = g & 1;
+          ok = mbar_wait(bar(bQFull0 + st), (g >> 1) & 1, abort_flag,
+                         p.status, kWaitNs);
+          if (ok && g > 0)
+            ok = mbar_wait(bar(bDqEmpty), (g - 1) & 1, abort_flag, p.status,
+                           kWaitNs);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t qb = sbase + kSQ + st * kTile;
+          const uint32_t ob = sbase + kSDO + st * kTile;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {  // S^T = K~ Q~^T
+            const uint32_t off = (k >> 2) * kHalf + (k & 3) * 32;
+            mma_ss(tA, sdesc_sw128(sbase + kSK + off, 16, 1024),
+                   sdesc_sw128(qb + off, 16, 1024), idKK, k > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {  // dP^T = V dO^T
+            const uint32_t off = (k >> 2) * kHalf + (k & 3) * 32;
+            mma_ss(tB, sdesc_sw128(sbase + kSV + off, 16, 1024),
+                   sdesc_sw128(ob + off, 16, 1024), idKK, k > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(bSFull));
+          ok = mbar_wait(bar(bPFull), g & 1, abort_flag, p.status, kWaitNs);
+          if (ok && first_q && n > 0)
+            ok = mbar_wait(bar(bAccEmpty), (n - 1) & 1, abort_flag, p.status,
+                           kWaitNs);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < 8; ++k)  // dV += P^T dO
+            mma_ts(tC, tA + 8 * k, sdesc_sw128(ob + 2048 * k, kHalf, 1024),
+                   idKM, (!first_q || k > 0) ? 1u : 0u);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)  // dK~ += dS^T Q~
+            mma_ts(tD, tB + 8 * k, sdesc_sw128(qb + 2048 * k, kHalf, 1024),
+                   idKM, (!first_q || k > 0) ? 1u : 0u);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)  // dQ~ = dS K~
+            mma_ss(tA, sdesc_sw128(sbase + kSDS + 2048 * k, kHalf, 1024),
+                   sdesc_sw128(sbase + kSK + 2048 * k, kHalf, 1024), idMM,
+                   k > 0 ? 1u : 0u);
+          mma_commit(bar(bDqFull));
+          mma_commit(bar(bQEmpty0 + st));
+          first_q = false;
+          ++g;
+        }
+        if (!ok) break;
+        mma_commit(bar(bAccFull));
+        mma_commit(bar(bKVEmpty));
+        ++n;
+      }
+      mma_commit(bar(bDoneB));
+      mbar_wait(bar(bDoneB), 0, nullptr, p.status, kWaitNs);
+    }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t st) {
+  if (a.B == 0 || a.N == 0 || a.H == 0) return cudaSuccess;
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_bnhd_map(&mq, a.q_rot, a.B, a.N, a.H) ||
+      !make_bnhd_map(&mk, a.k_rot, a.B, a.N, a.H) ||
+      !make_bnhd_map(&mv, a.v, a.B, a.N, a.H) ||
+      !make_bnhd_map(&mdo, a.dout, a.B, a.N, a.H))
+    return cudaErrorInvalidValue;
+  BwdParams p{};
+  p.row_end = a.row_end;
+  p.pos = a.pos;
+  p.table = reinterpret_cast<const float2*>(a.table);
+  p.q_lo = a.q_lo;
+  p.q_hi = a.q_hi;
+  p.order = a.order;
+  p.lse = a.lse;
+  p.delta = a.delta;
+  p.dq_acc = a.dq_acc;
+  p.dk = static_cast<__nv_bfloat16*>(a.dk);
+  p.dv = static_cast<__nv_bfloat16*>(a.dv);
+  p.status = a.status;
+  p.B = a.B;
+  p.N = a.N;
+  p.H = a.H;
+  p.Tk = (a.N + kBlock - 1) / kBlock;
+  p.G = 1;
+  for (int gg = 4; gg >= 1; --gg)
+    if (a.H % gg == 0) { p.G = gg; break; }
+  p.total_items = a.B * p.Tk * a.H;
+  p.scale = 1.f / sqrtf(float(kHeadDim));
+  p.scale_log2 = kLog2e * p.scale;
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, bwd_tc_kernel);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != kLaunchRegsBwd) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(bwd_tc_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kSmemBwd);
+  if (e != cudaSuccess) return e;
+  const int grid = std::min(sm_count(), p.total_items);
+  bwd_tc_kernel<<<grid, kThreadsBwd, kSmemBwd, st>>>(mq, mk, mv, mdo, p);
+  note_launch();
+  return cudaGetLastError();
+}
+
 }  // namespace lwm

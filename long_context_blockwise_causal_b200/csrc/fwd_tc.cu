@@ -254,212 +254,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t tmem = *tmem_holder;
   const int nitems = p.total_items;
 
-  if (warp == 12) {
-    // ------------------------------------------------ TMA producer
-    regs_dec<kRegsMisc>();
-    if (lane == 0) {
-      int qfill[2] = {0, 0};
-      int kfill = 0, vfill = 0;
-      bool ok = true;
-      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
-        Item m = get_item(p, it);
-        for (int s = 0; s < 2 && ok; ++s) {
-          if (!m.present[s]) continue;
-          if (qfill[s] > 0)
-            ok = mbar_wait(bar(C::bQEmpty + s), (qfill[s] - 1) & 1,
-                           abort_flag, p.status, kWaitLimitNs);
-          if (!ok) break;
-          uint32_t dst = sbase + C::kQ + s * kTileBytes;
-          mbar_arrive_expect_tx(bar(C::bQFull + s), kTileBytes);
-          tma_load_4d(dst, &tm_q, bar(C::bQFull + s), 0, m.h,
-                      m.t[s] * kBlock, m.b);
-          tma_load_4d(dst + kHalfTileBytes, &tm_q, bar(C::bQFull + s), 64,
-                      m.h, m.t[s] * kBlock, m.b);
-          qfill[s]++;
-        }
-        for (int j = m.jhi; j >= m.jlo && ok; --j) {
-          int ks = kfill % C::KS;
-          if (kfill >= C::KS)
-            ok = mbar_wait(bar(C::bKEmpty + ks), ((kfill / C::KS) - 1) & 1,
-                           abort_flag, p.status, kWaitLimitNs);
-          if (!ok) break;
-          uint32_t kd = sbase + C::kK + ks * kTileBytes;
-          mbar_arrive_expect_tx(bar(C::bKFull + ks),
-                                X3 ? 2 * kTileBytes : kTileBytes);
-          tma_load_4d(kd, &tm_k, bar(C::bKFull + ks), 0, m.h, j * kBlock,
-                      m.b);
-          tma_load_4d(kd + kHalfTileBytes, &tm_k, bar(C::bKFull + ks), 64,
-                      m.h, j * kBlock, m.b);
-          if (X3) {
-            uint32_t kl = sbase + C::kKlo + ks * kTileBytes;
-            tma_load_4d(kl, &tm_klo, bar(C::bKFull + ks), 0, m.h,
-                        j * kBlock, m.b);
-            tma_load_4d(kl + kHalfTileBytes, &tm_klo, bar(C::bKFull + ks),
-                        64, m.h, j * kBlock, m.b);
-          }
-          kfill++;
-          int vs = vfill % C::VS;
-          if (vfill >= C::VS)
-            ok = mbar_wait(bar(C::bVEmpty + vs), ((vfill / C::VS) - 1) & 1,
-                           abort_flag, p.status, kWaitLimitNs);
-          if (!ok) break;
-          uint32_t vd = sbase + C::kV + vs * kTileBytes;
-          mbar_arrive_expect_tx(bar(C::bVFull + vs), kTileBytes);
-          tma_load_4d(vd, &tm_v, bar(C::bVFull + vs), 0, m.h, j * kBlock,
-                      m.b);
-          tma_load_4d(vd + kHalfTileBytes, &tm_v, bar(C::bVFull + vs), 64,
-                      m.h, j * kBlock, m.b);
-          vfill++;
-        }
-      }
-      // Drain: every armed load must land before the CTA may exit (on the
-      // normal path these phases have completed already).
-      for (int s = 0; s < 2; ++s)
-        if (qfill[s] > 0)
-          mbar_wait(bar(C::bQFull + s), (qfill[s] - 1) & 1, nullptr,
-                    p.status, kWaitLimitNs);
-      for (int f = kfill - 1; f >= 0 && f >= kfill - C::KS; --f)
-        mbar_wait(bar(C::bKFull + f % C::KS), (f / C::KS) & 1, nullptr,
-                  p.status, kWaitLimitNs);
-      for (int f = vfill - 1; f >= 0 && f >= vfill - C::VS; --f)
-        mbar_wait(bar(C::bVFull + f % C::VS), (f / C::VS) & 1, nullptr,
-                  p.status, kWaitLimitNs);
-    }
-  } else if (warp >= 8 && warp < 12) {
-    // ------------------------------------------------ RoPE rotation
-    regs_dec<kRegsRope>();
-    const int r = threadIdx.x - 8 * 32;  // tile row owned by this thread
-    int qcount[2] = {0, 0};
-    bool ok = true;
-    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
-      Item m = get_item(p, it);
-      const int64_t rowbase = int64_t(m.b) * p.N;
-      for (int s = 0; s < 2 && ok; ++s) {
-        if (!m.present[s]) continue;
-        float4 cs0[8];
-        bool valid;
-        const float4* trow = rope_prefetch(p.pos, p.table, rowbase,
-                                           m.t[s] * kBlock + r, p.N, cs0,
-                                           valid);
-        ok = mbar_wait(bar(C::bQFull + s), qcount[s] & 1, abort_flag,
-                       p.status, kWaitLimitNs);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        qcount[s]++;
-        rope_row<X3>(smem + C::kQ + s * kTileBytes,
-                     smem + C::kQlo + s * kTileBytes, trow, cs0, r, valid);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(C::bQReady + s));
-      }
-    }
-  } else if (warp == 13) {
-    // ------------------------------------------------ tcgen05 issuer
-    regs_dec<kRegsMisc>();
-    if (lane == 0) {
-      const uint32_t idS = idesc_bf16(128, 128, 0, 0);
-      const uint32_t idPV = idesc_bf16(128, 128, 0, 1);
-      int kc = 0, vc = 0;
-      int qc[2] = {0, 0}, pc[2] = {0, 0}, oc[2] = {0, 0};
-      bool ok = true;
-      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
-        Item m = get_item(p, it);
-        bool qwaited[2] = {false, false};
-        bool pv_started[2] = {false, false};
-        int prev = -1;
-        for (int j = m.jhi; j >= m.jlo - 1 && ok; --j) {
-          const bool has_j = j >= m.jlo;
-          int ks = kc % C::KS;
-          if (has_j) {
-            ok = mbar_wait(bar(C::bKFull + ks), (kc / C::KS) & 1, abort_flag,
-                           p.status, kWaitLimitNs);
-            if (!ok) break;
-            tc_fence_after();
-          }
-          int vs = vc % C::VS;
-          if (prev >= 0) {
-            ok = mbar_wait(bar(C::bVFull + vs), (vc / C::VS) & 1, abort_flag,
-                           p.status, kWaitLimitNs);
-            if (!ok) break;
-            tc_fence_after();
-          }
-          for (int s = 0; s < 2 && ok; ++s) {
-            if (prev >= 0 && active(m, s, prev)) {
-              ok = mbar_wait(bar(C::bPFull + s), pc[s] & 1, abort_flag,
-                             p.status, kWaitLimitNs);
-              if (!ok) break;
-              pc[s]++;
-              if (!pv_started[s] && oc[s] > 0) {
-                ok = mbar_wait(bar(C::bOEmpty + s), (oc[s] - 1) & 1,
-                               abort_flag, p.status, kWaitLimitNs);
-                if (!ok) break;
-              }
-              tc_fence_after();
-              const uint32_t vbase = sbase + C::kV + vs * kTileBytes;
-              const uint32_t a_tm = tmem + s * 128;        // P over S_s
-              const uint32_t d_tm = tmem + 256 + s * 128;  // O_s
-#pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                uint64_t bd = sdesc_sw128(vbase + k * 2048, kHalfTileBytes,
-                                          1024);
-                mma_ts(d_tm, a_tm + k * 8, bd, idPV,
-                       (pv_started[s] || k > 0) ? 1u : 0u);
-              }
-              pv_started[s] = true;
-            }
-            if (has_j && active(m, s, j)) {
-              if (!qwaited[s]) {
-                ok = mbar_wait(bar(C::bQReady + s), qc[s] & 1, abort_flag,
-                               p.status, kWaitLimitNs);
-                if (!ok) break;
-                qc[s]++;
-                qwaited[s] = true;
-                tc_fence_after();
-              }
-              const uint32_t qb = sbase + C::kQ + s * kTileBytes;
-              const uint32_t kb = sbase + C::kK + ks * kTileBytes;
-              const uint32_t d_tm = tmem + s * 128;
-              int step = 0;
-              const int npass = X3 ? 3 : 1;
-              for (int pass = 0; pass < npass; ++pass) {
-                // pass 0: hi.hi, 1: hi(Q).lo(K), 2: lo(Q).hi(K)
-                uint32_t qa = qb + (pass == 2 ? (C::kQlo - C::kQ) : 0);
-                uint32_t kbb = kb + (pass == 1 ? (C::kKlo - C::kK) : 0);
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                  uint32_t off = (k >> 2) * kHalfTileBytes + (k & 3) * 32;
-                  uint64_t ad = sdesc_sw128(qa + off, 16, 1024);
-                  uint64_t bd = sdesc_sw128(kbb + off, 16, 1024);
-                  mma_ss(d_tm, ad, bd, idS, step > 0 ? 1u : 0u);
-                  ++step;
-                }
-              }
-              mma_commit(bar(C::bSFull + s));
-            }
-          }
-          if (!ok) break;
-          if (has_j) {
-            mma_commit(bar(C::bKEmpty + ks));
-            kc++;
-          }
-          if (prev >= 0) {
-            mma_commit(bar(C::bVEmpty + vs));
-            vc++;
-          }
-          prev = has_j ? j : -1;
-        }
-        if (!ok) break;
-        for (int s = 0; s < 2; ++s)
-          if (m.present[s]) {
-            mma_commit(bar(C::bOFull + s));
-            oc[s]++;
-          }
-      }
-      // every issued MMA must be complete before TMEM is released
-      mma_commit(bar(C::bDone));
-      mbar_wait(bar(C::bDone), 0, nullptr, p.status, kWaitLimitNs);
-    }
-  } else if (warp < 8) {
+  if (warp < 8) {
     // ------------------------------------------------ softmax (warps 0-7)
     regs_inc<kRegsSoftmax>();
     const int s = warp >> 2;                 // query sub-tile
@@ -622,8 +417,214 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             (m_used + __log2f(l)) * kLn2;
     }
     if (threadIdx.x == 0 || threadIdx.x == 128) bulk_wait0();
+  } else if (warp < 12) {
+    // ------------------------------------------------ RoPE rotation
+    regs_dec<kRegsRope>();
+    const int r = threadIdx.x - 8 * 32;  // tile row owned by this thread
+    int qcount[2] = {0, 0};
+    bool ok = true;
+    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+      Item m = get_item(p, it);
+      const int64_t rowbase = int64_t(m.b) * p.N;
+      for (int s = 0; s < 2 && ok; ++s) {
+        if (!m.present[s]) continue;
+        float4 cs0[8];
+        bool valid;
+        const float4* trow = rope_prefetch(p.pos, p.table, rowbase,
+                                           m.t[s] * kBlock + r, p.N, cs0,
+                                           valid);
+        ok = mbar_wait(bar(C::bQFull + s), qcount[s] & 1, abort_flag,
+                       p.status, kWaitLimitNs);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        qcount[s]++;
+        rope_row<X3>(smem + C::kQ + s * kTileBytes,
+                     smem + C::kQlo + s * kTileBytes, trow, cs0, r, valid);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::bQReady + s));
+      }
+    }
   } else {
-    regs_dec<kRegsMisc>();  // warps 14-15: no role
+    // warps 12-15 share one register budget (one setmaxnreg for the
+    // whole warpgroup), then split: 12 producer, 13 MMA, 14-15 idle
+    regs_dec<kRegsMisc>();
+    if (warp == 12) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int qfill[2] = {0, 0};
+      int kfill = 0, vfill = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+        Item m = get_item(p, it);
+        for (int s = 0; s < 2 && ok; ++s) {
+          if (!m.present[s]) continue;
+          if (qfill[s] > 0)
+            ok = mbar_wait(bar(C::bQEmpty + s), (qfill[s] - 1) & 1,
+                           abort_flag, p.status, kWaitLimitNs);
+          if (!ok) break;
+          uint32_t dst = sbase + C::kQ + s * kTileBytes;
+          mbar_arrive_expect_tx(bar(C::bQFull + s), kTileBytes);
+          tma_load_4d(dst, &tm_q, bar(C::bQFull + s), 0, m.h,
+                      m.t[s] * kBlock, m.b);
+          tma_load_4d(dst + kHalfTileBytes, &tm_q, bar(C::bQFull + s), 64,
+                      m.h, m.t[s] * kBlock, m.b);
+          qfill[s]++;
+        }
+        for (int j = m.jhi; j >= m.jlo && ok; --j) {
+          int ks = kfill % C::KS;
+          if (kfill >= C::KS)
+            ok = mbar_wait(bar(C::bKEmpty + ks), ((kfill / C::KS) - 1) & 1,
+                           abort_flag, p.status, kWaitLimitNs);
+          if (!ok) break;
+          uint32_t kd = sbase + C::kK + ks * kTileBytes;
+          mbar_arrive_expect_tx(bar(C::bKFull + ks),
+                                X3 ? 2 * kTileBytes : kTileBytes);
+          tma_load_4d(kd, &tm_k, bar(C::bKFull + ks), 0, m.h, j * kBlock,
+                      m.b);
+          tma_load_4d(kd + kHalfTileBytes, &tm_k, bar(C::bKFull + ks), 64,
+                      m.h, j * kBlock, m.b);
+          if (X3) {
+            uint32_t kl = sbase + C::kKlo + ks * kTileBytes;
+            tma_load_4d(kl, &tm_klo, bar(C::bKFull + ks), 0, m.h,
+                        j * kBlock, m.b);
+            tma_load_4d(kl + kHalfTileBytes, &tm_klo, bar(C::bKFull + ks),
+                        64, m.h, j * kBlock, m.b);
+          }
+          kfill++;
+          int vs = vfill % C::VS;
+          if (vfill >= C::VS)
+            ok = mbar_wait(bar(C::bVEmpty + vs), ((vfill / C::VS) - 1) & 1,
+                           abort_flag, p.status, kWaitLimitNs);
+          if (!ok) break;
+          uint32_t vd = sbase + C::kV + vs * kTileBytes;
+          mbar_arrive_expect_tx(bar(C::bVFull + vs), kTileBytes);
+          tma_load_4d(vd, &tm_v, bar(C::bVFull + vs), 0, m.h, j * kBlock,
+                      m.b);
+          tma_load_4d(vd + kHalfTileBytes, &tm_v, bar(C::bVFull + vs), 64,
+                      m.h, j * kBlock, m.b);
+          vfill++;
+        }
+      }
+      // Drain: every armed load must land before the CTA may exit (on the
+      // normal path these phases have completed already).
+      for (int s = 0; s < 2; ++s)
+        if (qfill[s] > 0)
+          mbar_wait(bar(C::bQFull + s), (qfill[s] - 1) & 1, nullptr,
+                    p.status, kWaitLimitNs);
+      for (int f = kfill - 1; f >= 0 && f >= kfill - C::KS; --f)
+        mbar_wait(bar(C::bKFull + f % C::KS), (f / C::KS) & 1, nullptr,
+                  p.status, kWaitLimitNs);
+      for (int f = vfill - 1; f >= 0 && f >= vfill - C::VS; --f)
+        mbar_wait(bar(C::bVFull + f % C::VS), (f / C::VS) & 1, nullptr,
+                  p.status, kWaitLimitNs);
+    }
+    } else if (warp == 13) {
+    // ------------------------------------------------ tcgen05 issuer
+    if (lane == 0) {
+      const uint32_t idS = idesc_bf16(128, 128, 0, 0);
+      const uint32_t idPV = idesc_bf16(128, 128, 0, 1);
+      int kc = 0, vc = 0;
+      int qc[2] = {0, 0}, pc[2] = {0, 0}, oc[2] = {0, 0};
+      bool ok = true;
+      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+        Item m = get_item(p, it);
+        bool qwaited[2] = {false, false};
+        bool pv_started[2] = {false, false};
+        int prev = -1;
+        for (int j = m.jhi; j >= m.jlo - 1 && ok; --j) {
+          const bool has_j = j >= m.jlo;
+          int ks = kc % C::KS;
+          if (has_j) {
+            ok = mbar_wait(bar(C::bKFull + ks), (kc / C::KS) & 1, abort_flag,
+                           p.status, kWaitLimitNs);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          int vs = vc % C::VS;
+          if (prev >= 0) {
+            ok = mbar_wait(bar(C::bVFull + vs), (vc / C::VS) & 1, abort_flag,
+                           p.status, kWaitLimitNs);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          for (int s = 0; s < 2 && ok; ++s) {
+            if (prev >= 0 && active(m, s, prev)) {
+              ok = mbar_wait(bar(C::bPFull + s), pc[s] & 1, abort_flag,
+                             p.status, kWaitLimitNs);
+              if (!ok) break;
+              pc[s]++;
+              if (!pv_started[s] && oc[s] > 0) {
+                ok = mbar_wait(bar(C::bOEmpty + s), (oc[s] - 1) & 1,
+                               abort_flag, p.status, kWaitLimitNs);
+                if (!ok) break;
+              }
+              tc_fence_after();
+              const uint32_t vbase = sbase + C::kV + vs * kTileBytes;
+              const uint32_t a_tm = tmem + s * 128;        // P over S_s
+              const uint32_t d_tm = tmem + 256 + s * 128;  // O_s
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                uint64_t bd = sdesc_sw128(vbase + k * 2048, kHalfTileBytes,
+                                          1024);
+                mma_ts(d_tm, a_tm + k * 8, bd, idPV,
+                       (pv_started[s] || k > 0) ? 1u : 0u);
+              }
+              pv_started[s] = true;
+            }
+            if (has_j && active(m, s, j)) {
+              if (!qwaited[s]) {
+                ok = mbar_wait(bar(C::bQReady + s), qc[s] & 1, abort_flag,
+                               p.status, kWaitLimitNs);
+                if (!ok) break;
+                qc[s]++;
+                qwaited[s] = true;
+                tc_fence_after();
+              }
+              const uint32_t qb = sbase + C::kQ + s * kTileBytes;
+              const uint32_t kb = sbase + C::kK + ks * kTileBytes;
+              const uint32_t d_tm = tmem + s * 128;
+              int step = 0;
+              const int npass = X3 ? 3 : 1;
+              for (int pass = 0; pass < npass; ++pass) {
+                // pass 0: hi.hi, 1: hi(Q).lo(K), 2: lo(Q).hi(K)
+                uint32_t qa = qb + (pass == 2 ? (C::kQlo - C::kQ) : 0);
+                uint32_t kbb = kb + (pass == 1 ? (C::kKlo - C::kK) : 0);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                  uint32_t off = (k >> 2) * kHalfTileBytes + (k & 3) * 32;
+                  uint64_t ad = sdesc_sw128(qa + off, 16, 1024);
+                  uint64_t bd = sdesc_sw128(kbb + off, 16, 1024);
+                  mma_ss(d_tm, ad, bd, idS, step > 0 ? 1u : 0u);
+                  ++step;
+                }
+              }
+              mma_commit(bar(C::bSFull + s));
+            }
+          }
+          if (!ok) break;
+          if (has_j) {
+            mma_commit(bar(C::bKEmpty + ks));
+            kc++;
+          }
+          if (prev >= 0) {
+            mma_commit(bar(C::bVEmpty + vs));
+            vc++;
+          }
+          prev = has_j ? j : -1;
+        }
+        if (!ok) break;
+        for (int s = 0; s < 2; ++s)
+          if (m.present[s]) {
+            mma_commit(bar(C::bOFull + s));
+            oc[s]++;
+          }
+      }
+      // every issued MMA must be complete before TMEM is released
+      mma_commit(bar(C::bDone));
+      mbar_wait(bar(C::bDone), 0, nullptr, p.status, kWaitLimitNs);
+    }
+    }
   }
 
   tc_fence_before();

@@ -1,6 +1,8 @@
 // Tensor-core (tcgen05) kernels of the blockwise attention path.
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace lwm {
@@ -44,6 +46,7 @@ struct BwdArgs {
   const int32_t* q_hi;
   const int32_t* order;
   const int32_t* row_start;
+  const int32_t* row_end;
   void* q_rot;             // scratch for R(pos) q, bf16 [B][N][H][D]
   void* k_rot;             // scratch for R(pos) k
   float* dq_acc;
@@ -54,6 +57,10 @@ struct BwdArgs {
 };
 
 cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t st);
+// 4-D TMA map over a bf16 [B][N][H][128] tensor, box 64 x 1 x 128 x 1,
+// 128-byte swizzle. False if the driver's encoder is unavailable/refuses.
+bool make_bnhd_map(CUtensorMap* m, const void* base, int B, int N, int H);
+int sm_count();
 cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t st);
 
 }  // namespace lwm
