@@ -13,7 +13,8 @@
 //          written back as bf16 over the first 64 columns of each region
 //   dV  += P^T dO_i, dK~ += dS^T Q~_i   (A operands read from TMEM)
 //   dQ~_i = dS K~               (A = dS, staged in shared memory; result in
-//          TMEM cols 0..127, added to an fp32 accumulator in global memory)
+//          TMEM cols 0..127, added to an fp32 accumulator in global memory
+//          by TMA reduce-add from the then-dead dS buffer)
 // Queries and keys arrive pre-rotated (R(pos) q, R(pos) k); dK = R(-pos)
 // (dK~ / sqrt(D)) in the epilogue, dQ the same in the conversion kernel.
 //
@@ -43,7 +44,8 @@ constexpr int kSK = 0, kSV = kTile, kSQ = 2 * kTile, kSDO = 4 * kTile,
               kSBars = kSAux + 4 * 128 * 4;
 enum {
   bKVFull = 0, bKVEmpty, bQFull0, bQFull1, bQEmpty0, bQEmpty1, bAux0, bAux1,
-  bSFull, bPFull, bDqFull, bDqEmpty, bAccFull, bAccEmpty, bDoneB, kNumBarsB
+  bSFull, bPFull, bDqFull, bDqEmpty, bAccFull, bAccEmpty, bDoneB, bDsFree,
+  kNumBarsB
 };
 constexpr int kSMisc = kSBars + kNumBarsB * 8;
 constexpr int kSmemBwd = kSMisc + 16;
@@ -96,6 +98,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
               const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v,
               const __grid_constant__ CUtensorMap tm_do,
+              const __grid_constant__ CUtensorMap tm_dq,
               const BwdParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
@@ -126,6 +129,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(bar(bAccFull), 1);
     mbar_init(bar(bAccEmpty), 4);
     mbar_init(bar(bDoneB), 1);
+    mbar_init(bar(bDsFree), 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -138,6 +142,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
     prefetch_tmap(&tm_do);
+    prefetch_tmap(&tm_dq);
   }
   tc_fence_before();
   __syncthreads();
@@ -176,6 +181,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         const float* ls = aux_lse + st * 128;
         const float* dl = aux_del + st * 128;
         uint8_t* dsrow = smem + kSDS + r * 128;
+        bool ds_ready = g == 0;  // the dS buffer also stages dQ of block g-1
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t sv[2][32], dv[2][32];
@@ -217,6 +223,12 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
             tmem_st16(tA + lane_off + c * 16, pp);
             tmem_st16(tB + lane_off + c * 16, pd);
+            if (!ds_ready) {
+              bool w = mbar_wait(bar(bDsFree), (g - 1) & 1, abort_flag,
+                                 p.status, kWaitNs);
+              ds_ready = true;
+              if (!__all_sync(0xffffffffu, w)) ok = false;
+            }
             // dS row r, queries c*32 .. c*32+31: query half (c >> 1),
             // 16-byte chunks (c & 1) * 4 .. +3 of that 128-byte row
 #pragma unroll
@@ -230,6 +242,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
         }
         tmem_wait_st();
+        if (!ok) break;
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
@@ -301,31 +314,49 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     int g = 0;
     bool ok = true;
     int pb = 0, ph = 0, pq0 = 0;  // the block whose dQ is pending
+    // dQ of block t: TMEM -> registers (then TMEM is free for the next
+    // S^T), registers -> the dead dS buffer (this warp's 32 rows, two
+    // 32-column chunks of 4 KB at a time, 128-byte swizzle), then a TMA
+    // reduce-add of each chunk into the fp32 accumulator.
+    const int wq = warp - 4;
+    const uint32_t stage = sbase + kSDS + wq * 8192;
     auto flush = [&](int t) -> bool {
       bool w = mbar_wait(bar(bDqFull), t & 1, abort_flag, p.status, kWaitNs);
       w = __all_sync(0xffffffffu, w);
       if (!w) return false;
       tc_fence_after();
-      const int q = pq0 + r;
-      float* dst = p.dq_acc + ((int64_t(pb) * p.N + (q < p.N ? q : 0)) * p.H + ph) *
-                                  kHeadDim;
+      uint32_t v[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tA + lane_off + c * 32, v);
-        tmem_wait_ld();
-        if (q < p.N) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            red_add_v4(dst + c * 32 + 4 * e, __uint_as_float(v[4 * e]),
-                       __uint_as_float(v[4 * e + 1]),
-                       __uint_as_float(v[4 * e + 2]),
-                       __uint_as_float(v[4 * e + 3]));
-        }
-      }
+      for (int c = 0; c < 4; ++c) tmem_ld32(tA + lane_off + c * 32, v[c]);
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(bDqEmpty));
+#pragma unroll
+      for (int round = 0; round < 2; ++round) {
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = 2 * round + cc;
+          uint8_t* rowp = smem + kSDS + wq * 8192 + cc * 4096 + lane * 128;
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            *reinterpret_cast<uint4*>(rowp + ((e ^ (lane & 7)) << 4)) =
+                make_uint4(v[c][4 * e], v[c][4 * e + 1], v[c][4 * e + 2],
+                           v[c][4 * e + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc)
+            tma_reduce_add_4d(&tm_dq, stage + cc * 4096, (2 * round + cc) * 32,
+                              ph, pq0 + wq * 32, pb);
+          bulk_commit();
+          bulk_wait_read0();
+        }
+        __syncwarp();
+      }
+      if (lane == 0) mbar_arrive(bar(bDsFree));
       return true;
     };
     for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
@@ -348,6 +379,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
     }
     if (ok && g > 0) flush(g - 1);
+    if (lane == 0) bulk_wait0();
   } else {
     // warps 8-11 share one register budget, then split: 8 producer,
     // 9 MMA, 10-11 idle
@@ -481,11 +513,12 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
 
 cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t st) {
   if (a.B == 0 || a.N == 0 || a.H == 0) return cudaSuccess;
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mdq;
   if (!make_bnhd_map(&mq, a.q_rot, a.B, a.N, a.H) ||
       !make_bnhd_map(&mk, a.k_rot, a.B, a.N, a.H) ||
       !make_bnhd_map(&mv, a.v, a.B, a.N, a.H) ||
-      !make_bnhd_map(&mdo, a.dout, a.B, a.N, a.H))
+      !make_bnhd_map(&mdo, a.dout, a.B, a.N, a.H) ||
+      !make_bnhd_f32_map(&mdq, a.dq_acc, a.B, a.N, a.H))
     return cudaErrorInvalidValue;
   BwdParams p{};
   p.row_end = a.row_end;
@@ -519,7 +552,8 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t st) {
                            kSmemBwd);
   if (e != cudaSuccess) return e;
   const int grid = std::min(sm_count(), p.total_items);
-  bwd_tc_kernel<<<grid, kThreadsBwd, kSmemBwd, st>>>(mq, mk, mv, mdo, p);
+  bwd_tc_kernel<<<grid, kThreadsBwd, kSmemBwd, st>>>(mq, mk, mv, mdo, mdq,
+                                                      p);
   note_launch();
   return cudaGetLastError();
 }

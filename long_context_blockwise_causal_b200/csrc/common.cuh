@@ -112,6 +112,18 @@ __device__ __forceinline__ void tma_store_4d(const void* tmap, uint32_t src,
       : "memory");
 }
 
+// Element-wise add of a shared-memory box into global memory (fp32 add
+// for an fp32 tensor map), tracked by the bulk async-group.
+__device__ __forceinline__ void tma_reduce_add_4d(const void* tmap,
+                                                  uint32_t src, int c0, int c1,
+                                                  int c2, int c3) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group "
+      "[%0, {%2, %3, %4, %5}], [%1];" ::"l"(tmap),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

@@ -680,6 +680,27 @@ bool make_bnhd_map(CUtensorMap* m, const void* base, int B, int N, int H) {
   return r == CUDA_SUCCESS;
 }
 
+// fp32 [B][N][H][128] tensor as a 4-D map {D, H, N, B}; box 32 x 1 x 32 x 1
+// (one 128-byte column chunk of 32 rows) with the 128-byte swizzle.
+bool make_bnhd_f32_map(CUtensorMap* m, const void* base, int B, int N,
+                       int H) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {cuuint64_t(kHeadDim), cuuint64_t(H), cuuint64_t(N),
+                        cuuint64_t(B)};
+  cuuint64_t strides[3] = {cuuint64_t(kHeadDim) * 4,
+                           cuuint64_t(H) * kHeadDim * 4,
+                           cuuint64_t(N) * H * kHeadDim * 4};
+  cuuint32_t box[4] = {32, 1, 32, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
+                  const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;

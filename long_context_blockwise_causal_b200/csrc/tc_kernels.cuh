@@ -60,6 +60,10 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t st);
 // 4-D TMA map over a bf16 [B][N][H][128] tensor, box 64 x 1 x 128 x 1,
 // 128-byte swizzle. False if the driver's encoder is unavailable/refuses.
 bool make_bnhd_map(CUtensorMap* m, const void* base, int B, int N, int H);
+// 4-D TMA map over an fp32 [B][N][H][128] tensor, box 32 x 1 x 32 x 1,
+// 128-byte swizzle (used for the dQ reduce-add).
+bool make_bnhd_f32_map(CUtensorMap* m, const void* base, int B, int N,
+                       int H);
 int sm_count();
 cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t st);
 
