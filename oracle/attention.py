@@ -73,7 +73,6 @@ def attn_fwd_rows(q, k, v, segment_ids, positions, theta, b, h, rows,
 
     Returns (out [len(rows), D], lse [len(rows)]), both fp64.
     """
-    q = q if isinstance(q, np.ndarray) else _f64(q)
     seg = _i64(segment_ids)[b]
     pos = _i64(positions)[b]
     rows = np.asarray(rows, dtype=np.int64)

@@ -190,11 +190,14 @@ def test_fwd_full_size_sampled_rows(cuda_dev, name, rows, heads):
 
 
 def check_sampled_rows(t, out, lse, nrows, heads, seed):
+    # the oracle pulls one head of K/V (and the sampled Q rows) at a time,
+    # so no full host copy of the 1M-token inputs is made
     N = t["q"].shape[1]
     H = t["q"].shape[2]
     rng = np.random.default_rng(seed)
     rows = np.unique(np.r_[0, N - 1, rng.integers(0, N, nrows - 2)])
-    h = host(t)
+    h = {k: (v.cpu() if k in ("segment_ids", "positions") else v)
+         for k, v in t.items()}
     heads = range(H) if heads is None else heads
     go = out[0, torch.from_numpy(rows).to(out.device)].float().cpu().numpy()
     gl = lse[0][:, torch.from_numpy(rows).to(lse.device)].cpu().numpy()
