@@ -734,8 +734,10 @@ static cudaError_t launch_fwd_impl(const FwdArgs& a, cudaStream_t st) {
   p.H = a.H;
   p.Tq = (a.N + kBlock - 1) / kBlock;
   p.U = (p.Tq + kFwdBlocksPerUnit - 1) / kFwdBlocksPerUnit;
+  // heads interleaved per scheduling round: 2 keeps the K/V of the heads
+  // in flight L2-resident while still mixing costs across CTAs
   p.G = 1;
-  for (int g = 4; g >= 1; --g)
+  for (int g = 2; g >= 1; --g)
     if (a.H % g == 0) { p.G = g; break; }
   p.total_items = a.B * p.U * a.H;
   p.scale_log2 = kLog2e / sqrtf(float(kHeadDim));
