@@ -180,6 +180,15 @@ LWM_API const char* lwm_status_string(int status);
 /* LWM_BLOCKATTN_VERSION of the built library. */
 LWM_API int lwm_blockattn_version(void);
 
+/* Self-test of the failure path: launches one small CTA that waits on an
+ * mbarrier nobody arrives on, with the same bounded wait the attention
+ * kernels use and a limit of limit_ns nanoseconds (clamped to [1 ms, 2 s]).
+ * When the limit passes, the kernel records LWM_ERR_TIMEOUT in the device
+ * status word and returns normally (no trap, the context stays usable);
+ * lwm_blockattn_last_status then reports and clears it. Test use only. */
+LWM_API int lwm_blockattn_selftest_wait_timeout(uint64_t limit_ns,
+                                                void* stream);
+
 /* Number of CUDA kernels this library has launched in this process (all
  * devices, all streams), counted on the host at each successful launch. */
 LWM_API uint64_t lwm_blockattn_kernel_launches(void);

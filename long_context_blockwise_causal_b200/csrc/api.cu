@@ -20,6 +20,22 @@ __device__ int g_check_words[2];
 static std::atomic<uint64_t> g_launches{0};
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
+// One CTA waits on a barrier that is never arrived on; the bounded wait
+// gives up after limit_ns and records LWM_ERR_TIMEOUT in *status.
+__global__ void selftest_wait_kernel(int* status, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar_storage;
+  __shared__ int abort_word;
+  const uint32_t bar = smem_u32(&bar_storage);
+  if (threadIdx.x == 0) {
+    abort_word = 0;
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0)
+    mbar_wait(bar, 0, &abort_word, status, limit_ns);
+}
+
 namespace {
 
 constexpr size_t kAlign = 256;
@@ -152,6 +168,17 @@ const char* lwm_status_string(int status) {
 }
 
 int lwm_blockattn_version(void) { return LWM_BLOCKATTN_VERSION; }
+
+int lwm_blockattn_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
+  if (limit_ns < 1000000ull) limit_ns = 1000000ull;
+  if (limit_ns > 2000000000ull) limit_ns = 2000000000ull;
+  int* st = status_word();
+  if (!st) return LWM_ERR_CUDA;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      st, limit_ns);
+  note_launch();
+  return cuda_status(cudaGetLastError());
+}
 
 uint64_t lwm_blockattn_kernel_launches(void) {
   return g_launches.load(std::memory_order_relaxed);

@@ -49,6 +49,7 @@ _SIGS = {
     "lwm_status_string": (ctypes.c_char_p, [_i]),
     "lwm_blockattn_version": (_i, []),
     "lwm_blockattn_kernel_launches": (ctypes.c_uint64, []),
+    "lwm_blockattn_selftest_wait_timeout": (_i, [ctypes.c_uint64, _vp]),
     "lwm_blockattn_fwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _d, _i, _i,
                                        _i, _i, _i, _i, _i, _i, _i, _vp, _vp,
                                        _vp]),
@@ -264,6 +265,13 @@ def check_inputs(segment_ids, positions, max_pos, stream=None):
 def kernel_launches() -> int:
     """Kernels the library has launched in this process so far."""
     return int(lib().lwm_blockattn_kernel_launches())
+
+
+def selftest_wait_timeout(limit_ns=20_000_000, stream=None):
+    """Launch the bounded-wait self-test kernel (see the header)."""
+    _check(lib().lwm_blockattn_selftest_wait_timeout(int(limit_ns),
+                                                     _stream(stream)),
+           "lwm_blockattn_selftest_wait_timeout")
 
 
 def last_status(stream=None) -> int:
