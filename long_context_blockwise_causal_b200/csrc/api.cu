@@ -61,6 +61,7 @@ struct Workspace {
   int32_t* row_start;    // [B][N] first row of each row's packed example
   int32_t* row_end;      // [B][N] its last row (backward only)
   uint64_t* sort_keys;   // [max(B*Uq, B*Uk)]
+  int32_t* counter;      // work counter of the attention kernel
   int32_t* order_fwd;    // [B*Uq] units of kFwdRowsPerCta rows, longest first
   // backward only
   int32_t* q_lo;         // [B][Tk]
@@ -89,6 +90,7 @@ Workspace carve(void* base, int B, int N, int H, int D, int max_pos,
   w.row_start = c.take<int32_t>(size_t(B) * N);
   if (backward) w.row_end = c.take<int32_t>(size_t(B) * N);
   w.sort_keys = c.take<uint64_t>(size_t(B) * (Uq > Uk ? Uq : Uk));
+  w.counter = c.take<int32_t>(64);
   w.order_fwd = c.take<int32_t>(size_t(B) * Uq);
   if (backward) {
     w.q_lo = c.take<int32_t>(size_t(B) * Tk);
@@ -238,6 +240,7 @@ int lwm_blockattn_fwd(const void* q, const void* k, const void* v,
   a.q = q; a.k = k; a.v = v; a.out = out; a.lse = lse;
   a.seg = segment_ids; a.pos = positions; a.table = w.table;
   a.kv_lo = w.kv_lo; a.kv_hi = w.kv_hi; a.order = w.order_fwd;
+  a.counter = w.counter;
   a.row_start = w.row_start;
   a.k_rot = w.k_rot; a.k_rot_lo = w.k_rot_lo;
   a.B = B; a.N = N; a.H = H;
@@ -248,7 +251,8 @@ int lwm_blockattn_fwd(const void* q, const void* k, const void* v,
   a.status = status_word();
   if (!a.status) return LWM_ERR_CUDA;
   LWM_TRY(launch_lpt_order(B, (N + kBlock - 1) / kBlock, kFwdBlocksPerUnit,
-                           w.kv_lo, w.kv_hi, w.sort_keys, w.order_fwd, st));
+                           w.kv_lo, w.kv_hi, w.sort_keys, w.order_fwd,
+                           w.counter, st));
   return cuda_status(launch_fwd_tc(a, st));
 }
 
@@ -313,11 +317,13 @@ int lwm_blockattn_bwd(const void* q, const void* k, const void* v,
                            (N + kBlock - 1) / kBlock, w.kv_lo, w.kv_hi, w.q_lo,
                            w.q_hi, st));
     LWM_TRY(launch_lpt_order(B, (N + kBlock - 1) / kBlock, kBwdBlocksPerUnit,
-                             w.q_lo, w.q_hi, w.sort_keys, w.order_bwd, st));
+                             w.q_lo, w.q_hi, w.sort_keys, w.order_bwd,
+                             w.counter, st));
     BwdArgs a{};
     a.q = q; a.k = k; a.v = v; a.dout = dout; a.lse = lse; a.delta = w.delta;
     a.seg = segment_ids; a.pos = positions; a.table = w.table;
     a.q_lo = w.q_lo; a.q_hi = w.q_hi; a.order = w.order_bwd;
+    a.counter = w.counter;
     a.row_start = w.row_start;
     a.dq_acc = w.dq_acc; a.dk = dk; a.dv = dv;
     a.q_rot = w.q_rot; a.k_rot = w.k_rot; a.row_end = w.row_end;

@@ -182,8 +182,9 @@ __global__ void unit_cost_kernel(int B, int T, int group,
 // memory; the sorted unit ids are written to order[].
 __global__ void __launch_bounds__(1024)
 lpt_sort_kernel(const uint64_t* __restrict__ keys, int n,
-                int32_t* __restrict__ order) {
+                int32_t* __restrict__ order, int32_t* __restrict__ counter) {
   extern __shared__ uint64_t sk[];
+  if (threadIdx.x == 0) *counter = 0;  // work counter of the next launch
   int p2 = 1;
   while (p2 < n) p2 <<= 1;
   for (int i = threadIdx.x; i < p2; i += blockDim.x)
@@ -208,8 +209,10 @@ lpt_sort_kernel(const uint64_t* __restrict__ keys, int n,
 
 // Fallback order for more units than one CTA can sort: per batch row, the
 // units from last to first (longest first for a causal row).
-__global__ void reverse_order_kernel(int B, int U, int32_t* __restrict__ order) {
+__global__ void reverse_order_kernel(int B, int U, int32_t* __restrict__ order,
+                                     int32_t* __restrict__ counter) {
   int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e == 0) *counter = 0;
   if (e >= B * U) return;
   int b = e / U, u = e - b * U;
   order[e] = b * U + (U - 1 - u);
@@ -362,7 +365,8 @@ cudaError_t launch_kv_meta(int B, int Tq, int Tk, const int32_t* kv_lo,
 
 cudaError_t launch_lpt_order(int B, int T, int group, const int32_t* lo,
                              const int32_t* hi, uint64_t* keys,
-                             int32_t* order, cudaStream_t st) {
+                             int32_t* order, int32_t* counter,
+                             cudaStream_t st) {
   int U = (T + group - 1) / group;
   int n = B * U;
   if (n == 0) return cudaSuccess;
@@ -379,10 +383,11 @@ cudaError_t launch_lpt_order(int B, int T, int group, const int32_t* lo,
           int(smem));
       if (e != cudaSuccess) return e;
     }
-    lpt_sort_kernel<<<1, 1024, smem, st>>>(keys, n, order);
+    lpt_sort_kernel<<<1, 1024, smem, st>>>(keys, n, order, counter);
     note_launch();
   } else {
-    reverse_order_kernel<<<(n + 255) / 256, 256, 0, st>>>(B, U, order);
+    reverse_order_kernel<<<(n + 255) / 256, 256, 0, st>>>(B, U, order,
+                                                           counter);
     note_launch();
   }
   return cudaGetLastError();

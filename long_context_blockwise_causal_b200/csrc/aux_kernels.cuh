@@ -26,10 +26,11 @@ cudaError_t launch_kv_meta(int B, int Tq, int Tk, const int32_t* kv_lo,
                            const int32_t* kv_hi, int32_t* q_lo, int32_t* q_hi,
                            cudaStream_t st);
 // Orders the units (b, u), u covering `group` consecutive blocks, by the
-// size of the union of their [lo, hi] ranges, longest first.
+// size of the union of their [lo, hi] ranges, longest first, and zeroes
+// the work counter the following attention launch hands units out with.
 cudaError_t launch_lpt_order(int B, int T, int group, const int32_t* lo,
                              const int32_t* hi, uint64_t* keys, int32_t* order,
-                             cudaStream_t st);
+                             int32_t* counter, cudaStream_t st);
 cudaError_t launch_check_inputs(const int32_t* seg, const int32_t* pos, int B,
                                 int N, int max_pos, int* res, cudaStream_t st);
 template <typename T>

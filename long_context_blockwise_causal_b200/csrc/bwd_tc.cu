@@ -45,12 +45,13 @@ constexpr int kSK = 0, kSV = kTile, kSQ = 2 * kTile, kSDO = 4 * kTile,
 enum {
   bKVFull = 0, bKVEmpty, bQFull0, bQFull1, bQEmpty0, bQEmpty1, bAux0, bAux1,
   bSFull, bPFull, bDqFull, bDqEmpty, bAccFull, bAccEmpty, bDoneB, bDsFree,
-  kNumBarsB
+  bItemFull0, bItemFull1, bItemEmpty0, bItemEmpty1, kNumBarsB
 };
 constexpr int kSMisc = kSBars + kNumBarsB * 8;
-constexpr int kSmemBwd = kSMisc + 16;
+constexpr int kSmemBwd = kSMisc + 16;   // tmem addr, abort, 2 work slots
 
 struct BwdParams {
+  int32_t* counter;
   const int32_t* row_end;
   const int32_t* pos;
   const float2* table;
@@ -105,6 +106,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   auto bar = [&](int i) { return sbase + kSBars + 8u * i; };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kSMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSMisc + 4);
+  // two-slot ring of work units (producer -> other roles)
+  volatile int* item_slot = reinterpret_cast<volatile int*>(smem + kSMisc + 8);
   float* aux_lse = reinterpret_cast<float*>(smem + kSAux);        // [2][128]
   float* aux_del = aux_lse + 2 * 128;                             // [2][128]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -130,6 +133,11 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(bar(bAccEmpty), 4);
     mbar_init(bar(bDoneB), 1);
     mbar_init(bar(bDsFree), 4);
+    mbar_init(bar(bItemFull0), 1);
+    mbar_init(bar(bItemFull1), 1);
+    // consumers: 4 compute warps, 4 dQ warps, the MMA lane
+    mbar_init(bar(bItemEmpty0), 9);
+    mbar_init(bar(bItemEmpty1), 9);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -158,7 +166,15 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     const uint32_t lane_off = uint32_t(warp * 32) << 16;
     int g = 0, n = 0;
     bool ok = true;
-    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+    for (int u = 0; ok; ++u) {
+      ok = mbar_wait(bar(bItemFull0 + (u & 1)), (u >> 1) & 1, abort_flag,
+                     p.status, kWaitNs);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      const int it = item_slot[u & 1];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(bItemEmpty0 + (u & 1)));
+      if (it < 0) break;
       const BItem m = get_bitem(p, it);
       const int64_t rowbase = int64_t(m.b) * p.N;
       const int k0 = m.j * kBlock;
@@ -359,7 +375,15 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (lane == 0) mbar_arrive(bar(bDsFree));
       return true;
     };
-    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+    for (int u = 0; ok; ++u) {
+      ok = mbar_wait(bar(bItemFull0 + (u & 1)), (u >> 1) & 1, abort_flag,
+                     p.status, kWaitNs);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      const int it = item_slot[u & 1];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(bItemEmpty0 + (u & 1)));
+      if (it < 0) break;
       const BItem m = get_bitem(p, it);
       const float* lse_bh = p.lse + (int64_t(m.b) * p.H + m.h) * p.N;
       const float* del_bh = p.delta + (int64_t(m.b) * p.H + m.h) * p.N;
@@ -389,7 +413,17 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (lane == 0) {
       int g = 0, n = 0;
       bool ok = true;
-      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+      for (int u = 0; ok; ++u) {
+        if (u >= 2) {
+          ok = mbar_wait(bar(bItemEmpty0 + (u & 1)), ((u >> 1) - 1) & 1,
+                         abort_flag, p.status, kWaitNs);
+          if (!ok) break;
+        }
+        int it = atomicAdd(p.counter, 1);
+        if (it >= nitems) it = -1;
+        item_slot[u & 1] = it;
+        mbar_arrive(bar(bItemFull0 + (u & 1)));
+        if (it < 0) break;
         const BItem m = get_bitem(p, it);
         if (n > 0)
           ok = mbar_wait(bar(bKVEmpty), (n - 1) & 1, abort_flag, p.status,
@@ -437,7 +471,13 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint32_t idMM = idesc_bf16(128, 128, 1, 1);  // A, B MN-major
       int g = 0, n = 0;
       bool ok = true;
-      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+      for (int u = 0; ok; ++u) {
+        ok = mbar_wait(bar(bItemFull0 + (u & 1)), (u >> 1) & 1, abort_flag,
+                       p.status, kWaitNs);
+        if (!ok) break;
+        const int it = item_slot[u & 1];
+        mbar_arrive(bar(bItemEmpty0 + (u & 1)));
+        if (it < 0) break;
         const BItem m = get_bitem(p, it);
         ok = mbar_wait(bar(bKVFull), n & 1, abort_flag, p.status, kWaitNs);
         if (!ok) break;
@@ -521,6 +561,7 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t st) {
       !make_bnhd_f32_map(&mdq, a.dq_acc, a.B, a.N, a.H))
     return cudaErrorInvalidValue;
   BwdParams p{};
+  p.counter = a.counter;
   p.row_end = a.row_end;
   p.pos = a.pos;
   p.table = reinterpret_cast<const float2*>(a.table);

@@ -35,7 +35,7 @@ namespace {
 constexpr int kThreadsFwd = 16 * 32;
 // Register budget per warpgroup after setmaxnreg (launch: 128 each). The
 // four groups share each SM sub-partition, so the sum must stay 4 x 128.
-constexpr int kRegsSoftmax = 176, kRegsRope = 96, kRegsMisc = 64;
+constexpr int kRegsSoftmax = 184, kRegsRope = 64, kRegsMisc = 80;
 static_assert(2 * kRegsSoftmax + kRegsRope + kRegsMisc == 4 * 128,
               "register split must equal the launch allocation");
 constexpr int kTileBytes = kBlock * kHeadDim * 2;       // 32 KB bf16 tile
@@ -56,14 +56,16 @@ struct FwdCfg {
   // barrier slots
   static constexpr int bQFull = 0, bQReady = 2, bQEmpty = 4, bSFull = 6,
                        bPFull = 8, bOFull = 10, bOEmpty = 12, bEpi = 14,
-                       bDone = 16, bKFull = 17, bKEmpty = bKFull + KS,
+                       bDone = 16, bItemFull = 17, bItemEmpty = 19,
+                       bKFull = 21, bKEmpty = bKFull + KS,
                        bVFull = bKEmpty + KS, bVEmpty = bVFull + VS,
                        kNumBars = bVEmpty + VS;
   static constexpr int kMisc = kBars + kNumBars * 8;
-  static constexpr int kSmem = kMisc + 16 + 1024;  // + alignment slack
+  static constexpr int kSmem = kMisc + 32 + 1024;  // + alignment slack
 };
 
 struct FwdParams {
+  int32_t* counter;
   const int32_t* seg;
   const int32_t* row_start;
   const int32_t* pos;
@@ -210,6 +212,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   auto bar = [&](int i) { return bars + 8u * i; };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMisc + 4);
+  // two-slot ring of work units: the producer takes the next unit from the
+  // global counter (longest first) and every other role reads it from here
+  volatile int* item_slot = reinterpret_cast<volatile int*>(smem + C::kMisc + 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -226,6 +231,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(bar(C::bEpi + s), 128);
     }
     mbar_init(bar(C::bDone), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(C::bItemFull + i), 1);
+      // consumers: 8 softmax warps, 4 RoPE warps, the MMA lane
+      mbar_init(bar(C::bItemEmpty + i), 13);
+    }
     for (int i = 0; i < C::KS; ++i) {
       mbar_init(bar(C::bKFull + i), 1);
       mbar_init(bar(C::bKEmpty + i), 1);
@@ -264,7 +274,15 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     const uint32_t tO = tmem + lane_off + 256 + s * 128;
     int sc = 0, oc = 0;
     bool ok = true;
-    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+    for (int n = 0; ok; ++n) {
+      ok = mbar_wait(bar(C::bItemFull + (n & 1)), (n >> 1) & 1, abort_flag,
+                     p.status, kWaitLimitNs);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      const int it = item_slot[n & 1];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::bItemEmpty + (n & 1)));
+      if (it < 0) break;
       Item m = get_item(p, it);
       if (!m.present[s]) continue;
       const int64_t rowbase = int64_t(m.b) * p.N;
@@ -423,7 +441,15 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int r = threadIdx.x - 8 * 32;  // tile row owned by this thread
     int qcount[2] = {0, 0};
     bool ok = true;
-    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+    for (int n = 0; ok; ++n) {
+      ok = mbar_wait(bar(C::bItemFull + (n & 1)), (n >> 1) & 1, abort_flag,
+                     p.status, kWaitLimitNs);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      const int it = item_slot[n & 1];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::bItemEmpty + (n & 1)));
+      if (it < 0) break;
       Item m = get_item(p, it);
       const int64_t rowbase = int64_t(m.b) * p.N;
       for (int s = 0; s < 2 && ok; ++s) {
@@ -455,7 +481,17 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       int qfill[2] = {0, 0};
       int kfill = 0, vfill = 0;
       bool ok = true;
-      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+      for (int n = 0; ok; ++n) {
+        if (n >= 2) {
+          ok = mbar_wait(bar(C::bItemEmpty + (n & 1)), ((n >> 1) - 1) & 1,
+                         abort_flag, p.status, kWaitLimitNs);
+          if (!ok) break;
+        }
+        int it = atomicAdd(p.counter, 1);
+        if (it >= nitems) it = -1;
+        item_slot[n & 1] = it;
+        mbar_arrive(bar(C::bItemFull + (n & 1)));
+        if (it < 0) break;
         Item m = get_item(p, it);
         for (int s = 0; s < 2 && ok; ++s) {
           if (!m.present[s]) continue;
@@ -524,10 +560,20 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (lane == 0) {
       const uint32_t idS = idesc_bf16(128, 128, 0, 0);
       const uint32_t idPV = idesc_bf16(128, 128, 0, 1);
+      // SW128 descriptors at shared-memory offset 0: K-major (Q, K tiles)
+      // and MN-major with the 64-wide d chunks 16 KB apart (V tiles)
+      const uint64_t kdesc0 = sdesc_sw128(sbase, 16, 1024);
+      const uint64_t vdesc0 = sdesc_sw128(sbase + C::kV, kHalfTileBytes, 1024);
       int kc = 0, vc = 0;
       int qc[2] = {0, 0}, pc[2] = {0, 0}, oc[2] = {0, 0};
       bool ok = true;
-      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+      for (int n = 0; ok; ++n) {
+        ok = mbar_wait(bar(C::bItemFull + (n & 1)), (n >> 1) & 1, abort_flag,
+                       p.status, kWaitLimitNs);
+        if (!ok) break;
+        const int it = item_slot[n & 1];
+        mbar_arrive(bar(C::bItemEmpty + (n & 1)));
+        if (it < 0) break;
         Item m = get_item(p, it);
         bool qwaited[2] = {false, false};
         bool pv_started[2] = {false, false};
@@ -560,16 +606,16 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 if (!ok) break;
               }
               tc_fence_after();
-              const uint32_t vbase = sbase + C::kV + vs * kTileBytes;
+              // descriptor start fields are addr >> 4 in the low 14 bits;
+              // offsets inside shared memory never carry out of them
+              const uint64_t vdesc =
+                  vdesc0 + uint64_t((vs * kTileBytes) >> 4);
               const uint32_t a_tm = tmem + s * 128;        // P over S_s
               const uint32_t d_tm = tmem + 256 + s * 128;  // O_s
 #pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                uint64_t bd = sdesc_sw128(vbase + k * 2048, kHalfTileBytes,
-                                          1024);
-                mma_ts(d_tm, a_tm + k * 8, bd, idPV,
-                       (pv_started[s] || k > 0) ? 1u : 0u);
-              }
+              for (int k = 0; k < 8; ++k)
+                mma_ts(d_tm, a_tm + k * 8, vdesc + uint64_t(k * (2048 >> 4)),
+                       idPV, (pv_started[s] || k > 0) ? 1u : 0u);
               pv_started[s] = true;
             }
             if (has_j && active(m, s, j)) {
@@ -581,22 +627,23 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 qwaited[s] = true;
                 tc_fence_after();
               }
-              const uint32_t qb = sbase + C::kQ + s * kTileBytes;
-              const uint32_t kb = sbase + C::kK + ks * kTileBytes;
+              const uint64_t qd = kdesc0 + uint64_t((C::kQ + s * kTileBytes) >> 4);
+              const uint64_t kd = kdesc0 + uint64_t((C::kK + ks * kTileBytes) >> 4);
               const uint32_t d_tm = tmem + s * 128;
-              int step = 0;
               const int npass = X3 ? 3 : 1;
+#pragma unroll
               for (int pass = 0; pass < npass; ++pass) {
                 // pass 0: hi.hi, 1: hi(Q).lo(K), 2: lo(Q).hi(K)
-                uint32_t qa = qb + (pass == 2 ? (C::kQlo - C::kQ) : 0);
-                uint32_t kbb = kb + (pass == 1 ? (C::kKlo - C::kK) : 0);
+                const uint64_t qa =
+                    qd + uint64_t(pass == 2 ? (C::kQlo - C::kQ) >> 4 : 0);
+                const uint64_t ka =
+                    kd + uint64_t(pass == 1 ? (C::kKlo - C::kK) >> 4 : 0);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                  uint32_t off = (k >> 2) * kHalfTileBytes + (k & 3) * 32;
-                  uint64_t ad = sdesc_sw128(qa + off, 16, 1024);
-                  uint64_t bd = sdesc_sw128(kbb + off, 16, 1024);
-                  mma_ss(d_tm, ad, bd, idS, step > 0 ? 1u : 0u);
-                  ++step;
+                  const uint64_t off =
+                      uint64_t(((k >> 2) * kHalfTileBytes + (k & 3) * 32) >> 4);
+                  mma_ss(d_tm, qa + off, ka + off, idS,
+                         (pass > 0 || k > 0) ? 1u : 0u);
                 }
               }
               mma_commit(bar(C::bSFull + s));
@@ -720,6 +767,7 @@ static cudaError_t launch_fwd_impl(const FwdArgs& a, cudaStream_t st) {
       !make_bnhd_map(&mklo, X3 ? a.k_rot_lo : a.k_rot, a.B, a.N, a.H))
     return cudaErrorInvalidValue;
   FwdParams p{};
+  p.counter = a.counter;
   p.seg = a.seg;
   p.row_start = a.row_start;
   p.pos = a.pos;

@@ -24,6 +24,7 @@ struct FwdArgs {
   const int32_t* kv_lo;
   const int32_t* kv_hi;
   const int32_t* order;
+  int32_t* counter;        // zeroed work counter (units handed out in order)
   const int32_t* row_start;
   const void* k_rot;       // R(pos) k, bf16 [B][N][H][D]
   const void* k_rot_lo;    // bf16 residual of k_rot (split-QK mode)
@@ -45,6 +46,7 @@ struct BwdArgs {
   const int32_t* q_lo;
   const int32_t* q_hi;
   const int32_t* order;
+  int32_t* counter;
   const int32_t* row_start;
   const int32_t* row_end;
   void* q_rot;             // scratch for R(pos) q, bf16 [B][N][H][D]
