@@ -7,14 +7,16 @@
 // and visits every 128-query block that can see it (the queries of the same
 // packed example at or after the key). Per query block i, with P recomputed
 // from the forward's logsumexp (scores in log2 units):
-//   S^T  = K~ Q~_i^T            (tcgen05, TMEM cols   0..127)
-//   dP^T = V dO_i^T             (tcgen05, TMEM cols 128..255)
-//   P^T  = 2^(S^T c - lse_i log2 e) (masked), dS^T = P^T (dP^T - D_i)
-//          written back as bf16 over the first 64 columns of each region
+//   S^T  = K~ Q~_i^T            (tcgen05, TMEM region A, cols   0..127)
+//   dP^T = V dO_i^T             (tcgen05, TMEM region B, cols 128..255)
+//   P^T  = 2^(S^T c - lse_i log2 e) (masked; computed as soon as S^T lands,
+//          while dP^T is still on the tensor pipe), dS^T = P^T (dP^T - D_i)
+//          written back as bf16 over the first 64 columns of A and B
 //   dV  += P^T dO_i, dK~ += dS^T Q~_i   (A operands read from TMEM)
 //   dQ~_i = dS K~               (A = dS, staged in shared memory; result in
-//          TMEM cols 0..127, added to an fp32 accumulator in global memory
-//          by TMA reduce-add from the then-dead dS buffer)
+//          region B once dK has read dS^T, so region A is free for the next
+//          S^T at once; added to an fp32 accumulator in global memory by
+//          TMA reduce-add, staged in the block's then-dead Q~/dO buffers)
 // Queries and keys arrive pre-rotated (R(pos) q, R(pos) k); dK = R(-pos)
 // (dK~ / sqrt(D)) in the epilogue, dQ the same in the conversion kernel.
 //
@@ -44,7 +46,7 @@ constexpr int kSK = 0, kSV = kTile, kSQ = 2 * kTile, kSDO = 4 * kTile,
               kSBars = kSAux + 4 * 128 * 4;
 enum {
   bKVFull = 0, bKVEmpty, bQFull0, bQFull1, bQEmpty0, bQEmpty1, bAux0, bAux1,
-  bSFull, bPFull, bDqFull, bDqEmpty, bAccFull, bAccEmpty, bDoneB, bDsFree,
+  bStFull, bDptFull, bPFull, bDqFull, bDqEmpty, bAccFull, bAccEmpty, bDoneB, bDsFree,
   bItemFull0, bItemFull1, bItemEmpty0, bItemEmpty1, kNumBarsB
 };
 constexpr int kSMisc = kSBars + kNumBarsB * 8;
@@ -121,18 +123,20 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(bar(bKVEmpty), 1);
     mbar_init(bar(bQFull0), 1);
     mbar_init(bar(bQFull1), 1);
-    mbar_init(bar(bQEmpty0), 1);
-    mbar_init(bar(bQEmpty1), 1);
+    // a Q~/dO stage is free once its MMAs are done (one commit) and the dQ
+    // warps have reduced dQ of that block out of it (one arrive per warp)
+    mbar_init(bar(bQEmpty0), 5);
+    mbar_init(bar(bQEmpty1), 5);
     mbar_init(bar(bAux0), 128);
     mbar_init(bar(bAux1), 128);
-    mbar_init(bar(bSFull), 1);
+    mbar_init(bar(bStFull), 1);
+    mbar_init(bar(bDptFull), 1);
     mbar_init(bar(bPFull), 4);
     mbar_init(bar(bDqFull), 1);
     mbar_init(bar(bDqEmpty), 4);
     mbar_init(bar(bAccFull), 1);
     mbar_init(bar(bAccEmpty), 4);
     mbar_init(bar(bDoneB), 1);
-    mbar_init(bar(bDsFree), 4);
     mbar_init(bar(bItemFull0), 1);
     mbar_init(bar(bItemFull1), 1);
     // consumers: 4 compute warps, 4 dQ warps, the MMA lane
@@ -185,7 +189,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       const int re_k0 = __ldg(p.row_end + rowbase + k0);
       for (int i = m.qlo; i <= m.qhi && ok; ++i) {
         const int st = g & 1;
-        ok = mbar_wait(bar(bSFull), g & 1, abort_flag, p.status, kWaitNs);
+        ok = mbar_wait(bar(bStFull), g & 1, abort_flag, p.status, kWaitNs);
         if (ok)
           ok = mbar_wait(bar(bAux0 + st), (g >> 1) & 1, abort_flag, p.status,
                          kWaitNs);
@@ -197,15 +201,15 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         const float* ls = aux_lse + st * 128;
         const float* dl = aux_del + st * 128;
         uint8_t* dsrow = smem + kSDS + r * 128;
-        bool ds_ready = g == 0;  // the dS buffer also stages dQ of block g-1
+        // phase 1 (while dP^T is still on the tensor pipe):
+        // P^T = 2^(S^T c - lse log2 e), masked; bf16 copy over S^T
+        float pf[4][32];
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          uint32_t sv[2][32], dv[2][32];
+          uint32_t sv[2][32];
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
+          for (int cc = 0; cc < 2; ++cc)
             tmem_ld32(tA + lane_off + (2 * half + cc) * 32, sv[cc]);
-            tmem_ld32(tB + lane_off + (2 * half + cc) * 32, dv[cc]);
-          }
           tmem_wait_ld();
           if (!full) {
 #pragma unroll
@@ -220,31 +224,58 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
           for (int cc = 0; cc < 2; ++cc) {
             const int c = 2 * half + cc;
-            uint32_t pp[16], pd[16];
+            uint32_t pp[16];
 #pragma unroll
-            for (int x = 0; x < 32; x += 2) {
-              const float4 l4 = *reinterpret_cast<const float4*>(ls + c * 32 + (x & ~3));
-              const float4 d4 = *reinterpret_cast<const float4*>(dl + c * 32 + (x & ~3));
-              const float la = (x & 3) ? l4.z : l4.x, lb = (x & 3) ? l4.w : l4.y;
-              const float da = (x & 3) ? d4.z : d4.x, db = (x & 3) ? d4.w : d4.y;
-              const float2 t = fma2(make_float2(__uint_as_float(sv[cc][x]),
-                                                __uint_as_float(sv[cc][x + 1])),
-                                    make_float2(p.scale_log2, p.scale_log2),
-                                    make_float2(-la, -lb));
-              const float p0 = ex2(t.x), p1 = ex2(t.y);
-              const float ds0 = p0 * (__uint_as_float(dv[cc][x]) - da);
-              const float ds1 = p1 * (__uint_as_float(dv[cc][x + 1]) - db);
-              pp[x >> 1] = pack_bf16x2(p0, p1);
-              pd[x >> 1] = pack_bf16x2(ds0, ds1);
+            for (int x = 0; x < 32; x += 4) {
+              const float4 l4 = *reinterpret_cast<const float4*>(ls + c * 32 + x);
+              const float2 t0 = fma2(make_float2(__uint_as_float(sv[cc][x]),
+                                                 __uint_as_float(sv[cc][x + 1])),
+                                     make_float2(p.scale_log2, p.scale_log2),
+                                     make_float2(-l4.x, -l4.y));
+              const float2 t1 = fma2(make_float2(__uint_as_float(sv[cc][x + 2]),
+                                                 __uint_as_float(sv[cc][x + 3])),
+                                     make_float2(p.scale_log2, p.scale_log2),
+                                     make_float2(-l4.z, -l4.w));
+              pf[c][x] = ex2(t0.x);
+              pf[c][x + 1] = ex2(t0.y);
+              pf[c][x + 2] = ex2(t1.x);
+              pf[c][x + 3] = ex2(t1.y);
+              pp[x >> 1] = pack_bf16x2(pf[c][x], pf[c][x + 1]);
+              pp[(x >> 1) + 1] = pack_bf16x2(pf[c][x + 2], pf[c][x + 3]);
             }
             tmem_st16(tA + lane_off + c * 16, pp);
-            tmem_st16(tB + lane_off + c * 16, pd);
-            if (!ds_ready) {
-              bool w = mbar_wait(bar(bDsFree), (g - 1) & 1, abort_flag,
-                                 p.status, kWaitNs);
-              ds_ready = true;
-              if (!__all_sync(0xffffffffu, w)) ok = false;
+          }
+        }
+        // phase 2: dS^T = P^T (dP^T - D) once dP^T has landed
+        ok = mbar_wait(bar(bDptFull), g & 1, abort_flag, p.status, kWaitNs);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) {
+          tmem_wait_st();
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t dv[2][32];
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc)
+            tmem_ld32(tB + lane_off + (2 * half + cc) * 32, dv[cc]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            const int c = 2 * half + cc;
+            uint32_t pd[16];
+#pragma unroll
+            for (int x = 0; x < 32; x += 4) {
+              const float4 d4 = *reinterpret_cast<const float4*>(dl + c * 32 + x);
+              const float ds0 = pf[c][x] * (__uint_as_float(dv[cc][x]) - d4.x);
+              const float ds1 = pf[c][x + 1] * (__uint_as_float(dv[cc][x + 1]) - d4.y);
+              const float ds2 = pf[c][x + 2] * (__uint_as_float(dv[cc][x + 2]) - d4.z);
+              const float ds3 = pf[c][x + 3] * (__uint_as_float(dv[cc][x + 3]) - d4.w);
+              pd[x >> 1] = pack_bf16x2(ds0, ds1);
+              pd[(x >> 1) + 1] = pack_bf16x2(ds2, ds3);
             }
+            tmem_st16(tB + lane_off + c * 16, pd);
             // dS row r, queries c*32 .. c*32+31: query half (c >> 1),
             // 16-byte chunks (c & 1) * 4 .. +3 of that 128-byte row
 #pragma unroll
@@ -258,7 +289,6 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
         }
         tmem_wait_st();
-        if (!ok) break;
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
@@ -331,11 +361,13 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     bool ok = true;
     int pb = 0, ph = 0, pq0 = 0;  // the block whose dQ is pending
     // dQ of block t: TMEM -> registers (then TMEM is free for the next
-    // S^T), registers -> the dead dS buffer (this warp's 32 rows, two
-    // 32-column chunks of 4 KB at a time, 128-byte swizzle), then a TMA
-    // reduce-add of each chunk into the fp32 accumulator.
+    // dP^T), registers -> the block's own Q~ and dO stage buffers, which
+    // its MMAs no longer read (this warp's 32 rows as four 32-column 4 KB
+    // boxes, 128-byte swizzle), then a TMA reduce-add of each box into the
+    // fp32 accumulator; the stage goes back to the producer after the
+    // reduce has read it.
     const int wq = warp - 4;
-    const uint32_t stage = sbase + kSDS + wq * 8192;
+    int pst = 0;  // stage of the pending block
     auto flush = [&](int t) -> bool {
       bool w = mbar_wait(bar(bDqFull), t & 1, abort_flag, p.status, kWaitNs);
       w = __all_sync(0xffffffffu, w);
@@ -343,36 +375,36 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       tc_fence_after();
       uint32_t v[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tA + lane_off + c * 32, v[c]);
+      for (int c = 0; c < 4; ++c) tmem_ld32(tB + lane_off + c * 32, v[c]);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(bDqEmpty));
+      const int qoff = kSQ + pst * kTile, ooff = kSDO + pst * kTile;
 #pragma unroll
-      for (int round = 0; round < 2; ++round) {
+      for (int c = 0; c < 4; ++c) {
+        const int box = (c < 2 ? qoff : ooff) + (wq * 2 + (c & 1)) * 4096;
+        uint8_t* rowp = smem + box + lane * 128;
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int c = 2 * round + cc;
-          uint8_t* rowp = smem + kSDS + wq * 8192 + cc * 4096 + lane * 128;
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            *reinterpret_cast<uint4*>(rowp + ((e ^ (lane & 7)) << 4)) =
-                make_uint4(v[c][4 * e], v[c][4 * e + 1], v[c][4 * e + 2],
-                           v[c][4 * e + 3]);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-#pragma unroll
-          for (int cc = 0; cc < 2; ++cc)
-            tma_reduce_add_4d(&tm_dq, stage + cc * 4096, (2 * round + cc) * 32,
-                              ph, pq0 + wq * 32, pb);
-          bulk_commit();
-          bulk_wait_read0();
-        }
-        __syncwarp();
+        for (int e = 0; e < 8; ++e)
+          *reinterpret_cast<uint4*>(rowp + ((e ^ (lane & 7)) << 4)) =
+              make_uint4(v[c][4 * e], v[c][4 * e + 1], v[c][4 * e + 2],
+                         v[c][4 * e + 3]);
       }
-      if (lane == 0) mbar_arrive(bar(bDsFree));
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int box = (c < 2 ? qoff : ooff) + (wq * 2 + (c & 1)) * 4096;
+          tma_reduce_add_4d(&tm_dq, sbase + box, c * 32, ph, pq0 + wq * 32,
+                            pb);
+        }
+        bulk_commit();
+        bulk_wait_read0();
+        mbar_arrive(bar(bQEmpty0 + pst));
+      }
+      __syncwarp();
       return true;
     };
     for (int u = 0; ok; ++u) {
@@ -399,6 +431,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         pb = m.b;
         ph = m.h;
         pq0 = i * kBlock;
+        pst = st;
         ++g;
       }
     }
@@ -486,26 +519,32 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           const int st = g & 1;
           ok = mbar_wait(bar(bQFull0 + st), (g >> 1) & 1, abort_flag,
                          p.status, kWaitNs);
-          if (ok && g > 0)
-            ok = mbar_wait(bar(bDqEmpty), (g - 1) & 1, abort_flag, p.status,
-                           kWaitNs);
           if (!ok) break;
           tc_fence_after();
           const uint32_t qb = sbase + kSQ + st * kTile;
           const uint32_t ob = sbase + kSDO + st * kTile;
+          // S^T = K~ Q~^T into A: A's last readers (dV of block g-1, the
+          // compute warps' loads) are done by issue order / p_full
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {  // S^T = K~ Q~^T
+          for (int k = 0; k < 8; ++k) {
             const uint32_t off = (k >> 2) * kHalf + (k & 3) * 32;
             mma_ss(tA, sdesc_sw128(sbase + kSK + off, 16, 1024),
                    sdesc_sw128(qb + off, 16, 1024), idKK, k > 0 ? 1u : 0u);
           }
+          mma_commit(bar(bStFull));
+          // dP^T = V dO^T into B once dQ of block g-1 has left it
+          if (g > 0)
+            ok = mbar_wait(bar(bDqEmpty), (g - 1) & 1, abort_flag, p.status,
+                           kWaitNs);
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {  // dP^T = V dO^T
+          for (int k = 0; k < 8; ++k) {
             const uint32_t off = (k >> 2) * kHalf + (k & 3) * 32;
             mma_ss(tB, sdesc_sw128(sbase + kSV + off, 16, 1024),
                    sdesc_sw128(ob + off, 16, 1024), idKK, k > 0 ? 1u : 0u);
           }
-          mma_commit(bar(bSFull));
+          mma_commit(bar(bDptFull));
           ok = mbar_wait(bar(bPFull), g & 1, abort_flag, p.status, kWaitNs);
           if (ok && first_q && n > 0)
             ok = mbar_wait(bar(bAccEmpty), (n - 1) & 1, abort_flag, p.status,
@@ -521,8 +560,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             mma_ts(tD, tB + 8 * k, sdesc_sw128(qb + 2048 * k, kHalf, 1024),
                    idKM, (!first_q || k > 0) ? 1u : 0u);
 #pragma unroll
-          for (int k = 0; k < 8; ++k)  // dQ~ = dS K~
-            mma_ss(tA, sdesc_sw128(sbase + kSDS + 2048 * k, kHalf, 1024),
+          for (int k = 0; k < 8; ++k)  // dQ~ = dS K~, into B after dK read it
+            mma_ss(tB, sdesc_sw128(sbase + kSDS + 2048 * k, kHalf, 1024),
                    sdesc_sw128(sbase + kSK + 2048 * k, kHalf, 1024), idMM,
                    k > 0 ? 1u : 0u);
           mma_commit(bar(bDqFull));
