@@ -187,17 +187,10 @@ def oracle_sample(w, t_host, budget_s, backward):
 
 # ------------------------------------------------------------------ main
 
-def init_dist():
-    ws = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if ws > 1:
-        import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group(
-            "nccl", timeout=datetime.timedelta(seconds=120),
-            device_id=torch.device("cuda", local))
-    return ws, rank, local
+def init_dist(impl):
+    from long_context_blockwise_causal_b200 import dist
+    # the reference arm runs on host cores only: no NCCL, no GPU
+    return dist.init_from_env("gloo" if impl == "reference" else "nccl")
 
 
 def barrier(ws):
@@ -206,11 +199,8 @@ def barrier(ws):
 
 
 def max_over_ranks(x, ws, dev):
-    if ws == 1:
-        return x
-    t = torch.tensor([x], dtype=torch.float64, device=dev)
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    return float(t.item())
+    from long_context_blockwise_causal_b200 import dist
+    return dist.max_over_ranks(x, ws, dev)
 
 
 def reference_arm(args, ws, rank):
@@ -258,6 +248,9 @@ def main():
                     help="override the workload's head count (profiling)")
     ap.add_argument("--B", type=int, default=None,
                     help="override the workload's batch rows (profiling)")
+    ap.add_argument("--shard", default="replica", choices=["replica", "heads"],
+                    help="N>1: each rank runs a full replica (weak scaling) or "
+                         "a slice of the heads of one job (strong scaling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
@@ -265,12 +258,12 @@ def main():
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
-    ws, rank, local = init_dist()
     if args.impl == "reference":
-        reference_arm(args, ws, rank)
-        if ws > 1:
-            torch.distributed.destroy_process_group()
+        # host cores only: rank 0 runs the oracle, other ranks have no work
+        rank = int(os.environ.get("RANK", "0"))
+        reference_arm(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
         return
+    ws, rank, local = init_dist(args.impl)
 
     from long_context_blockwise_causal_b200 import ops
 
@@ -282,12 +275,23 @@ def main():
         w = wl.Workload(w.name + "-reduced", args.B or w.B, args.N or w.N,
                         args.H or w.H, w.D, w.theta, w.segments, w.scale,
                         w.backward, seg_args=w.seg_args)
-    t = wl.make_inputs(w, args.seed + 1000 * rank, device=dev,
-                       with_dout=w.backward)
+    job_heads = w.H
+    if args.shard == "heads" and ws > 1:
+        from long_context_blockwise_causal_b200 import dist
+        h0, h1 = dist.head_shard(w.H, ws, rank)
+        t = wl.make_inputs(w, args.seed, device=dev, H=h1 - h0,
+                           with_dout=w.backward)
+    else:
+        t = wl.make_inputs(w, args.seed + 1000 * rank, device=dev,
+                           with_dout=w.backward)
     B, N, H, D = t["q"].shape
     pairs_per_head = wl.visible_pairs(t["lengths"])
     fwd_flop = 4.0 * D * pairs_per_head * H
     bwd_flop = 10.0 * D * pairs_per_head * H if w.backward else 0.0
+    strong = args.shard == "heads" and ws > 1
+    # whole-job work: replicas multiply it by the rank count, a head-sharded
+    # job is one workload split across the ranks
+    job_scale = (job_heads / H) if strong else ws
     max_pos = int(t["positions"].max().item()) + 1
     ws_bytes = max(ops.fwd_workspace_size(B, N, H, max_pos,
                                           qk_precision=qkp),
@@ -384,9 +388,9 @@ def main():
         e2.record(stream)
         torch.cuda.synchronize(dev)
         ems = max_over_ranks(s2.elapsed_time(e2) / ksteps, ws, dev)
-        e2e = {"value": (fwd_flop + bwd_flop) * ws / (ems / 1e3) / 1e12,
+        e2e = {"value": (fwd_flop + bwd_flop) * job_scale / (ems / 1e3) / 1e12,
                "unit": "TFLOP/s", "ms_per_step": ems,
-               "tokens_per_s": B * N * ws / (ems / 1e3),
+               "tokens_per_s": B * N * (1 if strong else ws) / (ems / 1e3),
                "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h)}
 
@@ -401,7 +405,7 @@ def main():
 
     if rank == 0:
         pk = peaks()
-        total_flop = (fwd_flop + bwd_flop) * ws
+        total_flop = (fwd_flop + bwd_flop) * job_scale
         value = total_flop / (ms / 1e3) / 1e12
         peak_burst = pk["bf16_tflops"]
         peak_sus = pk.get("bf16_tflops_sustained", peak_burst)
@@ -412,17 +416,20 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s",
             "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "strong" if strong else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "B": B, "N": N, "H": H, "D": D,
+            "config": {"workload": w.name, "B": B, "N": N, "H": job_heads,
+                       "heads_per_rank": H, "D": D,
                        "theta": w.theta, "qk_precision": qkp,
                        "segments": w.segments,
                        "visible_pairs_per_head": pairs_per_head,
                        "l2": "inputs larger than L2 (no flush)"
                        if 3 * t["q"].numel() * 2 > 126e6 else
                        "inputs smaller than L2 (re-read from L2)",
-                       "parallelism": f"replicas x{ws}"},
-            "tokens_per_s": B * N * ws / (ms / 1e3),
+                       "parallelism": (f"heads split over {ws} GPUs" if strong
+                                       else f"replicas x{ws}")},
+            "tokens_per_s": B * N * (1 if strong else ws) / (ms / 1e3),
             "fwd": {"ms": fwd_ms, "tflops": fwd_tf,
                     "frac_of_burst_peak": fwd_tf / peak_burst},
             "bwd": ({"ms": bwd_ms, "tflops": bwd_tf,
