@@ -233,6 +233,80 @@ def reference_arm(args, ws, rank):
     print(json.dumps(line), flush=True)
 
 
+DECODE_WORKLOADS = {
+    # one query token per (row, head) against a cache of L keys, one example
+    "decode1m": {"B": 1, "L": 1 << 20, "H": 32, "theta": 5e7},
+    "decode128k_b16": {"B": 16, "L": 1 << 17, "H": 32, "theta": 1e7},
+}
+
+
+def bench_decode(args):
+    """Decode attention: HBM-bound (every visible key and value row is read
+    once). Prints one JSON line with GB/s against the measured copy
+    bandwidth."""
+    from long_context_blockwise_causal_b200 import ops
+    cfg = DECODE_WORKLOADS[args.workload]
+    B, L, H, D = cfg["B"], cfg["L"], cfg["H"], 128
+    dev = torch.device("cuda", 0)
+    scale = 1.0 / math.sqrt(D)
+    k = wl.random_tensor((B, L, H, D), args.seed * 16 + 2, scale,
+                         torch.bfloat16, dev)
+    v = wl.random_tensor((B, L, H, D), args.seed * 16 + 3, scale,
+                         torch.bfloat16, dev)
+    q = wl.random_tensor((B, 1, H, D), args.seed * 16 + 1, scale,
+                         torch.bfloat16, dev)[:, 0].contiguous()
+    pos = torch.arange(L, dtype=torch.int32, device=dev).repeat(B, 1)
+    table = ops.rope_table(cfg["theta"], L, device=dev)
+    k_rot = ops.rope_apply(k, pos, table)
+    del k
+    kv_start = torch.zeros(B, dtype=torch.int32, device=dev)
+    kv_len = torch.full((B,), L, dtype=torch.int32, device=dev)
+    q_pos = torch.full((B,), L - 1, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H), dtype=torch.float32, device=dev)
+    ws = torch.empty(ops.decode_workspace_size(B, H, L), dtype=torch.uint8,
+                     device=dev)
+    step = lambda: ops.decode(q, k_rot, v, kv_start, kv_len, q_pos, table,
+                              out=out, lse=lse, workspace=ws)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev)
+    clocks.start()
+    time.sleep(0.3)
+    l0 = ops.kernel_launches()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    launches = ops.kernel_launches() - l0
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    nbytes = B * H * L * D * 2 * 2 + B * H * D * 4  # K, V rows + q, out
+    gbs = nbytes / (ms / 1e3) / 1e9
+    pk = peaks()
+    line = {"metric": "decode attention HBM GB/s (1 query token per row and "
+                      "head against the cache)",
+            "value": gbs, "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, "B": B, "L": L, "H": H,
+                       "D": D, "l2": "cache larger than L2"},
+            "tokens_per_s": B / (ms / 1e3),
+            "roofline": {"bound": "hbm", "kernel": "decode_split_kernel",
+                         "achieved": gbs, "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
+                         "traffic": None,
+                         "peak_kind": f"copy bandwidth ({pk['source']})"},
+            "gpu_launches": int(launches), "device_status": ops.last_status(),
+            "clocks": clk}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -240,7 +314,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="text32k",
-                    choices=sorted(wl.WORKLOADS))
+                    choices=sorted(wl.WORKLOADS) + sorted(DECODE_WORKLOADS))
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--N", type=int, default=None,
                     help="override the workload's sequence length (profiling)")
@@ -258,6 +332,10 @@ def main():
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
+    if args.workload in DECODE_WORKLOADS:
+        if args.impl != "reference":
+            bench_decode(args)
+        return
     if args.impl == "reference":
         # host cores only: rank 0 runs the oracle, other ranks have no work
         rank = int(os.environ.get("RANK", "0"))

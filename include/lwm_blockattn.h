@@ -180,6 +180,45 @@ LWM_API const char* lwm_status_string(int status);
 /* LWM_BLOCKATTN_VERSION of the built library. */
 LWM_API int lwm_blockattn_version(void);
 
+/* ---------------------------------------------------------------------
+ * Decode (inference against a long KV cache).
+ *
+ * lwm_blockattn_rope_apply: x_rot = R(pos) x for a bf16 [B][N][H][D] tensor
+ * (D == 128, interleaved pairs), using a table made by
+ * lwm_blockattn_rope_table for positions [0, max_pos). Rotating keys once as
+ * they enter a cache lets decode read them as they are. Async on stream.
+ * Returns LWM_OK or an error status (nothing launched on error). */
+LWM_API int lwm_blockattn_rope_apply(const void* x, const int32_t* positions,
+                                     const float* rope_table, int max_pos,
+                                     int B, int N, int H, int D, int dtype,
+                                     void* x_rot, void* stream);
+
+/* Bytes of workspace lwm_blockattn_decode needs (per-chunk partial sums). */
+LWM_API size_t lwm_blockattn_decode_workspace_size(int B, int H, int D,
+                                                   int L);
+
+/* One query token per (b, h) against a cache of L tokens.
+ *   q        [B][H][D] bf16, un-rotated; rotated here by R(q_pos[b])
+ *   k_rot    [B][L][H][D] bf16, keys already rotated (rope_apply)
+ *   v        [B][L][H][D] bf16
+ *   kv_start, kv_len [B] int32: the query sees cached keys
+ *            [kv_start[b], kv_len[b]) (its own packed example: the query is
+ *            the example's last token); values outside [0, L] are clamped
+ *   q_pos    [B] int32 RoPE position of the query, in [0, max_pos)
+ *   rope_table from lwm_blockattn_rope_table (max_pos positions)
+ *   out      [B][H][D] bf16;  lse [B][H] fp32 natural log (-inf if the
+ *            range is empty, with out = 0)
+ * Split over key chunks (partials in the workspace), then merged; reads
+ * each visible key and value row once. Only dtype LWM_DTYPE_BF16. Async on
+ * stream. */
+LWM_API int lwm_blockattn_decode(const void* q, const void* k_rot,
+                                 const void* v, const int32_t* kv_start,
+                                 const int32_t* kv_len, const int32_t* q_pos,
+                                 const float* rope_table, int max_pos, int B,
+                                 int L, int H, int D, int dtype, void* out,
+                                 float* lse, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
 /* Self-test of the failure path: launches one small CTA that waits on an
  * mbarrier nobody arrives on, with the same bounded wait the attention
  * kernels use and a limit of limit_ns nanoseconds (clamped to [1 ms, 2 s]).

@@ -6,6 +6,7 @@
 #include <cstring>
 
 #include "aux_kernels.cuh"
+#include "decode.cuh"
 #include "tc_kernels.cuh"
 
 namespace lwm {
@@ -170,6 +171,62 @@ const char* lwm_status_string(int status) {
 }
 
 int lwm_blockattn_version(void) { return LWM_BLOCKATTN_VERSION; }
+
+int lwm_blockattn_rope_apply(const void* x, const int32_t* positions,
+                             const float* rope_table, int max_pos, int B,
+                             int N, int H, int D, int dtype, void* x_rot,
+                             void* stream) {
+  if (B < 0 || N < 0 || H < 0 || max_pos < 0 ||
+      (int64_t(B) * N) >= (int64_t(1) << 31))
+    return LWM_ERR_INVALID_ARG;
+  if (D != kHeadDim) return LWM_ERR_UNSUPPORTED;
+  if (dtype != LWM_DTYPE_BF16) return LWM_ERR_UNSUPPORTED;
+  if (int64_t(B) * N * H == 0) return LWM_OK;
+  const void* ptrs[] = {x, positions, rope_table, x_rot};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return LWM_ERR_INVALID_ARG;
+  if (max_pos < 1) return LWM_ERR_INVALID_ARG;
+  return cuda_status(launch_rope_apply(x, positions, rope_table, B, N, H,
+                                       x_rot, nullptr,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+size_t lwm_blockattn_decode_workspace_size(int B, int H, int D, int L) {
+  if (B < 0 || H < 0 || D != kHeadDim || L < 0) return 0;
+  const size_t slots = size_t(B) * H * decode_splits(L);
+  return align_up(slots * sizeof(float)) * 2 +
+         align_up(slots * kHeadDim * sizeof(float));
+}
+
+int lwm_blockattn_decode(const void* q, const void* k_rot, const void* v,
+                         const int32_t* kv_start, const int32_t* kv_len,
+                         const int32_t* q_pos, const float* rope_table,
+                         int max_pos, int B, int L, int H, int D, int dtype,
+                         void* out, float* lse, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  if (B < 0 || L < 0 || H < 0 || max_pos < 0 ||
+      (int64_t(B) * L) >= (int64_t(1) << 31))
+    return LWM_ERR_INVALID_ARG;
+  if (D != kHeadDim || dtype != LWM_DTYPE_BF16) return LWM_ERR_UNSUPPORTED;
+  if (int64_t(B) * H == 0) return LWM_OK;
+  const void* ptrs[] = {q, k_rot, v, kv_start, kv_len, q_pos, rope_table,
+                        out, lse, workspace};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return LWM_ERR_INVALID_ARG;
+  if (max_pos < 1) return LWM_ERR_INVALID_ARG;
+  const size_t need = lwm_blockattn_decode_workspace_size(B, H, D, L);
+  if (workspace_bytes < need) return LWM_ERR_WORKSPACE;
+  const size_t slots = size_t(B) * H * decode_splits(L);
+  char* ws = static_cast<char*>(workspace);
+  float* part_m = reinterpret_cast<float*>(ws);
+  float* part_l = reinterpret_cast<float*>(ws + align_up(slots * sizeof(float)));
+  float* part_acc =
+      reinterpret_cast<float*>(ws + 2 * align_up(slots * sizeof(float)));
+  return cuda_status(launch_decode(q, k_rot, v, kv_start, kv_len, q_pos,
+                                   rope_table, max_pos, B, L, H, out, lse,
+                                   part_m, part_l, part_acc,
+                                   static_cast<cudaStream_t>(stream)));
+}
 
 int lwm_blockattn_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
   if (limit_ns < 1000000ull) limit_ns = 1000000ull;

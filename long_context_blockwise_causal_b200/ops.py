@@ -50,6 +50,11 @@ _SIGS = {
     "lwm_blockattn_version": (_i, []),
     "lwm_blockattn_kernel_launches": (ctypes.c_uint64, []),
     "lwm_blockattn_selftest_wait_timeout": (_i, [ctypes.c_uint64, _vp]),
+    "lwm_blockattn_rope_apply": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                                      _vp, _vp]),
+    "lwm_blockattn_decode_workspace_size": (_sz, [_i, _i, _i, _i]),
+    "lwm_blockattn_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i,
+                                  _i, _i, _i, _i, _vp, _vp, _vp, _sz, _vp]),
     "lwm_blockattn_fwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _d, _i, _i,
                                        _i, _i, _i, _i, _i, _i, _i, _vp, _vp,
                                        _vp]),
@@ -247,6 +252,42 @@ def rope_table(theta, max_pos, D=HEAD_DIM, device="cuda", stream=None):
                                         _stream(stream))
     _check(st, "lwm_blockattn_rope_table")
     return t
+
+
+def rope_apply(x, positions, table, stream=None, out=None):
+    """R(pos) x (bf16 [B,N,H,D]) with a table from rope_table()."""
+    _need_cuda(x, positions, table, out)
+    B, N, H, D = x.shape
+    out = torch.empty_like(x) if out is None else out
+    st = lib().lwm_blockattn_rope_apply(
+        _ptr(x), _ptr(positions), _ptr(table), table.shape[0], B, N, H, D,
+        _dtype_code(x), _ptr(out), _stream(stream))
+    _check(st, "lwm_blockattn_rope_apply")
+    return out
+
+
+def decode_workspace_size(B, H, L, D=HEAD_DIM) -> int:
+    return int(lib().lwm_blockattn_decode_workspace_size(B, H, D, L))
+
+
+def decode(q, k_rot, v, kv_start, kv_len, q_pos, table, out=None, lse=None,
+           workspace=None, stream=None):
+    """One query token per (b, h) [B,H,D] against a cache of rotated keys
+    and values [B,L,H,D]; returns (out [B,H,D], lse [B,H])."""
+    _need_cuda(q, k_rot, v, kv_start, kv_len, q_pos, table, out, lse,
+               workspace)
+    B, H, D = q.shape
+    L = k_rot.shape[1]
+    out = torch.empty_like(q) if out is None else out
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    ws = _workspace(decode_workspace_size(B, H, L, D), q.device, workspace)
+    st = lib().lwm_blockattn_decode(
+        _ptr(q), _ptr(k_rot), _ptr(v), _ptr(kv_start), _ptr(kv_len),
+        _ptr(q_pos), _ptr(table), table.shape[0], B, L, H, D, _dtype_code(q),
+        _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "lwm_blockattn_decode")
+    return out, lse
 
 
 def check_inputs(segment_ids, positions, max_pos, stream=None):
