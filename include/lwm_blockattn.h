@@ -134,6 +134,52 @@ LWM_API int lwm_blockattn_bwd(const void* q, const void* k, const void* v,
                       void* dq, void* dk, void* dv,
                       void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---------------------------------------------------------------------
+ * Ring attention building blocks ("开源巨兽LWM：如何用RingAttention撬动百万
+ * Token多模态世界", 3.1 RingAttention: each device keeps its query block,
+ * key/value blocks pass around a ring of devices, and each step's partial
+ * attention is folded into the running result with the log-sum-exp rule).
+ *
+ * Bytes of workspace lwm_blockattn_fwd_block needs: RoPE table and the
+ * per-row / per-block metadata of Nq queries against Nk keys. */
+LWM_API size_t lwm_blockattn_fwd_block_workspace_size(int B, int Nq, int Nk,
+                                                      int H, int D,
+                                                      int max_pos);
+
+/* Partial forward of query rows [q_off, q_off+Nq) of a packed sequence
+ * against its key/value rows [k_off, k_off+Nk) (global token indices; the
+ * two ranges may be any pieces of the same sequence). Row i sees key j iff
+ * j <= i and seg_q[i] == seg_k[j]; rows with no visible key get out = 0,
+ * lse = -inf.
+ *   q      [B][Nq][H][D] bf16, un-rotated; rotated here by R(pos_q)
+ *   k_rot  [B][Nk][H][D] bf16, keys already rotated (lwm_blockattn_rope_apply
+ *          with their own positions)
+ *   v      [B][Nk][H][D] bf16
+ *   seg_q  [B][Nq], pos_q [B][Nq], seg_k [B][Nk] int32; segment ids
+ *          non-decreasing along the whole sequence
+ *   out    [B][Nq][H][D] bf16, lse [B][H][Nq] fp32 (natural log), written
+ *          (not accumulated): fold them into a running result with
+ *          lwm_blockattn_merge.
+ * D == 128, bf16 only. Async on stream; nothing launched on error. */
+LWM_API int lwm_blockattn_fwd_block(const void* q, const void* k_rot,
+                                    const void* v, const int32_t* seg_q,
+                                    const int32_t* pos_q, const int32_t* seg_k,
+                                    int q_off, int k_off, double theta,
+                                    int max_pos, int B, int Nq, int Nk, int H,
+                                    int D, void* out, float* lse,
+                                    void* workspace, size_t workspace_bytes,
+                                    void* stream);
+
+/* In place: (out, lse) <- the attention over the union of two disjoint key
+ * sets, given (out, lse) over one and (out_part, lse_part) over the other:
+ * with w = exp(lse - M), w' = exp(lse_part - M), M = max(lse, lse_part),
+ * out = (w out + w' out_part) / (w + w'), lse = M + log(w + w').
+ * Rows where both lse are -inf stay (0, -inf). Shapes as in
+ * lwm_blockattn_fwd_block (N rows); D == 128, bf16 only. Async on stream. */
+LWM_API int lwm_blockattn_merge(void* out, float* lse, const void* out_part,
+                                const float* lse_part, int B, int N, int H,
+                                int D, int dtype, void* stream);
+
 /* Tile classifier (exported so it can be checked bit-exactly). For each
  * batch row b and query block t (Tq = ceil(N/block_q) blocks), key blocks
  * j (Tk = ceil(N/block_k)):

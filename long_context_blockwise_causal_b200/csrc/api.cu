@@ -54,16 +54,22 @@ struct Carve {
   }
 };
 
-// Workspace regions shared by forward and backward.
+enum class Pass { kFwd, kFwdBlock, kBwd };
+
+// Workspace regions (a pass carves only what it uses).
 struct Workspace {
   float* table;          // [max_pos][D/2] float2
   int32_t* kv_lo;        // [B][Tq]
   int32_t* kv_hi;        // [B][Tq]
-  int32_t* row_start;    // [B][N] first row of each row's packed example
-  int32_t* row_end;      // [B][N] its last row (backward only)
+  int32_t* row_lo;       // [B][Nq] forward: first visible key of each row
+  int32_t* row_hi;       // [B][Nq]           last visible key
+  int32_t* lo_max;       // [B][Tq] forward: all-visible bounds per block
+  int32_t* hi_min;       // [B][Tq]
+  int32_t* row_start;    // [B][N] backward: first row of each row's example
+  int32_t* row_end;      // [B][N]           its last row
   uint64_t* sort_keys;   // [max(B*Uq, B*Uk)]
   int32_t* counter;      // work counter of the attention kernel
-  int32_t* order_fwd;    // [B*Uq] units of kFwdRowsPerCta rows, longest first
+  int32_t* order_fwd;    // [B*Uq] units of two query blocks, longest first
   // backward only
   int32_t* q_lo;         // [B][Tk]
   int32_t* q_hi;         // [B][Tk]
@@ -77,19 +83,28 @@ struct Workspace {
   size_t bytes;
 };
 
-Workspace carve(void* base, int B, int N, int H, int D, int max_pos,
-                bool backward, int dtype, int qkp) {
+Workspace carve(void* base, int B, int Nq, int Nk, int H, int D, int max_pos,
+                Pass pass, int dtype, int qkp) {
   Carve c{static_cast<char*>(base)};
   Workspace w{};
-  int Tq = (N + kBlock - 1) / kBlock;
-  int Tk = Tq;
+  const bool backward = pass == Pass::kBwd;
+  const int N = Nq;  // backward: Nq == Nk
+  int Tq = (Nq + kBlock - 1) / kBlock;
+  int Tk = (Nk + kBlock - 1) / kBlock;
   int Uq = (Tq + kFwdBlocksPerUnit - 1) / kFwdBlocksPerUnit;
   int Uk = (Tk + kBwdBlocksPerUnit - 1) / kBwdBlocksPerUnit;
   w.table = c.take<float>(size_t(max_pos) * D);
   w.kv_lo = c.take<int32_t>(size_t(B) * Tq);
   w.kv_hi = c.take<int32_t>(size_t(B) * Tq);
-  w.row_start = c.take<int32_t>(size_t(B) * N);
-  if (backward) w.row_end = c.take<int32_t>(size_t(B) * N);
+  if (!backward) {
+    w.row_lo = c.take<int32_t>(size_t(B) * Nq);
+    w.row_hi = c.take<int32_t>(size_t(B) * Nq);
+    w.lo_max = c.take<int32_t>(size_t(B) * Tq);
+    w.hi_min = c.take<int32_t>(size_t(B) * Tq);
+  } else {
+    w.row_start = c.take<int32_t>(size_t(B) * N);
+    w.row_end = c.take<int32_t>(size_t(B) * N);
+  }
   w.sort_keys = c.take<uint64_t>(size_t(B) * (Uq > Uk ? Uq : Uk));
   w.counter = c.take<int32_t>(64);
   w.order_fwd = c.take<int32_t>(size_t(B) * Uq);
@@ -100,8 +115,8 @@ Workspace carve(void* base, int B, int N, int H, int D, int max_pos,
     w.delta = c.take<float>(size_t(B) * H * N);
     w.dq_acc = c.take<float>(size_t(B) * N * H * D);
   }
-  if (dtype == LWM_DTYPE_BF16) {
-    const size_t elems = size_t(B) * N * H * D;
+  if (dtype == LWM_DTYPE_BF16 && pass != Pass::kFwdBlock) {
+    const size_t elems = size_t(B) * Nk * H * D;
     w.k_rot = c.take<uint16_t>(elems);
     if (qkp == LWM_QK_BF16X3 && !backward)
       w.k_rot_lo = c.take<uint16_t>(elems);
@@ -141,13 +156,40 @@ int* status_word() {
   return static_cast<int*>(p);
 }
 
-// Common front half of both passes: RoPE table and block metadata.
-int prepare(const int32_t* seg, double theta, int B, int N, int D,
-            int max_pos, const Workspace& w, cudaStream_t st) {
+// Backward front half: RoPE table and block / row metadata.
+int prepare_bwd(const int32_t* seg, double theta, int B, int N, int D,
+                int max_pos, const Workspace& w, cudaStream_t st) {
   LWM_TRY(launch_rope_table(theta, D, max_pos, w.table, st));
   LWM_TRY(launch_block_meta(seg, B, N, kBlock, kBlock, w.kv_lo, w.kv_hi, st));
   LWM_TRY(launch_row_start(seg, B, N, w.row_start, w.row_end, st));
   return LWM_OK;
+}
+
+// Shared tail of lwm_blockattn_fwd and lwm_blockattn_fwd_block: metadata of
+// queries [q_off, q_off+Nq) against keys [k_off, k_off+Nk), the
+// longest-first order and the attention kernel (table already built).
+int run_forward(const void* q, const void* k_rot, const void* k_rot_lo,
+                const void* v, const int32_t* seg_q, const int32_t* pos_q,
+                const int32_t* seg_k, int q_off, int k_off, int B, int Nq,
+                int Nk, int H, bool x3, void* out, float* lse,
+                const Workspace& w, cudaStream_t st) {
+  LWM_TRY(launch_cross_meta(seg_q, seg_k, B, Nq, Nk, q_off, k_off, w.row_lo,
+                            w.row_hi, w.kv_lo, w.kv_hi, w.lo_max, w.hi_min,
+                            st));
+  LWM_TRY(launch_lpt_order(B, (Nq + kBlock - 1) / kBlock, kFwdBlocksPerUnit,
+                           w.kv_lo, w.kv_hi, w.sort_keys, w.order_fwd,
+                           w.counter, st));
+  FwdArgs a{};
+  a.q = q; a.k_rot = k_rot; a.k_rot_lo = k_rot_lo; a.v = v;
+  a.out = out; a.lse = lse; a.pos_q = pos_q; a.table = w.table;
+  a.kv_lo = w.kv_lo; a.kv_hi = w.kv_hi; a.row_lo = w.row_lo;
+  a.row_hi = w.row_hi; a.lo_max = w.lo_max; a.hi_min = w.hi_min;
+  a.order = w.order_fwd; a.counter = w.counter;
+  a.B = B; a.Nq = Nq; a.Nk = Nk; a.H = H; a.k_off = k_off;
+  a.qk_x3 = x3;
+  a.status = status_word();
+  if (!a.status) return LWM_ERR_CUDA;
+  return cuda_status(launch_fwd_tc(a, st));
 }
 
 }  // namespace
@@ -248,7 +290,8 @@ size_t lwm_blockattn_fwd_workspace_size(int B, int N, int H, int D,
                                         int max_pos, int dtype,
                                         int qk_precision) {
   if (!sizes_ok(B, N, H, D, block_q, block_k, max_pos)) return 0;
-  return carve(nullptr, B, N, H, D, max_pos, false, dtype, qk_precision)
+  return carve(nullptr, B, N, N, H, D, max_pos, Pass::kFwd, dtype,
+               qk_precision)
       .bytes;
 }
 
@@ -257,7 +300,8 @@ size_t lwm_blockattn_bwd_workspace_size(int B, int N, int H, int D,
                                         int max_pos, int dtype,
                                         int qk_precision) {
   if (!sizes_ok(B, N, H, D, block_q, block_k, max_pos)) return 0;
-  return carve(nullptr, B, N, H, D, max_pos, true, dtype, qk_precision)
+  return carve(nullptr, B, N, N, H, D, max_pos, Pass::kBwd, dtype,
+               qk_precision)
       .bytes;
 }
 
@@ -281,36 +325,82 @@ int lwm_blockattn_fwd(const void* q, const void* k, const void* v,
   const void* ptrs[] = {q, k, v, segment_ids, positions, out, lse, workspace};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return LWM_ERR_INVALID_ARG;
-  Workspace w = carve(workspace, B, N, H, D, max_pos, false, dtype,
+  Workspace w = carve(workspace, B, N, N, H, D, max_pos, Pass::kFwd, dtype,
                       qk_precision);
   if (workspace_bytes < w.bytes) return LWM_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  s = prepare(segment_ids, theta, B, N, D, max_pos, w, st);
-  if (s != LWM_OK) return s;
+  LWM_TRY(launch_rope_table(theta, D, max_pos, w.table, st));
   if (dtype == LWM_DTYPE_FP32) {
+    LWM_TRY(launch_block_meta(segment_ids, B, N, kBlock, kBlock, w.kv_lo,
+                              w.kv_hi, st));
     return cuda_status(launch_fwd_simt<float>(
         static_cast<const float*>(q), static_cast<const float*>(k),
         static_cast<const float*>(v), segment_ids, positions, w.table,
         w.kv_lo, B, N, H, static_cast<float*>(out), lse, st));
   }
-  FwdArgs a{};
-  a.q = q; a.k = k; a.v = v; a.out = out; a.lse = lse;
-  a.seg = segment_ids; a.pos = positions; a.table = w.table;
-  a.kv_lo = w.kv_lo; a.kv_hi = w.kv_hi; a.order = w.order_fwd;
-  a.counter = w.counter;
-  a.row_start = w.row_start;
-  a.k_rot = w.k_rot; a.k_rot_lo = w.k_rot_lo;
-  a.B = B; a.N = N; a.H = H;
-  a.qk_x3 = qk_precision == LWM_QK_BF16X3;
   // keys are reused by every query block that sees them: rotate them once
   LWM_TRY(launch_rope_apply(k, positions, w.table, B, N, H, w.k_rot,
                             w.k_rot_lo, st));
-  a.status = status_word();
-  if (!a.status) return LWM_ERR_CUDA;
-  LWM_TRY(launch_lpt_order(B, (N + kBlock - 1) / kBlock, kFwdBlocksPerUnit,
-                           w.kv_lo, w.kv_hi, w.sort_keys, w.order_fwd,
-                           w.counter, st));
-  return cuda_status(launch_fwd_tc(a, st));
+  return run_forward(q, w.k_rot, w.k_rot_lo, v, segment_ids, positions,
+                     segment_ids, 0, 0, B, N, N, H,
+                     qk_precision == LWM_QK_BF16X3, out, lse, w, st);
+}
+
+size_t lwm_blockattn_fwd_block_workspace_size(int B, int Nq, int Nk, int H,
+                                              int D, int max_pos) {
+  if (!sizes_ok(B, Nq, H, D, kBlock, kBlock, max_pos) || Nk < 0) return 0;
+  return carve(nullptr, B, Nq, Nk, H, D, max_pos, Pass::kFwdBlock,
+               LWM_DTYPE_BF16, LWM_QK_BF16)
+      .bytes;
+}
+
+int lwm_blockattn_fwd_block(const void* q, const void* k_rot, const void* v,
+                            const int32_t* seg_q, const int32_t* pos_q,
+                            const int32_t* seg_k, int q_off, int k_off,
+                            double theta, int max_pos, int B, int Nq, int Nk,
+                            int H, int D, void* out, float* lse,
+                            void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  if (!sizes_ok(B, Nq, H, D, kBlock, kBlock, max_pos) || Nk < 0 ||
+      q_off < 0 || k_off < 0 || (int64_t(B) * Nk) >= (int64_t(1) << 31))
+    return LWM_ERR_INVALID_ARG;
+  if (!(theta > 0.0) || !std::isfinite(theta)) return LWM_ERR_INVALID_ARG;
+  if (D != kHeadDim) return LWM_ERR_UNSUPPORTED;
+  if (int64_t(B) * Nq * H == 0) return LWM_OK;
+  if (max_pos < 1) return LWM_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, pos_q, seg_q, out, lse, workspace};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return LWM_ERR_INVALID_ARG;
+  if (Nk > 0) {
+    const void* kp[] = {k_rot, v, seg_k};
+    for (const void* p : kp)
+      if (!p || !aligned16(p)) return LWM_ERR_INVALID_ARG;
+  }
+  Workspace w = carve(workspace, B, Nq, Nk, H, D, max_pos, Pass::kFwdBlock,
+                      LWM_DTYPE_BF16, LWM_QK_BF16);
+  if (workspace_bytes < w.bytes) return LWM_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (Nk == 0) {  // no key: every row sees nothing
+    LWM_TRY(cudaMemsetAsync(out, 0, size_t(B) * Nq * H * D * 2, st));
+    LWM_TRY(launch_fill(lse, -INFINITY, size_t(B) * H * Nq, st));
+    return LWM_OK;
+  }
+  LWM_TRY(launch_rope_table(theta, D, max_pos, w.table, st));
+  return run_forward(q, k_rot, nullptr, v, seg_q, pos_q, seg_k, q_off, k_off,
+                     B, Nq, Nk, H, false, out, lse, w, st);
+}
+
+int lwm_blockattn_merge(void* out, float* lse, const void* out_part,
+                        const float* lse_part, int B, int N, int H, int D,
+                        int dtype, void* stream) {
+  if (B < 0 || N < 0 || H < 0) return LWM_ERR_INVALID_ARG;
+  if (D != kHeadDim || dtype != LWM_DTYPE_BF16) return LWM_ERR_UNSUPPORTED;
+  if (int64_t(B) * N * H == 0) return LWM_OK;
+  const void* ptrs[] = {out, lse, out_part, lse_part};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return LWM_ERR_INVALID_ARG;
+  return cuda_status(launch_merge(out, lse, out_part, lse_part, B, N, H,
+                                  static_cast<cudaStream_t>(stream)));
 }
 
 int lwm_blockattn_bwd(const void* q, const void* k, const void* v,
@@ -335,11 +425,11 @@ int lwm_blockattn_bwd(const void* q, const void* k, const void* v,
                         dq, dk, dv, workspace};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return LWM_ERR_INVALID_ARG;
-  Workspace w = carve(workspace, B, N, H, D, max_pos, true, dtype,
+  Workspace w = carve(workspace, B, N, N, H, D, max_pos, Pass::kBwd, dtype,
                       qk_precision);
   if (workspace_bytes < w.bytes) return LWM_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  s = prepare(segment_ids, theta, B, N, D, max_pos, w, st);
+  s = prepare_bwd(segment_ids, theta, B, N, D, max_pos, w, st);
   if (s != LWM_OK) return s;
   const float scale = 1.f / std::sqrt(float(D));
   LWM_TRY(cudaMemsetAsync(w.dq_acc, 0, sizeof(float) * size_t(B) * N * H * D,

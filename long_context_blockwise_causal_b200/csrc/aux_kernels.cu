@@ -96,6 +96,132 @@ __global__ void row_start_kernel(const int32_t* __restrict__ seg, int B, int N,
   }
 }
 
+// Visible key range of each query row against a block of keys, in global
+// token indices: row i (global q_off + ii) sees the keys of the block whose
+// segment id equals its own and whose index is <= i. With non-decreasing
+// ids those keys are contiguous: [row_lo, row_hi] (empty when lo > hi).
+__global__ void cross_rows_kernel(const int32_t* __restrict__ seg_q,
+                                  const int32_t* __restrict__ seg_k, int B,
+                                  int Nq, int Nk, int q_off, int k_off,
+                                  int32_t* __restrict__ row_lo,
+                                  int32_t* __restrict__ row_hi) {
+  int64_t total = int64_t(B) * Nq;
+  for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < total;
+       e += int64_t(gridDim.x) * blockDim.x) {
+    const int b = int(e / Nq);
+    const int ii = int(e - int64_t(b) * Nq);
+    const int32_t* sk = seg_k + int64_t(b) * Nk;
+    const int v = seg_q[e];
+    int a = 0, z = Nk;  // first key with seg >= v
+    while (a < z) { int m = (a + z) >> 1; if (sk[m] < v) a = m + 1; else z = m; }
+    int lo = a;
+    z = Nk;             // first key with seg > v
+    while (a < z) { int m = (a + z) >> 1; if (sk[m] <= v) a = m + 1; else z = m; }
+    const int hi_seg = a - 1;
+    row_lo[e] = k_off + lo;
+    row_hi[e] = min(k_off + hi_seg, q_off + ii);
+  }
+}
+
+// Per query block t: the key blocks [kv_lo, kv_hi] (block-local) holding any
+// visible key (empty: lo = 1, hi = 0), and the tightest row range the block
+// shares (lo_max, hi_min; lo_max = INT_MAX if some row is past Nq or sees
+// nothing) for the all-visible test of a key block.
+__global__ void cross_tiles_kernel(const int32_t* __restrict__ row_lo,
+                                   const int32_t* __restrict__ row_hi, int B,
+                                   int Nq, int Nk, int k_off, int bq, int bk,
+                                   int Tq, int32_t* __restrict__ kv_lo,
+                                   int32_t* __restrict__ kv_hi,
+                                   int32_t* __restrict__ lo_max,
+                                   int32_t* __restrict__ hi_min) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= B * Tq) return;
+  const int b = e / Tq, t = e - b * Tq;
+  int mn = 0x7fffffff, mx = -1, lmax = -0x7fffffff, hmin = 0x7fffffff;
+  bool all = true;
+  for (int r = 0; r < bq; ++r) {
+    const int ii = t * bq + r;
+    if (ii >= Nq) { all = false; break; }
+    const int lo = row_lo[int64_t(b) * Nq + ii], hi = row_hi[int64_t(b) * Nq + ii];
+    if (lo > hi) { all = false; continue; }
+    mn = min(mn, lo);
+    mx = max(mx, hi);
+    lmax = max(lmax, lo);
+    hmin = min(hmin, hi);
+  }
+  if (mx < 0 || mn > mx) {
+    kv_lo[e] = 1;
+    kv_hi[e] = 0;
+  } else {
+    kv_lo[e] = (mn - k_off) / bk;
+    kv_hi[e] = min((mx - k_off) / bk, (Nk - 1) / bk);
+  }
+  lo_max[e] = all ? lmax : 0x7fffffff;
+  hi_min[e] = all ? hmin : -0x7fffffff;
+}
+
+// out, lse <- the softmax-weighted combination of (out, lse) and
+// (out_part, lse_part) over disjoint key sets: with M = max(lse, lse_p),
+// w = e^(lse - M), w_p = e^(lse_p - M): out = (w out + w_p out_p)/(w + w_p),
+// lse = M + log(w + w_p). Rows where both are -inf stay (0, -inf).
+// Sixteen lanes own one (b, n, h) row (16 bytes each); the lse of a row is
+// read by all of them before lane 0 of the group overwrites it.
+__global__ void merge_kernel(__nv_bfloat16* __restrict__ out,
+                             float* __restrict__ lse,
+                             const __nv_bfloat16* __restrict__ out_p,
+                             const float* __restrict__ lse_p, int B, int N,
+                             int H) {
+  constexpr int kLanesPerRow = kHeadDim / 8;
+  constexpr int kRowsPerWarp = 32 / kLanesPerRow;
+  const int64_t rows = int64_t(B) * N * H;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5;
+  const int64_t warps = (int64_t(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t r0 = warp * kRowsPerWarp; r0 < rows; r0 += warps * kRowsPerWarp) {
+    const int64_t row = r0 + lane / kLanesPerRow;  // (b, n, h)
+    const bool ok = row < rows;
+    int64_t li = 0;
+    float l1 = -INFINITY, l2 = -INFINITY;
+    if (ok) {
+      const int h = int(row % H);
+      const int64_t bn = row / H;
+      const int n = int(bn % N);
+      const int b = int(bn / N);
+      li = (int64_t(b) * H + h) * N + n;
+      l1 = lse[li];
+      l2 = lse_p[li];
+    }
+    __syncwarp();
+    if (!ok) continue;
+    const float M = fmaxf(l1, l2);
+    float w1 = 0.f, w2 = 0.f;
+    if (M != -INFINITY) {
+      w1 = __expf(l1 - M);
+      w2 = __expf(l2 - M);
+    }
+    const float den = w1 + w2;
+    const float a = den > 0.f ? w1 / den : 0.f, c = den > 0.f ? w2 / den : 0.f;
+    const int64_t e = row * kLanesPerRow + (lane % kLanesPerRow);
+    uint4 x = reinterpret_cast<const uint4*>(out)[e];
+    const uint4 y = reinterpret_cast<const uint4*>(out_p)[e];
+    uint32_t* xs = reinterpret_cast<uint32_t*>(&x);
+    const uint32_t* ys = reinterpret_cast<const uint32_t*>(&y);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      xs[k] = pack_bf16x2(a * bf16lo_to_f32(xs[k]) + c * bf16lo_to_f32(ys[k]),
+                          a * bf16hi_to_f32(xs[k]) + c * bf16hi_to_f32(ys[k]));
+    reinterpret_cast<uint4*>(out)[e] = x;
+    if (lane % kLanesPerRow == 0)
+      lse[li] = den > 0.f ? M + __logf(den) : -INFINITY;
+  }
+}
+
+__global__ void fill_kernel(float* __restrict__ x, float v, int64_t n) {
+  for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < n;
+       e += int64_t(gridDim.x) * blockDim.x)
+    x[e] = v;
+}
+
 __global__ void block_meta_kernel(const int32_t* __restrict__ seg, int B,
                                   int N, int bq, int bk, int Tq,
                                   int32_t* __restrict__ kv_lo,
@@ -168,12 +294,13 @@ __global__ void unit_cost_kernel(int B, int T, int group,
   if (e >= B * U) return;
   int b = e / U, u = e - b * U;
   int t0 = u * group, t1 = min(t0 + group, T) - 1;
-  int l = lo[b * T + t0], h = hi[b * T + t0];
-  for (int t = t0 + 1; t <= t1; ++t) {
+  int l = 0x7fffffff, h = -1;
+  for (int t = t0; t <= t1; ++t) {
+    if (lo[b * T + t] > hi[b * T + t]) continue;  // no visible key block
     l = min(l, lo[b * T + t]);
     h = max(h, hi[b * T + t]);
   }
-  int cost = max(0, h - l + 1);
+  int cost = h >= l ? h - l + 1 : 0;
   // ascending key order == descending cost, then ascending unit id
   keys[e] = (uint64_t(0x7FFFFFFF - cost) << 32) | uint32_t(e);
 }
@@ -325,6 +452,43 @@ cudaError_t launch_rope_apply(const void* x, const int32_t* pos,
       static_cast<const __nv_bfloat16*>(x), pos,
       reinterpret_cast<const float2*>(table), chunks, H,
       static_cast<__nv_bfloat16*>(hi), static_cast<__nv_bfloat16*>(lo));
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_cross_meta(const int32_t* seg_q, const int32_t* seg_k,
+                              int B, int Nq, int Nk, int q_off, int k_off,
+                              int32_t* row_lo, int32_t* row_hi, int32_t* kv_lo,
+                              int32_t* kv_hi, int32_t* lo_max, int32_t* hi_min,
+                              cudaStream_t st) {
+  const int64_t n = int64_t(B) * Nq;
+  if (n == 0) return cudaSuccess;
+  cross_rows_kernel<<<grid_for(n, 256, 148 * 16), 256, 0, st>>>(
+      seg_q, seg_k, B, Nq, Nk, q_off, k_off, row_lo, row_hi);
+  note_launch();
+  const int Tq = (Nq + kBlock - 1) / kBlock;
+  cross_tiles_kernel<<<(B * Tq + 127) / 128, 128, 0, st>>>(
+      row_lo, row_hi, B, Nq, Nk, k_off, kBlock, kBlock, Tq, kv_lo, kv_hi,
+      lo_max, hi_min);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge(void* out, float* lse, const void* out_p,
+                         const float* lse_p, int B, int N, int H,
+                         cudaStream_t st) {
+  const int64_t n = int64_t(B) * N * H * (kHeadDim / 8);
+  if (n == 0) return cudaSuccess;
+  merge_kernel<<<grid_for(n, 256, 148 * 16), 256, 0, st>>>(
+      static_cast<__nv_bfloat16*>(out), lse,
+      static_cast<const __nv_bfloat16*>(out_p), lse_p, B, N, H);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fill(float* x, float v, int64_t n, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  fill_kernel<<<grid_for(n, 256, 148 * 8), 256, 0, st>>>(x, v, n);
   note_launch();
   return cudaGetLastError();
 }

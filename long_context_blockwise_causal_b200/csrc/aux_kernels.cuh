@@ -15,6 +15,19 @@ cudaError_t launch_block_meta(const int32_t* seg, int B, int N, int bq, int bk,
 cudaError_t launch_rope_apply(const void* x, const int32_t* pos,
                               const float* table, int B, int N, int H,
                               void* hi, void* lo, cudaStream_t st);
+// Per-row visible key ranges of queries [q_off, q_off+Nq) against keys
+// [k_off, k_off+Nk) (global indices), and per query block the key-block
+// range plus the shared row range used for the all-visible test.
+cudaError_t launch_cross_meta(const int32_t* seg_q, const int32_t* seg_k,
+                              int B, int Nq, int Nk, int q_off, int k_off,
+                              int32_t* row_lo, int32_t* row_hi, int32_t* kv_lo,
+                              int32_t* kv_hi, int32_t* lo_max, int32_t* hi_min,
+                              cudaStream_t st);
+// Combine a partial (out_p, lse_p) over another key set into (out, lse).
+cudaError_t launch_merge(void* out, float* lse, const void* out_p,
+                         const float* lse_p, int B, int N, int H,
+                         cudaStream_t st);
+cudaError_t launch_fill(float* x, float v, int64_t n, cudaStream_t st);
 // rs[i]: first row of row i's packed example; re[i] (if re != nullptr):
 // its last row.
 cudaError_t launch_row_start(const int32_t* seg, int B, int N, int32_t* rs,

@@ -66,16 +66,18 @@ struct FwdCfg {
 
 struct FwdParams {
   int32_t* counter;
-  const int32_t* seg;
-  const int32_t* row_start;
-  const int32_t* pos;
+  const int32_t* pos_q;
   const float2* table;
   const int32_t* kv_lo;
   const int32_t* kv_hi;
+  const int32_t* row_lo;
+  const int32_t* row_hi;
+  const int32_t* lo_max;
+  const int32_t* hi_min;
   const int32_t* order;
   float* lse;
   int* status;
-  int B, N, H, Tq, U, G;
+  int B, Nq, Nk, H, Tq, U, G, k_off;
   int total_items;
   float scale_log2;
 };
@@ -107,8 +109,10 @@ __device__ __forceinline__ Item get_item(const FwdParams& p, int it) {
     if (m.present[s]) {
       m.lo[s] = p.kv_lo[m.b * p.Tq + m.t[s]];
       m.hi[s] = p.kv_hi[m.b * p.Tq + m.t[s]];
-      m.jlo = min(m.jlo, m.lo[s]);
-      m.jhi = max(m.jhi, m.hi[s]);
+      if (m.lo[s] <= m.hi[s]) {  // a query block may see no key block
+        m.jlo = min(m.jlo, m.lo[s]);
+        m.jhi = max(m.jhi, m.hi[s]);
+      }
     } else {
       m.lo[s] = 1;
       m.hi[s] = 0;
@@ -285,16 +289,15 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (it < 0) break;
       Item m = get_item(p, it);
       if (!m.present[s]) continue;
-      const int64_t rowbase = int64_t(m.b) * p.N;
+      const int64_t rowbase = int64_t(m.b) * p.Nq;
       const int q0 = m.t[s] * kBlock;
       const int i = q0 + r;
-      const bool valid = i < p.N;
-      // allowed keys of row i: rs_i <= kj <= hi_i (empty for rows >= N)
-      const int rs_i = valid ? __ldg(p.row_start + rowbase + i) : 0;
-      const int hi_i = valid ? i : -1;
-      const int q_last = q0 + kBlock - 1;
-      const int rs_last = q_last < p.N ? __ldg(p.row_start + rowbase + q_last)
-                                       : 0x7fffffff;
+      const bool valid = i < p.Nq;
+      // allowed keys of this row (global indices): lo_i <= key <= hi_i
+      const int lo_i = valid ? __ldg(p.row_lo + rowbase + i) : 1;
+      const int hi_i = valid ? __ldg(p.row_hi + rowbase + i) : 0;
+      const int lo_max = __ldg(p.lo_max + m.b * p.Tq + m.t[s]);
+      const int hi_min = __ldg(p.hi_min + m.b * p.Tq + m.t[s]);
       float m_used = -INFINITY, l = 0.f;
       bool first = true;
       for (int j = m.hi[s]; j >= m.lo[s] && ok; --j) {
@@ -304,20 +307,19 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (!ok) break;
         sc++;
         tc_fence_after();
-        const int k0 = j * kBlock;
-        // every pair of the tile allowed: keys end before the first query,
-        // all queries valid, and the last query's example starts at or
-        // before the first key
-        const bool full = (k0 + kBlock - 1 < q0) && (k0 >= rs_last);
+        const int k0 = p.k_off + j * kBlock;  // global index of key 0
+        // every pair of the tile allowed: every row of the block sees the
+        // whole key block
+        const bool full = lo_max <= k0 && hi_min >= k0 + kBlock - 1;
         // the whole 128-column S row of this thread in registers
         uint32_t v[4][32];
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, v[c]);
         tmem_wait_ld();
-        if (!full) {  // mask: keep rs_i <= key <= hi_i
+        if (!full) {  // mask: keep lo_i <= key <= hi_i
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            const int lo = rs_i - (k0 + c * 32), hi = hi_i - (k0 + c * 32);
+            const int lo = lo_i - (k0 + c * 32), hi = hi_i - (k0 + c * 32);
 #pragma unroll
             for (int x = 0; x < 32; ++x)
               v[c][x] = (x >= lo && x <= hi) ? v[c][x] : 0xff800000u;
@@ -402,9 +404,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
+        // rows that saw no key (l == 0) write 0; O was never written then
         for (int x = 0; x < 32; x += 2)
-          pk[x >> 1] = pack_bf16x2(__uint_as_float(v[x]) * inv,
-                                   __uint_as_float(v[x + 1]) * inv);
+          pk[x >> 1] = l > 0.f ? pack_bf16x2(__uint_as_float(v[x]) * inv,
+                                             __uint_as_float(v[x + 1]) * inv)
+                               : 0u;
         // columns c*32 .. c*32+31 = d chunk (c>>1), 16-byte chunks
         // (c&1)*4 .. +3 of that 128-byte row
 #pragma unroll
@@ -431,8 +435,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_arrive(bar(C::bQEmpty + s));
       }
       if (valid)
-        p.lse[(int64_t(m.b) * p.H + m.h) * p.N + i] =
-            (m_used + __log2f(l)) * kLn2;
+        p.lse[(int64_t(m.b) * p.H + m.h) * p.Nq + i] =
+            l > 0.f ? (m_used + __log2f(l)) * kLn2 : -INFINITY;
     }
     if (threadIdx.x == 0 || threadIdx.x == 128) bulk_wait0();
   } else if (warp < 12) {
@@ -451,13 +455,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (lane == 0) mbar_arrive(bar(C::bItemEmpty + (n & 1)));
       if (it < 0) break;
       Item m = get_item(p, it);
-      const int64_t rowbase = int64_t(m.b) * p.N;
+      const int64_t rowbase = int64_t(m.b) * p.Nq;
       for (int s = 0; s < 2 && ok; ++s) {
         if (!m.present[s]) continue;
         float4 cs0[8];
         bool valid;
-        const float4* trow = rope_prefetch(p.pos, p.table, rowbase,
-                                           m.t[s] * kBlock + r, p.N, cs0,
+        const float4* trow = rope_prefetch(p.pos_q, p.table, rowbase,
+                                           m.t[s] * kBlock + r, p.Nq, cs0,
                                            valid);
         ok = mbar_wait(bar(C::bQFull + s), qcount[s] & 1, abort_flag,
                        p.status, kWaitLimitNs);
@@ -661,6 +665,16 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           prev = has_j ? j : -1;
         }
         if (!ok) break;
+        // a sub-tile that sees no key block issued no MMA: its Q tile is
+        // still consumed here, so the rotation is done with it before the
+        // epilogue stages the (zero) output in the same buffer
+        for (int s = 0; s < 2 && ok; ++s)
+          if (m.present[s] && !qwaited[s]) {
+            ok = mbar_wait(bar(C::bQReady + s), qc[s] & 1, abort_flag,
+                           p.status, kWaitLimitNs);
+            qc[s]++;
+          }
+        if (!ok) break;
         for (int s = 0; s < 2; ++s)
           if (m.present[s]) {
             mma_commit(bar(C::bOFull + s));
@@ -760,27 +774,31 @@ int sm_count() {
 template <bool X3>
 static cudaError_t launch_fwd_impl(const FwdArgs& a, cudaStream_t st) {
   CUtensorMap mq, mk, mv, mo, mklo;
-  if (!make_bnhd_map(&mq, a.q, a.B, a.N, a.H) ||
-      !make_bnhd_map(&mk, a.k_rot, a.B, a.N, a.H) ||
-      !make_bnhd_map(&mv, a.v, a.B, a.N, a.H) ||
-      !make_bnhd_map(&mo, a.out, a.B, a.N, a.H) ||
-      !make_bnhd_map(&mklo, X3 ? a.k_rot_lo : a.k_rot, a.B, a.N, a.H))
+  if (!make_bnhd_map(&mq, a.q, a.B, a.Nq, a.H) ||
+      !make_bnhd_map(&mk, a.k_rot, a.B, a.Nk, a.H) ||
+      !make_bnhd_map(&mv, a.v, a.B, a.Nk, a.H) ||
+      !make_bnhd_map(&mo, a.out, a.B, a.Nq, a.H) ||
+      !make_bnhd_map(&mklo, X3 ? a.k_rot_lo : a.k_rot, a.B, a.Nk, a.H))
     return cudaErrorInvalidValue;
   FwdParams p{};
   p.counter = a.counter;
-  p.seg = a.seg;
-  p.row_start = a.row_start;
-  p.pos = a.pos;
+  p.pos_q = a.pos_q;
   p.table = reinterpret_cast<const float2*>(a.table);
   p.kv_lo = a.kv_lo;
   p.kv_hi = a.kv_hi;
+  p.row_lo = a.row_lo;
+  p.row_hi = a.row_hi;
+  p.lo_max = a.lo_max;
+  p.hi_min = a.hi_min;
   p.order = a.order;
   p.lse = a.lse;
   p.status = a.status;
   p.B = a.B;
-  p.N = a.N;
+  p.Nq = a.Nq;
+  p.Nk = a.Nk;
   p.H = a.H;
-  p.Tq = (a.N + kBlock - 1) / kBlock;
+  p.k_off = a.k_off;
+  p.Tq = (a.Nq + kBlock - 1) / kBlock;
   p.U = (p.Tq + kFwdBlocksPerUnit - 1) / kFwdBlocksPerUnit;
   // heads interleaved per scheduling round: 2 keeps the K/V of the heads
   // in flight L2-resident while still mixing costs across CTAs
@@ -808,7 +826,7 @@ static cudaError_t launch_fwd_impl(const FwdArgs& a, cudaStream_t st) {
 }
 
 cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t st) {
-  if (a.B == 0 || a.N == 0 || a.H == 0) return cudaSuccess;
+  if (a.B == 0 || a.Nq == 0 || a.Nk == 0 || a.H == 0) return cudaSuccess;
   return a.qk_x3 ? launch_fwd_impl<true>(a, st) : launch_fwd_impl<false>(a, st);
 }
 

@@ -12,23 +12,29 @@ namespace lwm {
 constexpr int kFwdBlocksPerUnit = 2;
 constexpr int kBwdBlocksPerUnit = 1;
 
+// Forward of query rows [q_off, q_off + Nq) (global token indices) against
+// rotated keys / values [k_off, k_off + Nk) of the same packed row; self-
+// attention is q_off = k_off = 0, Nq = Nk. Visibility comes as per-row key
+// ranges (row_lo/row_hi) and per query block key-block ranges (kv_lo/kv_hi)
+// plus the all-visible bounds (lo_max/hi_min), all from launch_cross_meta.
 struct FwdArgs {
-  const void* q;
-  const void* k;
-  const void* v;
-  void* out;
-  float* lse;
-  const int32_t* seg;
-  const int32_t* pos;
+  const void* q;           // [B][Nq][H][D], un-rotated
+  const void* k_rot;       // [B][Nk][H][D], R(pos) k
+  const void* k_rot_lo;    // bf16 residual of k_rot (split-QK mode)
+  const void* v;           // [B][Nk][H][D]
+  void* out;               // [B][Nq][H][D]
+  float* lse;              // [B][H][Nq]
+  const int32_t* pos_q;    // [B][Nq]
   const float* table;
   const int32_t* kv_lo;
   const int32_t* kv_hi;
+  const int32_t* row_lo;
+  const int32_t* row_hi;
+  const int32_t* lo_max;
+  const int32_t* hi_min;
   const int32_t* order;
   int32_t* counter;        // zeroed work counter (units handed out in order)
-  const int32_t* row_start;
-  const void* k_rot;       // R(pos) k, bf16 [B][N][H][D]
-  const void* k_rot_lo;    // bf16 residual of k_rot (split-QK mode)
-  int B, N, H;
+  int B, Nq, Nk, H, k_off;
   bool qk_x3;
   int* status;
 };

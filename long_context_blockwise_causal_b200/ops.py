@@ -58,6 +58,12 @@ _SIGS = {
     "lwm_blockattn_fwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _d, _i, _i,
                                        _i, _i, _i, _i, _i, _i, _i, _vp, _vp,
                                        _vp]),
+    "lwm_blockattn_fwd_block_workspace_size": (_sz, [_i] * 6),
+    "lwm_blockattn_fwd_block": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i,
+                                     _d, _i, _i, _i, _i, _i, _i, _vp, _vp,
+                                     _vp, _sz, _vp]),
+    "lwm_blockattn_merge": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
+                                 _vp]),
 }
 
 
@@ -224,6 +230,46 @@ def bwd(q, k, v, out, dout, lse, segment_ids, positions, theta,
         _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(), _stream(stream))
     _check(st, "lwm_blockattn_bwd")
     return dq, dk, dv
+
+
+def fwd_block_workspace_size(B, Nq, Nk, H, max_pos, D=HEAD_DIM) -> int:
+    return int(lib().lwm_blockattn_fwd_block_workspace_size(
+        B, Nq, Nk, H, D, max_pos))
+
+
+def fwd_block(q, k_rot, v, seg_q, pos_q, seg_k, q_off, k_off, theta,
+              max_pos, out=None, lse=None, workspace=None, stream=None):
+    """Partial forward of query rows [q_off, q_off+Nq) against the rotated
+    key / value rows [k_off, k_off+Nk) of the same packed sequence (one step
+    of a ring). Returns (out [B,Nq,H,D] bf16, lse [B,H,Nq] fp32); rows that
+    see no key get (0, -inf)."""
+    _need_cuda(q, k_rot, v, seg_q, pos_q, seg_k, out, lse, workspace)
+    B, Nq, H, D = q.shape
+    Nk = k_rot.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    ws = _workspace(fwd_block_workspace_size(B, Nq, Nk, H, max_pos, D),
+                    q.device, workspace)
+    st = lib().lwm_blockattn_fwd_block(
+        _ptr(q), _ptr(k_rot), _ptr(v), _ptr(seg_q), _ptr(pos_q), _ptr(seg_k),
+        int(q_off), int(k_off), float(theta), int(max_pos), B, Nq, Nk, H, D,
+        _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "lwm_blockattn_fwd_block")
+    return out, lse
+
+
+def merge(out, lse, out_part, lse_part, stream=None):
+    """In place: fold the partial (out_part, lse_part) over another key set
+    into (out, lse) with the log-sum-exp rule. Returns (out, lse)."""
+    _need_cuda(out, lse, out_part, lse_part)
+    B, N, H, D = out.shape
+    st = lib().lwm_blockattn_merge(_ptr(out), _ptr(lse), _ptr(out_part),
+                                   _ptr(lse_part), B, N, H, D,
+                                   _dtype_code(out), _stream(stream))
+    _check(st, "lwm_blockattn_merge")
+    return out, lse
 
 
 def classify(segment_ids, block_q=BLOCK, block_k=BLOCK, with_class=True,

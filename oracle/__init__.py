@@ -33,6 +33,8 @@ Modules:
   rope       -- RoPE frequencies, angles and rotation.
   attention  -- dense fp64 forward/backward (row-blocked), sampled rows.
   blockwise  -- CPU online-softmax restatement in ring order (invariance pin).
+  ring       -- partial attention over a key block, the log-sum-exp merge and
+                a P-device ring run in order (RingAttention).
   classify   -- tile classification (brute force and a counting form).
 """
 
@@ -42,6 +44,9 @@ from .attention import (  # noqa: F401
     attn_bwd_cols, SOFTMAX_SCALE_RULE,
 )
 from .blockwise import blockwise_fwd  # noqa: F401
+from .ring import (  # noqa: F401
+    attn_fwd_partial, merge_partials, ring_chunks, ring_fwd,
+)
 from .classify import (  # noqa: F401
     classify_bruteforce, classify_count, TILE_EMPTY, TILE_PARTIAL, TILE_FULL,
 )
