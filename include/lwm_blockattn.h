@@ -180,6 +180,53 @@ LWM_API int lwm_blockattn_merge(void* out, float* lse, const void* out_part,
                                 const float* lse_part, int B, int N, int H,
                                 int D, int dtype, void* stream);
 
+/* Backward of the ring (same page, 3.1: the gradients of a key/value
+ * block travel around the ring with it and come back to its owner).
+ *
+ * D_i = sum_d dout_i[d] out_i[d] as fp32 [B][H][N] (out, dout [B][N][H][D]
+ * bf16): computed once per query chunk from its final out. */
+LWM_API int lwm_blockattn_bwd_delta(const void* out, const void* dout, int B,
+                                    int N, int H, int D, int dtype,
+                                    float* delta, void* stream);
+
+/* Bytes of workspace lwm_blockattn_bwd_block needs (key-side metadata). */
+LWM_API size_t lwm_blockattn_bwd_block_workspace_size(int B, int Nq, int Nk,
+                                                      int H, int D);
+
+/* Partial backward of query rows [q_off, q_off+Nq) against the key/value
+ * rows [k_off, k_off+Nk) of the same packed sequence (visibility as in
+ * lwm_blockattn_fwd_block), given the FINAL lse of the queries (over all
+ * keys) and their delta. Adds into fp32 accumulators in the rotated frame
+ * and without the 1/sqrt(D) factor:
+ *   dq_acc [B][Nq][H][D] += dS K~,   dk_acc [B][Nk][H][D] += dS^T Q~,
+ *   dv_acc [B][Nk][H][D] += P^T dO,
+ * with P = exp(Q~K~^T/sqrt(D) - lse) on visible pairs, dS = P (dO V^T - D).
+ *   q_rot [B][Nq][H][D], k_rot [B][Nk][H][D]: bf16, already rotated
+ *   v [B][Nk][H][D], dout [B][Nq][H][D]: bf16; lse, delta [B][H][Nq] fp32
+ *   seg_q [B][Nq], seg_k [B][Nk] int32
+ * The accumulators are the caller's, zeroed before the first call; turn
+ * them into gradients with lwm_blockattn_grad_finish. dq_acc receives
+ * atomic adds (order not fixed). D == 128. Async on stream. */
+LWM_API int lwm_blockattn_bwd_block(const void* q_rot, const void* k_rot,
+                                    const void* v, const void* dout,
+                                    const float* lse, const float* delta,
+                                    const int32_t* seg_q, const int32_t* seg_k,
+                                    int q_off, int k_off, int B, int Nq,
+                                    int Nk, int H, int D, float* dq_acc,
+                                    float* dk_acc, float* dv_acc,
+                                    void* workspace, size_t workspace_bytes,
+                                    void* stream);
+
+/* grad (bf16 [B][N][H][D]) from an fp32 accumulator of the same shape:
+ * with positions (int32 [B][N]) and a table from lwm_blockattn_rope_table,
+ * grad = R(-pos) acc / sqrt(D) (dq, dk); with positions == NULL,
+ * grad = acc (dv). Async on stream. */
+LWM_API int lwm_blockattn_grad_finish(const float* acc,
+                                      const int32_t* positions,
+                                      const float* rope_table, int max_pos,
+                                      int B, int N, int H, int D, int dtype,
+                                      void* grad, void* stream);
+
 /* Tile classifier (exported so it can be checked bit-exactly). For each
  * batch row b and query block t (Tq = ceil(N/block_q) blocks), key blocks
  * j (Tk = ceil(N/block_k)):

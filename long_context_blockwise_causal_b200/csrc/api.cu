@@ -54,26 +54,30 @@ struct Carve {
   }
 };
 
-enum class Pass { kFwd, kFwdBlock, kBwd };
+enum class Pass { kFwd, kFwdBlock, kBwd, kBwdBlock };
 
 // Workspace regions (a pass carves only what it uses).
 struct Workspace {
   float* table;          // [max_pos][D/2] float2
+  // forward: per query block the key-block range and all-visible bounds,
+  // per query row its visible keys (launch_cross_meta)
   int32_t* kv_lo;        // [B][Tq]
-  int32_t* kv_hi;        // [B][Tq]
-  int32_t* row_lo;       // [B][Nq] forward: first visible key of each row
-  int32_t* row_hi;       // [B][Nq]           last visible key
-  int32_t* lo_max;       // [B][Tq] forward: all-visible bounds per block
-  int32_t* hi_min;       // [B][Tq]
-  int32_t* row_start;    // [B][N] backward: first row of each row's example
-  int32_t* row_end;      // [B][N]           its last row
-  uint64_t* sort_keys;   // [max(B*Uq, B*Uk)]
-  int32_t* counter;      // work counter of the attention kernel
+  int32_t* kv_hi;
+  int32_t* lo_max;
+  int32_t* hi_min;
+  int32_t* row_lo;       // [B][Nq]
+  int32_t* row_hi;
   int32_t* order_fwd;    // [B*Uq] units of two query blocks, longest first
-  // backward only
+  // backward: the key-side view (launch_cross_meta_keys)
   int32_t* q_lo;         // [B][Tk]
-  int32_t* q_hi;         // [B][Tk]
-  int32_t* order_bwd;    // [B*Uk]
+  int32_t* q_hi;
+  int32_t* klo_max;
+  int32_t* khi_min;
+  int32_t* col_lo;       // [B][Nk]
+  int32_t* col_hi;
+  int32_t* order_bwd;    // [B*Tk]
+  uint64_t* sort_keys;   // [B*Uq] or [B*Tk]
+  int32_t* counter;      // work counter of the attention kernel
   float* delta;          // [B][H][N]
   float* dq_acc;         // [B][N][H][D]
   // bf16 path: rotated keys (and queries for the backward), [B][N][H][D]
@@ -87,40 +91,43 @@ Workspace carve(void* base, int B, int Nq, int Nk, int H, int D, int max_pos,
                 Pass pass, int dtype, int qkp) {
   Carve c{static_cast<char*>(base)};
   Workspace w{};
-  const bool backward = pass == Pass::kBwd;
-  const int N = Nq;  // backward: Nq == Nk
-  int Tq = (Nq + kBlock - 1) / kBlock;
-  int Tk = (Nk + kBlock - 1) / kBlock;
-  int Uq = (Tq + kFwdBlocksPerUnit - 1) / kFwdBlocksPerUnit;
-  int Uk = (Tk + kBwdBlocksPerUnit - 1) / kBwdBlocksPerUnit;
-  w.table = c.take<float>(size_t(max_pos) * D);
-  w.kv_lo = c.take<int32_t>(size_t(B) * Tq);
-  w.kv_hi = c.take<int32_t>(size_t(B) * Tq);
-  if (!backward) {
-    w.row_lo = c.take<int32_t>(size_t(B) * Nq);
-    w.row_hi = c.take<int32_t>(size_t(B) * Nq);
+  const bool fwd = pass == Pass::kFwd || pass == Pass::kFwdBlock;
+  const bool tc = dtype == LWM_DTYPE_BF16 && qkp == LWM_QK_BF16;
+  const int Tq = (Nq + kBlock - 1) / kBlock;
+  const int Tk = (Nk + kBlock - 1) / kBlock;
+  const int Uq = (Tq + kFwdBlocksPerUnit - 1) / kFwdBlocksPerUnit;
+  if (pass != Pass::kBwdBlock) w.table = c.take<float>(size_t(max_pos) * D);
+  if (fwd) {
+    w.kv_lo = c.take<int32_t>(size_t(B) * Tq);
+    w.kv_hi = c.take<int32_t>(size_t(B) * Tq);
     w.lo_max = c.take<int32_t>(size_t(B) * Tq);
     w.hi_min = c.take<int32_t>(size_t(B) * Tq);
+    w.row_lo = c.take<int32_t>(size_t(B) * Nq);
+    w.row_hi = c.take<int32_t>(size_t(B) * Nq);
+    w.order_fwd = c.take<int32_t>(size_t(B) * Uq);
+    w.sort_keys = c.take<uint64_t>(size_t(B) * Uq);
   } else {
-    w.row_start = c.take<int32_t>(size_t(B) * N);
-    w.row_end = c.take<int32_t>(size_t(B) * N);
-  }
-  w.sort_keys = c.take<uint64_t>(size_t(B) * (Uq > Uk ? Uq : Uk));
-  w.counter = c.take<int32_t>(64);
-  w.order_fwd = c.take<int32_t>(size_t(B) * Uq);
-  if (backward) {
     w.q_lo = c.take<int32_t>(size_t(B) * Tk);
     w.q_hi = c.take<int32_t>(size_t(B) * Tk);
-    w.order_bwd = c.take<int32_t>(size_t(B) * Uk);
-    w.delta = c.take<float>(size_t(B) * H * N);
-    w.dq_acc = c.take<float>(size_t(B) * N * H * D);
+    w.klo_max = c.take<int32_t>(size_t(B) * Tk);
+    w.khi_min = c.take<int32_t>(size_t(B) * Tk);
+    w.col_lo = c.take<int32_t>(size_t(B) * Nk);
+    w.col_hi = c.take<int32_t>(size_t(B) * Nk);
+    w.order_bwd = c.take<int32_t>(size_t(B) * Tk);
+    w.sort_keys = c.take<uint64_t>(size_t(B) * Tk);
   }
-  if (dtype == LWM_DTYPE_BF16 && pass != Pass::kFwdBlock) {
-    const size_t elems = size_t(B) * Nk * H * D;
-    w.k_rot = c.take<uint16_t>(elems);
-    if (qkp == LWM_QK_BF16X3 && !backward)
-      w.k_rot_lo = c.take<uint16_t>(elems);
-    if (backward) w.q_rot = c.take<uint16_t>(elems);
+  w.counter = c.take<int32_t>(64);
+  if (pass == Pass::kBwd) {
+    w.delta = c.take<float>(size_t(B) * H * Nq);
+    w.dq_acc = c.take<float>(size_t(B) * Nq * H * D);
+  }
+  if (dtype == LWM_DTYPE_BF16 && pass == Pass::kFwd) {
+    w.k_rot = c.take<uint16_t>(size_t(B) * Nk * H * D);
+    if (qkp == LWM_QK_BF16X3) w.k_rot_lo = c.take<uint16_t>(size_t(B) * Nk * H * D);
+  }
+  if (tc && pass == Pass::kBwd) {
+    w.k_rot = c.take<uint16_t>(size_t(B) * Nk * H * D);
+    w.q_rot = c.take<uint16_t>(size_t(B) * Nq * H * D);
   }
   w.bytes = c.off;
   return w;
@@ -156,13 +163,23 @@ int* status_word() {
   return static_cast<int*>(p);
 }
 
-// Backward front half: RoPE table and block / row metadata.
-int prepare_bwd(const int32_t* seg, double theta, int B, int N, int D,
-                int max_pos, const Workspace& w, cudaStream_t st) {
-  LWM_TRY(launch_rope_table(theta, D, max_pos, w.table, st));
-  LWM_TRY(launch_block_meta(seg, B, N, kBlock, kBlock, w.kv_lo, w.kv_hi, st));
-  LWM_TRY(launch_row_start(seg, B, N, w.row_start, w.row_end, st));
-  return LWM_OK;
+// Shared tail of lwm_blockattn_bwd and lwm_blockattn_bwd_block: key-side
+// metadata of queries [q_off, q_off+Nq) against keys [k_off, k_off+Nk), the
+// longest-first order of the key blocks and the attention kernel.
+int run_backward(BwdArgs a, const int32_t* seg_q, const int32_t* seg_k,
+                 int k_off, const Workspace& w, cudaStream_t st) {
+  LWM_TRY(launch_cross_meta_keys(seg_q, seg_k, a.B, a.Nq, a.Nk, a.q_off,
+                                 k_off, w.col_lo, w.col_hi, w.q_lo, w.q_hi,
+                                 w.klo_max, w.khi_min, st));
+  LWM_TRY(launch_lpt_order(a.B, (a.Nk + kBlock - 1) / kBlock,
+                           kBwdBlocksPerUnit, w.q_lo, w.q_hi, w.sort_keys,
+                           w.order_bwd, w.counter, st));
+  a.q_lo = w.q_lo; a.q_hi = w.q_hi; a.col_lo = w.col_lo; a.col_hi = w.col_hi;
+  a.klo_max = w.klo_max; a.khi_min = w.khi_min;
+  a.order = w.order_bwd; a.counter = w.counter;
+  a.status = status_word();
+  if (!a.status) return LWM_ERR_CUDA;
+  return cuda_status(launch_bwd_tc(a, st));
 }
 
 // Shared tail of lwm_blockattn_fwd and lwm_blockattn_fwd_block: metadata of
@@ -429,8 +446,7 @@ int lwm_blockattn_bwd(const void* q, const void* k, const void* v,
                       qk_precision);
   if (workspace_bytes < w.bytes) return LWM_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  s = prepare_bwd(segment_ids, theta, B, N, D, max_pos, w, st);
-  if (s != LWM_OK) return s;
+  LWM_TRY(launch_rope_table(theta, D, max_pos, w.table, st));
   const float scale = 1.f / std::sqrt(float(D));
   LWM_TRY(cudaMemsetAsync(w.dq_acc, 0, sizeof(float) * size_t(B) * N * H * D,
                           st));
@@ -460,32 +476,92 @@ int lwm_blockattn_bwd(const void* q, const void* k, const void* v,
         segment_ids, positions, w.table, B, N, H, w.dq_acc,
         static_cast<T*>(dk), static_cast<T*>(dv), st));
   } else {
-    LWM_TRY(launch_kv_meta(B, (N + kBlock - 1) / kBlock,
-                           (N + kBlock - 1) / kBlock, w.kv_lo, w.kv_hi, w.q_lo,
-                           w.q_hi, st));
-    LWM_TRY(launch_lpt_order(B, (N + kBlock - 1) / kBlock, kBwdBlocksPerUnit,
-                             w.q_lo, w.q_hi, w.sort_keys, w.order_bwd,
-                             w.counter, st));
-    BwdArgs a{};
-    a.q = q; a.k = k; a.v = v; a.dout = dout; a.lse = lse; a.delta = w.delta;
-    a.seg = segment_ids; a.pos = positions; a.table = w.table;
-    a.q_lo = w.q_lo; a.q_hi = w.q_hi; a.order = w.order_bwd;
-    a.counter = w.counter;
-    a.row_start = w.row_start;
-    a.dq_acc = w.dq_acc; a.dk = dk; a.dv = dv;
-    a.q_rot = w.q_rot; a.k_rot = w.k_rot; a.row_end = w.row_end;
-    // queries and keys are both re-read inside the key-major sweep
+    // queries and keys are both re-read inside the key-major sweep: rotate
+    // them once
     LWM_TRY(launch_rope_apply(q, positions, w.table, B, N, H, w.q_rot,
                               nullptr, st));
     LWM_TRY(launch_rope_apply(k, positions, w.table, B, N, H, w.k_rot,
                               nullptr, st));
-    a.B = B; a.N = N; a.H = H;
-    a.status = status_word();
-    if (!a.status) return LWM_ERR_CUDA;
-    LWM_TRY(launch_bwd_tc(a, st));
+    BwdArgs a{};
+    a.q_rot = w.q_rot; a.k_rot = w.k_rot; a.v = v; a.dout = dout;
+    a.lse = lse; a.delta = w.delta; a.pos_k = positions; a.table = w.table;
+    a.dq_acc = w.dq_acc; a.dk = dk; a.dv = dv;
+    a.B = B; a.Nq = N; a.Nk = N; a.H = H; a.q_off = 0;
+    s = run_backward(a, segment_ids, segment_ids, 0, w, st);
+    if (s != LWM_OK) return s;
   }
   return cuda_status(launch_dq_convert<T>(w.dq_acc, positions, w.table, B, N,
                                           H, scale, static_cast<T*>(dq), st));
+}
+
+size_t lwm_blockattn_bwd_block_workspace_size(int B, int Nq, int Nk, int H,
+                                              int D) {
+  if (!sizes_ok(B, Nq, H, D, kBlock, kBlock, 0) || Nk < 0 ||
+      (int64_t(B) * Nk) >= (int64_t(1) << 31))
+    return 0;
+  return carve(nullptr, B, Nq, Nk, H, D, 0, Pass::kBwdBlock, LWM_DTYPE_BF16,
+               LWM_QK_BF16)
+      .bytes;
+}
+
+int lwm_blockattn_bwd_block(const void* q_rot, const void* k_rot,
+                            const void* v, const void* dout, const float* lse,
+                            const float* delta, const int32_t* seg_q,
+                            const int32_t* seg_k, int q_off, int k_off, int B,
+                            int Nq, int Nk, int H, int D, float* dq_acc,
+                            float* dk_acc, float* dv_acc, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  if (!sizes_ok(B, Nq, H, D, kBlock, kBlock, 0) || Nk < 0 || q_off < 0 ||
+      k_off < 0 || (int64_t(B) * Nk) >= (int64_t(1) << 31))
+    return LWM_ERR_INVALID_ARG;
+  if (D != kHeadDim) return LWM_ERR_UNSUPPORTED;
+  if (int64_t(B) * Nq * Nk * H == 0) return LWM_OK;
+  const void* ptrs[] = {q_rot, k_rot, v, dout, lse, delta, seg_q, seg_k,
+                        dq_acc, dk_acc, dv_acc, workspace};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return LWM_ERR_INVALID_ARG;
+  Workspace w = carve(workspace, B, Nq, Nk, H, D, 0, Pass::kBwdBlock,
+                      LWM_DTYPE_BF16, LWM_QK_BF16);
+  if (workspace_bytes < w.bytes) return LWM_ERR_WORKSPACE;
+  BwdArgs a{};
+  a.q_rot = q_rot; a.k_rot = k_rot; a.v = v; a.dout = dout;
+  a.lse = lse; a.delta = delta;
+  a.dq_acc = dq_acc; a.dk_acc = dk_acc; a.dv_acc = dv_acc;
+  a.B = B; a.Nq = Nq; a.Nk = Nk; a.H = H; a.q_off = q_off;
+  return run_backward(a, seg_q, seg_k, k_off, w,
+                      static_cast<cudaStream_t>(stream));
+}
+
+int lwm_blockattn_bwd_delta(const void* out, const void* dout, int B, int N,
+                            int H, int D, int dtype, float* delta,
+                            void* stream) {
+  if (B < 0 || N < 0 || H < 0) return LWM_ERR_INVALID_ARG;
+  if (D != kHeadDim || dtype != LWM_DTYPE_BF16) return LWM_ERR_UNSUPPORTED;
+  if (int64_t(B) * N * H == 0) return LWM_OK;
+  const void* ptrs[] = {out, dout, delta};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return LWM_ERR_INVALID_ARG;
+  using T = __nv_bfloat16;
+  return cuda_status(launch_bwd_delta<T>(static_cast<const T*>(out),
+                                         static_cast<const T*>(dout), B, N, H,
+                                         delta,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+int lwm_blockattn_grad_finish(const float* acc, const int32_t* positions,
+                              const float* rope_table, int max_pos, int B,
+                              int N, int H, int D, int dtype, void* grad,
+                              void* stream) {
+  if (B < 0 || N < 0 || H < 0 || max_pos < 0) return LWM_ERR_INVALID_ARG;
+  if (D != kHeadDim || dtype != LWM_DTYPE_BF16) return LWM_ERR_UNSUPPORTED;
+  if (int64_t(B) * N * H == 0) return LWM_OK;
+  if (!acc || !grad || !aligned16(acc) || !aligned16(grad))
+    return LWM_ERR_INVALID_ARG;
+  if (positions && (!rope_table || max_pos < 1)) return LWM_ERR_INVALID_ARG;
+  const float scale = positions ? 1.f / std::sqrt(float(D)) : 1.f;
+  return cuda_status(launch_dq_convert<__nv_bfloat16>(
+      acc, positions, rope_table, B, N, H, scale,
+      static_cast<__nv_bfloat16*>(grad), static_cast<cudaStream_t>(stream)));
 }
 
 int lwm_blockattn_classify(const int32_t* segment_ids, int B, int N,

@@ -160,6 +160,68 @@ __global__ void cross_tiles_kernel(const int32_t* __restrict__ row_lo,
   hi_min[e] = all ? hmin : -0x7fffffff;
 }
 
+// Key-side view of the same rule, for the key-major backward: key k
+// (global k_off + jj) is seen by the queries col_lo[k] .. col_hi[k]
+// (global indices, empty when lo > hi): those of its segment from k on.
+__global__ void cross_cols_kernel(const int32_t* __restrict__ seg_q,
+                                  const int32_t* __restrict__ seg_k, int B,
+                                  int Nq, int Nk, int q_off, int k_off,
+                                  int32_t* __restrict__ col_lo,
+                                  int32_t* __restrict__ col_hi) {
+  int64_t total = int64_t(B) * Nk;
+  for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < total;
+       e += int64_t(gridDim.x) * blockDim.x) {
+    const int b = int(e / Nk);
+    const int jj = int(e - int64_t(b) * Nk);
+    const int32_t* sq = seg_q + int64_t(b) * Nq;
+    const int v = seg_k[e];
+    int a = 0, z = Nq;  // first query with seg >= v
+    while (a < z) { int m = (a + z) >> 1; if (sq[m] < v) a = m + 1; else z = m; }
+    const int first = a;
+    z = Nq;             // first query with seg > v
+    while (a < z) { int m = (a + z) >> 1; if (sq[m] <= v) a = m + 1; else z = m; }
+    col_lo[e] = max(q_off + first, k_off + jj);
+    col_hi[e] = q_off + a - 1;
+  }
+}
+
+// Per key block j: the query blocks [q_lo, q_hi] (chunk-local) holding a
+// query that sees one of its keys (none: lo = 1, hi = 0), and the tightest
+// shared query range (klo_max, khi_min; klo_max = INT_MAX if some key is
+// past Nk or seen by nobody) for the all-visible test of a query block.
+__global__ void cross_kblocks_kernel(const int32_t* __restrict__ col_lo,
+                                     const int32_t* __restrict__ col_hi,
+                                     int B, int Nq, int Nk, int q_off, int Tk,
+                                     int32_t* __restrict__ q_lo,
+                                     int32_t* __restrict__ q_hi,
+                                     int32_t* __restrict__ klo_max,
+                                     int32_t* __restrict__ khi_min) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= B * Tk) return;
+  const int b = e / Tk, j = e - b * Tk;
+  int mn = 0x7fffffff, mx = -1, lmax = -0x7fffffff, hmin = 0x7fffffff;
+  bool all = true;
+  for (int r = 0; r < kBlock; ++r) {
+    const int jj = j * kBlock + r;
+    if (jj >= Nk) { all = false; break; }
+    const int lo = col_lo[int64_t(b) * Nk + jj], hi = col_hi[int64_t(b) * Nk + jj];
+    if (lo > hi) { all = false; continue; }
+    mn = min(mn, lo);
+    mx = max(mx, hi);
+    lmax = max(lmax, lo);
+    hmin = min(hmin, hi);
+  }
+  if (mx < 0 || mn > mx) {
+    q_lo[e] = 1;
+    q_hi[e] = 0;
+  } else {
+    q_lo[e] = (mn - q_off) / kBlock;
+    q_hi[e] = min((mx - q_off) / kBlock, (Nq - 1) / kBlock);
+  }
+  klo_max[e] = all ? lmax : 0x7fffffff;
+  khi_min[e] = all ? hmin : -0x7fffffff;
+}
+
 // out, lse <- the softmax-weighted combination of (out, lse) and
 // (out_part, lse_part) over disjoint key sets: with M = max(lse, lse_p),
 // w = e^(lse - M), w_p = e^(lse_p - M): out = (w out + w_p out_p)/(w + w_p),
@@ -403,10 +465,15 @@ __global__ void dq_convert_kernel(const float* __restrict__ acc,
     int k = int(e % (kHeadDim / 2));
     int64_t bnh = e / (kHeadDim / 2);
     int64_t bn = bnh / H;
-    float2 cs = table[int64_t(pos[bn]) * (kHeadDim / 2) + k];
     float2 x = reinterpret_cast<const float2*>(acc)[e];
     x.x *= scale;
     x.y *= scale;
+    if (!pos) {  // plain conversion
+      dq[2 * e] = T(x.x);
+      dq[2 * e + 1] = T(x.y);
+      continue;
+    }
+    float2 cs = table[int64_t(pos[bn]) * (kHeadDim / 2) + k];
     // inverse rotation: (a, b) -> (a c + b s, -a s + b c)
     float a = x.x * cs.x + x.y * cs.y;
     float c = x.y * cs.x - x.x * cs.y;
@@ -470,6 +537,24 @@ cudaError_t launch_cross_meta(const int32_t* seg_q, const int32_t* seg_k,
   cross_tiles_kernel<<<(B * Tq + 127) / 128, 128, 0, st>>>(
       row_lo, row_hi, B, Nq, Nk, k_off, kBlock, kBlock, Tq, kv_lo, kv_hi,
       lo_max, hi_min);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_cross_meta_keys(const int32_t* seg_q, const int32_t* seg_k,
+                                   int B, int Nq, int Nk, int q_off,
+                                   int k_off, int32_t* col_lo,
+                                   int32_t* col_hi, int32_t* q_lo,
+                                   int32_t* q_hi, int32_t* klo_max,
+                                   int32_t* khi_min, cudaStream_t st) {
+  const int64_t n = int64_t(B) * Nk;
+  if (n == 0) return cudaSuccess;
+  cross_cols_kernel<<<grid_for(n, 256, 148 * 16), 256, 0, st>>>(
+      seg_q, seg_k, B, Nq, Nk, q_off, k_off, col_lo, col_hi);
+  note_launch();
+  const int Tk = (Nk + kBlock - 1) / kBlock;
+  cross_kblocks_kernel<<<(B * Tk + 127) / 128, 128, 0, st>>>(
+      col_lo, col_hi, B, Nq, Nk, q_off, Tk, q_lo, q_hi, klo_max, khi_min);
   note_launch();
   return cudaGetLastError();
 }

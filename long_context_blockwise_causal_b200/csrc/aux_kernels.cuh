@@ -23,6 +23,15 @@ cudaError_t launch_cross_meta(const int32_t* seg_q, const int32_t* seg_k,
                               int32_t* row_lo, int32_t* row_hi, int32_t* kv_lo,
                               int32_t* kv_hi, int32_t* lo_max, int32_t* hi_min,
                               cudaStream_t st);
+// Key-side metadata of the same pair of ranges for the key-major backward:
+// per key the queries that see it (global indices), per key block the query
+// block range and the shared query range of the all-visible test.
+cudaError_t launch_cross_meta_keys(const int32_t* seg_q, const int32_t* seg_k,
+                                   int B, int Nq, int Nk, int q_off,
+                                   int k_off, int32_t* col_lo,
+                                   int32_t* col_hi, int32_t* q_lo,
+                                   int32_t* q_hi, int32_t* klo_max,
+                                   int32_t* khi_min, cudaStream_t st);
 // Combine a partial (out_p, lse_p) over another key set into (out, lse).
 cudaError_t launch_merge(void* out, float* lse, const void* out_p,
                          const float* lse_p, int B, int N, int H,
@@ -49,6 +58,7 @@ cudaError_t launch_check_inputs(const int32_t* seg, const int32_t* pos, int B,
 template <typename T>
 cudaError_t launch_bwd_delta(const T* out, const T* dout, int B, int N, int H,
                              float* delta, cudaStream_t st);
+// dq = R(-pos) acc * scale in T; pos == nullptr: dq = acc * scale.
 template <typename T>
 cudaError_t launch_dq_convert(const float* acc, const int32_t* pos,
                               const float* table, int B, int N, int H,

@@ -54,8 +54,11 @@ constexpr int kSmemBwd = kSMisc + 16;   // tmem addr, abort, 2 work slots
 
 struct BwdParams {
   int32_t* counter;
-  const int32_t* row_end;
-  const int32_t* pos;
+  const int32_t* col_lo;
+  const int32_t* col_hi;
+  const int32_t* klo_max;
+  const int32_t* khi_min;
+  const int32_t* pos_k;
   const float2* table;
   const int32_t* q_lo;
   const int32_t* q_hi;
@@ -65,8 +68,10 @@ struct BwdParams {
   float* dq_acc;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
+  float* dk_acc;
+  float* dv_acc;
   int* status;
-  int B, N, H, Tk, G, total_items;
+  int B, Nq, Nk, H, Tk, G, q_off, total_items;
   float scale_log2, scale;
 };
 
@@ -180,13 +185,16 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (lane == 0) mbar_arrive(bar(bItemEmpty0 + (u & 1)));
       if (it < 0) break;
       const BItem m = get_bitem(p, it);
-      const int64_t rowbase = int64_t(m.b) * p.N;
+      const int64_t rowbase = int64_t(m.b) * p.Nk;
       const int k0 = m.j * kBlock;
       const int kj = k0 + r;
-      const bool valid_k = kj < p.N;
-      // key kj is seen by queries kj .. re_k (none for a key >= N)
-      const int re_k = valid_k ? __ldg(p.row_end + rowbase + kj) : -1;
-      const int re_k0 = __ldg(p.row_end + rowbase + k0);
+      const bool valid_k = kj < p.Nk;
+      // key kj is seen by the queries lo_k .. hi_k (global indices; none
+      // for a key >= Nk)
+      const int lo_k = valid_k ? __ldg(p.col_lo + rowbase + kj) : 1;
+      const int hi_k = valid_k ? __ldg(p.col_hi + rowbase + kj) : 0;
+      const int klo_max = __ldg(p.klo_max + m.b * p.Tk + m.j);
+      const int khi_min = __ldg(p.khi_min + m.b * p.Tk + m.j);
       for (int i = m.qlo; i <= m.qhi && ok; ++i) {
         const int st = g & 1;
         ok = mbar_wait(bar(bStFull), g & 1, abort_flag, p.status, kWaitNs);
@@ -196,8 +204,9 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        const int q0 = i * kBlock;
-        const bool full = (k0 + kBlock - 1 < q0) && (re_k0 >= q0 + kBlock - 1);
+        const int q0 = p.q_off + i * kBlock;  // global index of query 0
+        // every key of the block seen by every query of the block
+        const bool full = klo_max <= q0 && khi_min >= q0 + kBlock - 1;
         const float* ls = aux_lse + st * 128;
         const float* dl = aux_del + st * 128;
         uint8_t* dsrow = smem + kSDS + r * 128;
@@ -215,7 +224,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
               const int qb = q0 + (2 * half + cc) * 32;
-              const int lo = kj - qb, hi = re_k - qb;
+              const int lo = lo_k - qb, hi = hi_k - qb;
 #pragma unroll
               for (int x = 0; x < 32; ++x)
                 sv[cc][x] = (x >= lo && x <= hi) ? sv[cc][x] : 0xff800000u;
@@ -302,11 +311,40 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (!ok) break;
       tc_fence_after();
       const int64_t orow = ((rowbase + (valid_k ? kj : 0)) * p.H + m.h) * kHeadDim;
+      // a key block no query sees issued no MMA: its accumulators hold
+      // nothing of this item (bf16 mode writes zeros, fp32 mode adds none)
+      const bool seen = m.qlo <= m.qhi;
+      if (p.dk_acc) {
+        // fp32 accumulators carried across calls: add dV and the unscaled,
+        // rotated dK~ (this thread owns key row kj of this launch)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint32_t v[32];
+          tmem_ld32((c < 4 ? tC : tD) + lane_off + (c & 3) * 32, v);
+          tmem_wait_ld();
+          if (valid_k && seen) {
+            float4* dst = reinterpret_cast<float4*>(
+                (c < 4 ? p.dv_acc : p.dk_acc) + orow + (c & 3) * 32);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              float4 a = dst[e];
+              a.x += __uint_as_float(v[4 * e]);
+              a.y += __uint_as_float(v[4 * e + 1]);
+              a.z += __uint_as_float(v[4 * e + 2]);
+              a.w += __uint_as_float(v[4 * e + 3]);
+              dst[e] = a;
+            }
+          }
+        }
+      } else {
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t v[32];
         tmem_ld32(tC + lane_off + c * 32, v);
         tmem_wait_ld();
+        if (!seen)
+#pragma unroll
+          for (int x = 0; x < 32; ++x) v[x] = 0u;
         if (valid_k) {
           uint4* dst = reinterpret_cast<uint4*>(p.dv + orow + c * 32);
 #pragma unroll
@@ -319,13 +357,16 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
       }
       const float4* trow = reinterpret_cast<const float4*>(
-          p.table + int64_t(valid_k ? __ldg(p.pos + rowbase + kj) : 0) *
+          p.table + int64_t(valid_k ? __ldg(p.pos_k + rowbase + kj) : 0) *
                         (kHeadDim / 2));
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t v[32];
         tmem_ld32(tD + lane_off + c * 32, v);
         tmem_wait_ld();
+        if (!seen)
+#pragma unroll
+          for (int x = 0; x < 32; ++x) v[x] = 0u;
         if (valid_k) {
           uint32_t o[16];
 #pragma unroll
@@ -346,6 +387,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           for (int e = 0; e < 4; ++e)
             dst[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
         }
+      }
       }
       tc_fence_before();
       __syncwarp();
@@ -417,15 +459,15 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (lane == 0) mbar_arrive(bar(bItemEmpty0 + (u & 1)));
       if (it < 0) break;
       const BItem m = get_bitem(p, it);
-      const float* lse_bh = p.lse + (int64_t(m.b) * p.H + m.h) * p.N;
-      const float* del_bh = p.delta + (int64_t(m.b) * p.H + m.h) * p.N;
+      const float* lse_bh = p.lse + (int64_t(m.b) * p.H + m.h) * p.Nq;
+      const float* del_bh = p.delta + (int64_t(m.b) * p.H + m.h) * p.Nq;
       for (int i = m.qlo; i <= m.qhi && ok; ++i) {
         const int st = g & 1;
         const int q = i * kBlock + r;
         // stage (lse log2 e, D) of this block; the slot's previous user
         // (block g-2) finished with it before its dQ, flushed last round
-        aux_lse[st * 128 + r] = q < p.N ? __ldg(lse_bh + q) * kLog2e : 0.f;
-        aux_del[st * 128 + r] = q < p.N ? __ldg(del_bh + q) : 0.f;
+        aux_lse[st * 128 + r] = q < p.Nq ? __ldg(lse_bh + q) * kLog2e : 0.f;
+        aux_del[st * 128 + r] = q < p.Nq ? __ldg(del_bh + q) : 0.f;
         mbar_arrive(bar(bAux0 + st));
         if (g > 0) ok = flush(g - 1);
         pb = m.b;
@@ -570,6 +612,13 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           ++g;
         }
         if (!ok) break;
+        // a key block no query sees issued no MMA and so never waited for
+        // the previous item's epilogue: wait here, or bAccFull would
+        // complete a second phase before the compute warps saw the first
+        if (first_q && n > 0)
+          ok = mbar_wait(bar(bAccEmpty), (n - 1) & 1, abort_flag, p.status,
+                         kWaitNs);
+        if (!ok) break;
         mma_commit(bar(bAccFull));
         mma_commit(bar(bKVEmpty));
         ++n;
@@ -591,18 +640,22 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
 }  // namespace
 
 cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t st) {
-  if (a.B == 0 || a.N == 0 || a.H == 0) return cudaSuccess;
+  if (a.B == 0 || a.Nq == 0 || a.Nk == 0 || a.H == 0) return cudaSuccess;
   CUtensorMap mq, mk, mv, mdo, mdq;
-  if (!make_bnhd_map(&mq, a.q_rot, a.B, a.N, a.H) ||
-      !make_bnhd_map(&mk, a.k_rot, a.B, a.N, a.H) ||
-      !make_bnhd_map(&mv, a.v, a.B, a.N, a.H) ||
-      !make_bnhd_map(&mdo, a.dout, a.B, a.N, a.H) ||
-      !make_bnhd_f32_map(&mdq, a.dq_acc, a.B, a.N, a.H))
+  if (!make_bnhd_map(&mq, a.q_rot, a.B, a.Nq, a.H) ||
+      !make_bnhd_map(&mk, a.k_rot, a.B, a.Nk, a.H) ||
+      !make_bnhd_map(&mv, a.v, a.B, a.Nk, a.H) ||
+      !make_bnhd_map(&mdo, a.dout, a.B, a.Nq, a.H) ||
+      !make_bnhd_f32_map(&mdq, a.dq_acc, a.B, a.Nq, a.H))
     return cudaErrorInvalidValue;
+  if (!a.dk_acc != !a.dv_acc) return cudaErrorInvalidValue;
   BwdParams p{};
   p.counter = a.counter;
-  p.row_end = a.row_end;
-  p.pos = a.pos;
+  p.col_lo = a.col_lo;
+  p.col_hi = a.col_hi;
+  p.klo_max = a.klo_max;
+  p.khi_min = a.khi_min;
+  p.pos_k = a.pos_k;
   p.table = reinterpret_cast<const float2*>(a.table);
   p.q_lo = a.q_lo;
   p.q_hi = a.q_hi;
@@ -612,11 +665,15 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t st) {
   p.dq_acc = a.dq_acc;
   p.dk = static_cast<__nv_bfloat16*>(a.dk);
   p.dv = static_cast<__nv_bfloat16*>(a.dv);
+  p.dk_acc = a.dk_acc;
+  p.dv_acc = a.dv_acc;
   p.status = a.status;
   p.B = a.B;
-  p.N = a.N;
+  p.Nq = a.Nq;
+  p.Nk = a.Nk;
   p.H = a.H;
-  p.Tk = (a.N + kBlock - 1) / kBlock;
+  p.q_off = a.q_off;
+  p.Tk = (a.Nk + kBlock - 1) / kBlock;
   // one head per scheduling round: the fp32 dQ accumulator, Q~ and dO of
   // a head (16 + 8 + 8 MB at 32K) then stay L2-resident while ~148 key
   // blocks of that head reduce into it (4 heads at once measured 7% slower

@@ -39,28 +39,38 @@ struct FwdArgs {
   int* status;
 };
 
+// Backward of query rows [q_off, q_off + Nq) against keys / values
+// [k_off, k_off + Nk) (key-major: one key block per work unit). Visibility
+// comes per key as the range of queries that see it (col_lo/col_hi, global
+// indices) and per key block as the query-block range (q_lo/q_hi) plus the
+// all-visible bounds (klo_max/khi_min), all from launch_cross_meta_keys.
+// dQ~ (unscaled, rotated frame) is reduce-added into dq_acc. dK, dV either
+// go out as bf16 (dk = R(-pos_k) dK~ / sqrt(D), dv; dk_acc == nullptr) or
+// are added, unscaled and in the rotated frame, into fp32 accumulators
+// dk_acc / dv_acc that the caller carries across calls.
 struct BwdArgs {
-  const void* q;
-  const void* k;
-  const void* v;
-  const void* dout;
-  const float* lse;
-  const float* delta;
-  const int32_t* seg;
-  const int32_t* pos;
-  const float* table;
+  const void* q_rot;       // [B][Nq][H][D], R(pos) q
+  const void* k_rot;       // [B][Nk][H][D], R(pos) k
+  const void* v;           // [B][Nk][H][D]
+  const void* dout;        // [B][Nq][H][D]
+  const float* lse;        // [B][H][Nq]
+  const float* delta;      // [B][H][Nq]
+  const int32_t* pos_k;    // [B][Nk] (bf16 output mode only)
+  const float* table;      // (bf16 output mode only)
   const int32_t* q_lo;
   const int32_t* q_hi;
+  const int32_t* col_lo;
+  const int32_t* col_hi;
+  const int32_t* klo_max;
+  const int32_t* khi_min;
   const int32_t* order;
   int32_t* counter;
-  const int32_t* row_start;
-  const int32_t* row_end;
-  void* q_rot;             // scratch for R(pos) q, bf16 [B][N][H][D]
-  void* k_rot;             // scratch for R(pos) k
-  float* dq_acc;
-  void* dk;
+  float* dq_acc;           // [B][Nq][H][D] fp32
+  void* dk;                // [B][Nk][H][D] bf16, or
   void* dv;
-  int B, N, H;
+  float* dk_acc;           // [B][Nk][H][D] fp32 accumulators
+  float* dv_acc;
+  int B, Nq, Nk, H, q_off;
   int* status;
 };
 

@@ -64,6 +64,14 @@ _SIGS = {
                                      _vp, _sz, _vp]),
     "lwm_blockattn_merge": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                  _vp]),
+    "lwm_blockattn_bwd_delta": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp,
+                                     _vp]),
+    "lwm_blockattn_bwd_block_workspace_size": (_sz, [_i] * 5),
+    "lwm_blockattn_bwd_block": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                     _i, _i, _i, _i, _i, _i, _i, _vp, _vp,
+                                     _vp, _vp, _sz, _vp]),
+    "lwm_blockattn_grad_finish": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                                       _vp, _vp]),
 }
 
 
@@ -270,6 +278,58 @@ def merge(out, lse, out_part, lse_part, stream=None):
                                    _dtype_code(out), _stream(stream))
     _check(st, "lwm_blockattn_merge")
     return out, lse
+
+
+def bwd_delta(out, dout, delta=None, stream=None):
+    """D = rowsum(dout * out) as fp32 [B,H,N]."""
+    _need_cuda(out, dout, delta)
+    B, N, H, D = out.shape
+    if delta is None:
+        delta = torch.empty((B, H, N), dtype=torch.float32, device=out.device)
+    st = lib().lwm_blockattn_bwd_delta(_ptr(out), _ptr(dout), B, N, H, D,
+                                       _dtype_code(out), _ptr(delta),
+                                       _stream(stream))
+    _check(st, "lwm_blockattn_bwd_delta")
+    return delta
+
+
+def bwd_block_workspace_size(B, Nq, Nk, H, D=HEAD_DIM) -> int:
+    return int(lib().lwm_blockattn_bwd_block_workspace_size(B, Nq, Nk, H, D))
+
+
+def bwd_block(q_rot, k_rot, v, dout, lse, delta, seg_q, seg_k, q_off, k_off,
+              dq_acc, dk_acc, dv_acc, workspace=None, stream=None):
+    """Partial backward of a query chunk against a key chunk: adds into the
+    fp32 accumulators dq_acc [B,Nq,H,D], dk_acc and dv_acc [B,Nk,H,D]
+    (rotated frame, no 1/sqrt(D); finish them with grad_finish)."""
+    _need_cuda(q_rot, k_rot, v, dout, lse, delta, seg_q, seg_k, dq_acc,
+               dk_acc, dv_acc, workspace)
+    B, Nq, H, D = q_rot.shape
+    Nk = k_rot.shape[1]
+    ws = _workspace(bwd_block_workspace_size(B, Nq, Nk, H, D), q_rot.device,
+                    workspace)
+    st = lib().lwm_blockattn_bwd_block(
+        _ptr(q_rot), _ptr(k_rot), _ptr(v), _ptr(dout), _ptr(lse),
+        _ptr(delta), _ptr(seg_q), _ptr(seg_k), int(q_off), int(k_off), B, Nq,
+        Nk, H, D, _ptr(dq_acc), _ptr(dk_acc), _ptr(dv_acc), _ptr(ws),
+        ws.numel(), _stream(stream))
+    _check(st, "lwm_blockattn_bwd_block")
+    return dq_acc, dk_acc, dv_acc
+
+
+def grad_finish(acc, positions=None, table=None, out=None, stream=None):
+    """bf16 gradient from an fp32 accumulator: R(-pos) acc / sqrt(D) when
+    positions are given (dq, dk), else acc (dv)."""
+    _need_cuda(acc, positions, table, out)
+    B, N, H, D = acc.shape
+    if out is None:
+        out = torch.empty(acc.shape, dtype=torch.bfloat16, device=acc.device)
+    st = lib().lwm_blockattn_grad_finish(
+        _ptr(acc), _ptr(positions), _ptr(table),
+        0 if table is None else table.shape[0], B, N, H, D, DTYPE_BF16,
+        _ptr(out), _stream(stream))
+    _check(st, "lwm_blockattn_grad_finish")
+    return out
 
 
 def classify(segment_ids, block_q=BLOCK, block_k=BLOCK, with_class=True,

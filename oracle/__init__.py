@@ -45,7 +45,8 @@ from .attention import (  # noqa: F401
 )
 from .blockwise import blockwise_fwd  # noqa: F401
 from .ring import (  # noqa: F401
-    attn_fwd_partial, merge_partials, ring_chunks, ring_fwd,
+    attn_fwd_partial, merge_partials, ring_chunks, ring_fwd, bwd_delta,
+    attn_bwd_partial, ring_bwd,
 )
 from .classify import (  # noqa: F401
     classify_bruteforce, classify_count, TILE_EMPTY, TILE_PARTIAL, TILE_FULL,

@@ -9,6 +9,13 @@ and the partial results are combined exactly with the log-sum-exp rule
 (the same online-softmax identity as "LWM：突破 100 万 Token 的开源大模型",
 配置参数, blockwise attention).
 
+The backward follows the same ring: every step applies the chain rule of
+the dense forward to the pairs of the visiting block only, with the final
+lse and D_i = rowsum(dO * O) of the finished forward; dq collects at the
+query's device, dk and dv travel with their block and are back at its
+owner after the last step. The gradient is linear in the pairs, so the
+block sums equal the dense gradient.
+
 Readings: the mask of a partial is the dense one (same packed example,
 key token index <= query token index) restricted to the visiting keys; a
 row with no visible key in a partial has out = 0 and lse = -inf, and
@@ -101,3 +108,68 @@ def ring_fwd(q, k, v, segment_ids, positions, theta, P):
         out[:, qo:qo + qn] = o
         lse[:, :, qo:qo + qn] = l_
     return out, lse
+
+
+def bwd_delta(out, dout):
+    """D [B,H,N] = sum over d of dout * out (the finished forward's out)."""
+    return np.einsum("bnhd,bnhd->bhn", _f64(out), _f64(dout))
+
+
+def attn_bwd_partial(q, k, v, dout, lse, delta, seg_q, seg_k, pos_q, pos_k,
+                     q_off, k_off, theta):
+    """Gradient contributions of the pairs (query of [q_off, q_off+Nq), key
+    of [k_off, k_off+Nk)) given the final lse and D of the queries.
+    Returns dq [B,Nq,H,D], dk, dv [B,Nk,H,D] (w.r.t. un-rotated q, k)."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    lse, delta = _f64(lse), _f64(delta)
+    seg_q, seg_k, pos_q, pos_k = (_i64(x) for x in (seg_q, seg_k, pos_q,
+                                                    pos_k))
+    B, Nq, H, D = q.shape
+    Nk = k.shape[1]
+    scale = 1.0 / np.sqrt(D)
+    dq = np.zeros((B, Nq, H, D))
+    dk = np.zeros((B, Nk, H, D))
+    dv = np.zeros((B, Nk, H, D))
+    gi = q_off + np.arange(Nq)
+    gj = k_off + np.arange(Nk)
+    for b in range(B):
+        mask = (seg_q[b][:, None] == seg_k[b][None, :]) & \
+               (gj[None, :] <= gi[:, None])
+        for h in range(H):
+            qr = rope_rotate(q[b, :, h], pos_q[b], theta)
+            kr = rope_rotate(k[b, :, h], pos_k[b], theta)
+            s = (qr @ kr.T) * scale
+            p = np.where(mask, np.exp(np.where(mask, s, 0.0)
+                                      - lse[b, h][:, None]), 0.0)
+            dv[b, :, h] = p.T @ dout[b, :, h]
+            dp = dout[b, :, h] @ v[b, :, h].T
+            ds = p * (dp - delta[b, h][:, None])
+            dq[b, :, h] = rope_rotate((ds @ kr) * scale, pos_q[b], theta,
+                                      sign=-1)
+            dk[b, :, h] = rope_rotate((ds.T @ qr) * scale, pos_k[b], theta,
+                                      sign=-1)
+    return dq, dk, dv
+
+
+def ring_bwd(q, k, v, dout, segment_ids, positions, theta, P):
+    """Backward of a P-device ring, every device in ring order, on the CPU.
+    Returns dq, dk, dv [B,N,H,D]."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    seg, pos = _i64(segment_ids), _i64(positions)
+    out, lse = ring_fwd(q, k, v, seg, pos, theta, P)
+    delta = bwd_delta(out, dout)
+    dq, dk, dv = (np.zeros_like(q) for _ in range(3))
+    chunks = ring_chunks(q.shape[1], P)
+    for i, (qo, qn) in enumerate(chunks):
+        qs = slice(qo, qo + qn)
+        for s in range(P):
+            ko, kn = chunks[(i - s) % P]
+            ks = slice(ko, ko + kn)
+            a, b_, c = attn_bwd_partial(
+                q[:, qs], k[:, ks], v[:, ks], dout[:, qs], lse[:, :, qs],
+                delta[:, :, qs], seg[:, qs], seg[:, ks], pos[:, qs],
+                pos[:, ks], qo, ko, theta)
+            dq[:, qs] += a
+            dk[:, ks] += b_
+            dv[:, ks] += c
+    return dq, dk, dv

@@ -33,6 +33,38 @@ class OracleBackend:
                                       out_part.numpy(), lse_part.numpy())
         return torch.from_numpy(o), torch.from_numpy(l_)
 
+    # backward: accumulators hold gradients w.r.t. the rotated q and k
+    # (scaled), so finish only rotates back
+    def delta(self, out, dout):
+        return torch.from_numpy(oracle.bwd_delta(out, dout))
+
+    def zeros_acc(self, like):
+        return torch.zeros(like.shape, dtype=torch.float64)
+
+    def partial_bwd(self, q_rot, k_rot, v, dout, lse, delta, seg_q, seg_k,
+                    q_off, k_off, dq_acc, dk_acc, dv_acc):
+        zq = np.zeros(tuple(seg_q.shape), dtype=np.int64)
+        zk = np.zeros(tuple(seg_k.shape), dtype=np.int64)
+        a, b, c = oracle.attn_bwd_partial(q_rot, k_rot, v, dout, lse, delta,
+                                          seg_q, seg_k, zq, zk, q_off, k_off,
+                                          self.theta)
+        dq_acc += torch.from_numpy(a)
+        dk_acc += torch.from_numpy(b)
+        dv_acc += torch.from_numpy(c)
+
+    def finish(self, acc, positions):
+        x = acc.numpy()
+        pos = positions.numpy()
+        out = np.empty_like(x)
+        for b in range(x.shape[0]):
+            for h in range(x.shape[2]):
+                out[b, :, h] = oracle.rope_rotate(x[b, :, h], pos[b],
+                                                  self.theta, sign=-1)
+        return torch.from_numpy(out)
+
+    def finish_v(self, acc):
+        return acc.clone()
+
     def empty(self, q):
         B, N, H, _ = q.shape
         return (torch.zeros(q.shape, dtype=torch.float64),

@@ -139,3 +139,204 @@ def test_ring_of_one_equals_full_forward(cuda_dev):
     torch.cuda.synchronize()
     # the same kernel over the same tiles: identical results
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+# ------------------------------------------------------------ backward
+
+BWD_REL = 2e-2   # of max |reference|, as for the full backward
+
+
+def _with_dout(t, seed):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    t["dout"] = torch.randn(t["q"].shape, generator=g, device="cuda",
+                            dtype=torch.float32).to(torch.bfloat16)
+    return t
+
+
+def _final_lse_delta(t):
+    """lse and D of the finished dense forward (oracle, fp64 -> fp32); both
+    sides of a partial-backward check receive these same values."""
+    out, lse = oracle.attn_fwd(t["q"], t["k"], t["v"], t["segment_ids"],
+                               t["positions"], t["theta"])
+    delta = oracle.bwd_delta(out, t["dout"])
+    return (np.ascontiguousarray(lse, dtype=np.float32),
+            np.ascontiguousarray(delta, dtype=np.float32))
+
+
+@pytest.mark.parametrize("q_off,nq,k_off,nk", [
+    (0, 700, 0, 700),          # diagonal chunk, ragged
+    (700, 700, 0, 700),        # strictly earlier keys
+    (1000, 333, 517, 300),     # unaligned offsets
+    (384, 256, 256, 512),      # keys straddle the queries
+    (0, 300, 300, 300),        # keys all in the future: nothing added
+])
+def test_partial_backward_matches_oracle(cuda_dev, q_off, nq, k_off, nk):
+    t = _with_dout(_case(1600, 2, 2, 21), 22)
+    lse, delta = _final_lse_delta(t)
+    mp = int(t["positions"].max()) + 1
+    table = ops.rope_table(t["theta"], mp)
+    qs, ks = slice(q_off, q_off + nq), slice(k_off, k_off + nk)
+    seg, pos = t["segment_ids"], t["positions"]
+
+    def c(x, s):
+        return x[:, s].contiguous()
+
+    q_rot = ops.rope_apply(c(t["q"], qs), c(pos, qs), table)
+    k_rot = ops.rope_apply(c(t["k"], ks), c(pos, ks), table)
+    lse_q = torch.from_numpy(np.ascontiguousarray(lse[:, :, qs])).cuda()
+    del_q = torch.from_numpy(np.ascontiguousarray(delta[:, :, qs])).cuda()
+    dq_acc = torch.zeros(q_rot.shape, dtype=torch.float32, device="cuda")
+    dk_acc = torch.zeros(k_rot.shape, dtype=torch.float32, device="cuda")
+    dv_acc = torch.zeros(k_rot.shape, dtype=torch.float32, device="cuda")
+    ops.bwd_block(q_rot, k_rot, c(t["v"], ks), c(t["dout"], qs), lse_q,
+                  del_q, c(seg, qs), c(seg, ks), q_off, k_off, dq_acc,
+                  dk_acc, dv_acc)
+    dq = ops.grad_finish(dq_acc, c(pos, qs), table)
+    dk = ops.grad_finish(dk_acc, c(pos, ks), table)
+    dv = ops.grad_finish(dv_acc)
+    torch.cuda.synchronize()
+    assert ops.last_status() == ops.OK
+    ref = oracle.attn_bwd_partial(
+        t["q"][:, qs], t["k"][:, ks], t["v"][:, ks], t["dout"][:, qs],
+        lse[:, :, qs], delta[:, :, qs], seg[:, qs], seg[:, ks], pos[:, qs],
+        pos[:, ks], q_off, k_off, t["theta"])
+    for name, g, r in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
+        gg = g.float().cpu().numpy()
+        if not r.any():
+            assert not gg.any(), name
+            continue
+        err = np.abs(gg - r).max()
+        assert err <= BWD_REL * np.abs(r).max(), f"{name}: {err}"
+
+
+def test_partial_backward_many_items_per_cta(cuda_dev):
+    # adjacent chunks of a packed row: only the example that straddles the
+    # boundary links them, so most key blocks are seen by no query. Eight
+    # heads give each CTA several items, empty ones (sorted last) after
+    # non-empty ones.
+    t = _with_dout(_case(8192, 8, 1, 29, lo=300, hi=2500), 30)
+    lse, delta = _final_lse_delta(t)
+    mp = int(t["positions"].max()) + 1
+    table = ops.rope_table(t["theta"], mp)
+    qs, ks = slice(4096, 8192), slice(0, 4096)
+    seg, pos = t["segment_ids"], t["positions"]
+
+    def c(x, s):
+        return x[:, s].contiguous()
+
+    q_rot = ops.rope_apply(c(t["q"], qs), c(pos, qs), table)
+    k_rot = ops.rope_apply(c(t["k"], ks), c(pos, ks), table)
+    acc = [torch.zeros(x.shape, dtype=torch.float32, device="cuda")
+           for x in (q_rot, k_rot, k_rot)]
+    ops.bwd_block(q_rot, k_rot, c(t["v"], ks), c(t["dout"], qs),
+                  torch.from_numpy(np.ascontiguousarray(lse[:, :, qs])).cuda(),
+                  torch.from_numpy(np.ascontiguousarray(delta[:, :, qs])).cuda(),
+                  c(seg, qs), c(seg, ks), 4096, 0, *acc)
+    o, l_ = ops.fwd_block(c(t["q"], qs), k_rot, c(t["v"], ks), c(seg, qs),
+                          c(pos, qs), c(seg, ks), 4096, 0, t["theta"], mp)
+    torch.cuda.synchronize()
+    assert ops.last_status() == ops.OK
+    # the reference, on the two heads and the rows / keys that matter
+    for h in (0, 5):
+        sl = slice(h, h + 1)
+        ro, rl = oracle.attn_fwd_partial(
+            t["q"][:, qs, sl], t["k"][:, ks, sl], t["v"][:, ks, sl],
+            seg[:, qs], seg[:, ks], pos[:, qs], pos[:, ks], 4096, 0,
+            t["theta"])
+        assert np.abs(o[:, :, sl].float().cpu().numpy() - ro).max() <= OUT_TOL
+        fin = np.isfinite(rl)
+        assert np.array_equal(np.isfinite(l_[:, sl].cpu().numpy()), fin)
+        ref = oracle.attn_bwd_partial(
+            t["q"][:, qs, sl], t["k"][:, ks, sl], t["v"][:, ks, sl],
+            t["dout"][:, qs, sl], lse[:, sl, qs], delta[:, sl, qs],
+            seg[:, qs], seg[:, ks], pos[:, qs], pos[:, ks], 4096, 0,
+            t["theta"])
+        got = (ops.grad_finish(acc[0][:, :, sl].contiguous(), c(pos, qs),
+                               table),
+               ops.grad_finish(acc[1][:, :, sl].contiguous(), c(pos, ks),
+                               table),
+               ops.grad_finish(acc[2][:, :, sl].contiguous()))
+        for name, g, r in zip(("dq", "dk", "dv"), got, ref):
+            gg = g.float().cpu().numpy()
+            assert not gg[:, np.abs(r).max(axis=(0, 2, 3)) == 0].any(), name
+            err = np.abs(gg - r).max()
+            assert err <= BWD_REL * np.abs(r).max(), f"{name} h{h}: {err}"
+
+
+def test_partial_backward_accumulates(cuda_dev):
+    # two calls over two halves of the keys add up to one call over all
+    t = _with_dout(_case(900, 2, 1, 23), 24)
+    lse, delta = _final_lse_delta(t)
+    mp = int(t["positions"].max()) + 1
+    table = ops.rope_table(t["theta"], mp)
+    q_rot = ops.rope_apply(t["q"], t["positions"], table)
+    k_rot = ops.rope_apply(t["k"], t["positions"], table)
+    lse_d = torch.from_numpy(lse).cuda()
+    del_d = torch.from_numpy(delta).cuda()
+    seg = t["segment_ids"]
+
+    def acc():
+        return [torch.zeros(t["q"].shape, dtype=torch.float32, device="cuda")
+                for _ in range(3)]
+
+    whole = acc()
+    ops.bwd_block(q_rot, k_rot, t["v"], t["dout"], lse_d, del_d, seg, seg, 0,
+                  0, *whole)
+    halves = acc()
+    dk_parts = []
+    for k0, k1 in ((0, 384), (384, 900)):
+        dk_p = torch.zeros((1, k1 - k0, 2, 128), dtype=torch.float32,
+                           device="cuda")
+        dv_p = torch.zeros_like(dk_p)
+        ops.bwd_block(q_rot, k_rot[:, k0:k1].contiguous(),
+                      t["v"][:, k0:k1].contiguous(), t["dout"], lse_d, del_d,
+                      seg, seg[:, k0:k1].contiguous(), 0, k0, halves[0], dk_p,
+                      dv_p)
+        dk_parts.append((dk_p, dv_p))
+    torch.cuda.synchronize()
+    dk_cat = torch.cat([p[0] for p in dk_parts], dim=1)
+    dv_cat = torch.cat([p[1] for p in dk_parts], dim=1)
+    # same tiles, same per-key order: dK and dV are identical; dQ is
+    # summed in another order across the two calls
+    assert torch.equal(dk_cat, whole[1]) and torch.equal(dv_cat, whole[2])
+    scale = whole[0].abs().max().item()
+    assert (halves[0] - whole[0]).abs().max().item() <= 1e-5 * scale
+
+
+@pytest.mark.parametrize("P", [2, 3])
+def test_simulated_ring_backward_matches_dense_oracle(cuda_dev, P):
+    t = _with_dout(_case(1500, 2, 1, 25), 26)
+    mp = int(t["positions"].max()) + 1
+    be = ring.CudaBackend(t["theta"], mp)
+    out, lse = ring.simulate_ring_fwd(t["q"], t["k"], t["v"],
+                                      t["segment_ids"], t["positions"], P, be)
+    dq, dk, dv = ring.simulate_ring_bwd(t["q"], t["k"], t["v"], out,
+                                        t["dout"], lse, t["segment_ids"],
+                                        t["positions"], P, be)
+    torch.cuda.synchronize()
+    assert ops.last_status() == ops.OK
+    ref = oracle.attn_bwd(t["q"], t["k"], t["v"], t["dout"],
+                          t["segment_ids"], t["positions"], t["theta"])
+    for name, g in (("dq", dq), ("dk", dk), ("dv", dv)):
+        gg = g.float().cpu().numpy()
+        err = np.abs(gg - ref[name]).max()
+        assert err <= BWD_REL * np.abs(ref[name]).max(), f"{name}: {err}"
+
+
+def test_ring_of_one_backward_equals_full_backward(cuda_dev):
+    t = _with_dout(_case(1000, 2, 1, 27), 28)
+    mp = int(t["positions"].max()) + 1
+    out, lse = ops.fwd(t["q"], t["k"], t["v"], t["segment_ids"],
+                       t["positions"], t["theta"], mp)
+    full = ops.bwd(t["q"], t["k"], t["v"], out, t["dout"], lse,
+                   t["segment_ids"], t["positions"], t["theta"], mp)
+    be = ring.CudaBackend(t["theta"], mp)
+    one = ring.simulate_ring_bwd(t["q"], t["k"], t["v"], out, t["dout"], lse,
+                                 t["segment_ids"], t["positions"], 1, be)
+    torch.cuda.synchronize()
+    # dK and dV: the same kernel over the same tiles, rounded once (here
+    # through the fp32 accumulator); dQ differs by summation order only
+    for name, a, b in zip(("dq", "dk", "dv"), full, one):
+        scale = a.float().abs().max().item()
+        err = (a.float() - b.float()).abs().max().item()
+        assert err <= 2 ** -7 * scale, f"{name}: {err}"

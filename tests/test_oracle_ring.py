@@ -118,3 +118,25 @@ def test_merge_identity_and_symmetry():
     np.testing.assert_allclose(o1[0, 2, 1], oa[0, 2, 1], atol=1e-15)
     o, l_ = oracle.merge_partials(empty_o, empty_l, empty_o, empty_l)
     assert np.all(o == 0) and np.all(np.isneginf(l_))
+
+
+@pytest.mark.parametrize("P", [1, 2, 3, 5])
+def test_ring_backward_equals_dense(P):
+    q, k, v, seg, pos = _case(8, N=150)
+    dout = np.random.default_rng(9).standard_normal(q.shape)
+    ref = oracle.attn_bwd(q, k, v, dout, seg, pos, 1e5)
+    dq, dk, dv = oracle.ring_bwd(q, k, v, dout, seg, pos, 1e5, P)
+    for got, name in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        np.testing.assert_allclose(got, ref[name], atol=1e-11)
+
+
+def test_backward_partial_of_future_block_is_zero():
+    q, k, v, seg, pos = _case(10, N=120)
+    dout = np.random.default_rng(11).standard_normal(q.shape)
+    out, lse = oracle.attn_fwd(q, k, v, seg, pos, 1e4)
+    delta = oracle.bwd_delta(out, dout)
+    dq, dk, dv = oracle.attn_bwd_partial(
+        q[:, :60], k[:, 60:], v[:, 60:], dout[:, :60], lse[:, :, :60],
+        delta[:, :, :60], seg[:, :60], seg[:, 60:], pos[:, :60], pos[:, 60:],
+        0, 60, 1e4)
+    assert not dq.any() and not dk.any() and not dv.any()

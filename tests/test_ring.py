@@ -66,6 +66,22 @@ def test_simulated_ring_with_oracle_steps_equals_dense(P):
     np.testing.assert_allclose(rl.numpy(), lse, atol=1e-12)
 
 
+@pytest.mark.parametrize("P", [1, 2, 3, 5])
+def test_simulated_ring_backward_with_oracle_steps_equals_dense(P):
+    t = _inputs(N=150, seed=8)
+    g = torch.Generator().manual_seed(3)
+    dout = torch.randn(t["q"].shape, generator=g, dtype=torch.float64)
+    ref = oracle.attn_bwd(t["q"], t["k"], t["v"], dout, t["segment_ids"],
+                          t["positions"], THETA)
+    out = torch.from_numpy(ref["out"])
+    lse = torch.from_numpy(ref["lse"])
+    dq, dk, dv = ring.simulate_ring_bwd(
+        t["q"].double(), t["k"].double(), t["v"].double(), out, dout, lse,
+        t["segment_ids"], t["positions"], P, OracleBackend(THETA))
+    for got, name in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        np.testing.assert_allclose(got.numpy(), ref[name], atol=1e-11)
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
@@ -86,22 +102,34 @@ def _worker(rank, world, port, q):
         t["q"][:, sl].contiguous(), t["k"][:, sl].contiguous(),
         t["v"][:, sl].contiguous(), t["segment_ids"][:, sl].contiguous(),
         t["positions"][:, sl].contiguous(), N, OracleBackend(THETA))
+    g = torch.Generator().manual_seed(3)
+    dout = torch.randn(t["q"].shape, generator=g, dtype=torch.float64)
+    grads = ring.ring_bwd(
+        t["q"][:, sl].double().contiguous(), t["k"][:, sl].double().contiguous(),
+        t["v"][:, sl].double().contiguous(), out, dout[:, sl].contiguous(),
+        lse, t["segment_ids"][:, sl].contiguous(),
+        t["positions"][:, sl].contiguous(), N, OracleBackend(THETA))
     outs = [None] * world
-    torch.distributed.all_gather_object(outs, (out.numpy(), lse.numpy()))
+    torch.distributed.all_gather_object(
+        outs, (out.numpy(), lse.numpy()) + tuple(x.numpy() for x in grads))
     if rank == 0:
-        ref_o, ref_l = oracle.attn_fwd(t["q"], t["k"], t["v"],
-                                       t["segment_ids"], t["positions"],
-                                       THETA)
-        got_o = np.concatenate([o for o, _ in outs], axis=1)
-        got_l = np.concatenate([l_ for _, l_ in outs], axis=2)
-        q.put((float(np.abs(got_o - ref_o).max()),
-               float(np.abs(got_l - ref_l).max())))
+        ref = oracle.attn_bwd(t["q"], t["k"], t["v"], dout,
+                              t["segment_ids"], t["positions"], THETA)
+        errs = [float(np.abs(np.concatenate([o[0] for o in outs], axis=1)
+                             - ref["out"]).max()),
+                float(np.abs(np.concatenate([o[1] for o in outs], axis=2)
+                             - ref["lse"]).max())]
+        for i, name in ((2, "dq"), (3, "dk"), (4, "dv")):
+            errs.append(float(np.abs(np.concatenate([o[i] for o in outs],
+                                                    axis=1)
+                                     - ref[name]).max()))
+        q.put(errs)
     torch.distributed.barrier()
     torch.distributed.destroy_process_group()
 
 
 @pytest.mark.parametrize("world", [2, 3])
-def test_ring_over_gloo_ranks_equals_dense(world):
+def test_ring_forward_and_backward_over_gloo_ranks_equals_dense(world):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
@@ -109,8 +137,9 @@ def test_ring_over_gloo_ranks_equals_dense(world):
              for r in range(world)]
     for p in procs:
         p.start()
-    err_o, err_l = q.get(timeout=180)
+    errs = q.get(timeout=180)
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    assert err_o < 1e-12 and err_l < 1e-12
+    # forward out, lse; then dq, dk, dv after the ring backward
+    assert max(errs[:2]) < 1e-12 and max(errs[2:]) < 1e-11, errs
