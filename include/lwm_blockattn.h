@@ -86,6 +86,15 @@ typedef enum {
 typedef enum { LWM_DTYPE_BF16 = 0, LWM_DTYPE_FP32 = 1 } lwm_dtype;
 typedef enum { LWM_QK_BF16 = 0, LWM_QK_BF16X3 = 1 } lwm_qk_precision;
 
+/* Which head dims RoPE rotates together with frequency theta^(-2k/D):
+ * LWM_ROPE_INTERLEAVED pairs (x[2k], x[2k+1]) (the Jax/EasyLM layout the
+ * LWM checkpoints were trained in); LWM_ROPE_HALF pairs (x[k], x[k+D/2]),
+ * the rotate-half layout of Hugging Face LlamaForCausalLM, which is how the
+ * PyTorch models load ("LWM：突破 100 万 Token 的开源大模型", 脚本运行说明,
+ * 运行 PyTorch 模型). The two give the same attention once the head dims of
+ * q and k are permuted; gradients come back in the inputs' layout. */
+typedef enum { LWM_ROPE_INTERLEAVED = 0, LWM_ROPE_HALF = 1 } lwm_rope_layout;
+
 /* Tile classes written by lwm_blockattn_classify. */
 enum { LWM_TILE_EMPTY = 0, LWM_TILE_PARTIAL = 1, LWM_TILE_FULL = 2 };
 
@@ -110,7 +119,8 @@ LWM_API size_t lwm_blockattn_bwd_workspace_size(int B, int N, int H, int D,
 
 /* Forward. Writes out [B][N][H][D] (dtype) and lse [B][H][N] (fp32,
  * natural log of the softmax denominator of the scaled scores).
- * theta > 0 is the RoPE base; positions must lie in [0, max_pos).
+ * theta > 0 is the RoPE base; positions must lie in [0, max_pos);
+ * rope_layout is an lwm_rope_layout.
  * The workspace is scratch owned by the caller (>= the size above, 256-byte
  * aligned); its content on entry does not matter and is clobbered.
  * Returns LWM_OK or an error status (nothing launched on error). */
@@ -118,7 +128,7 @@ LWM_API int lwm_blockattn_fwd(const void* q, const void* k, const void* v,
                       const int32_t* segment_ids, const int32_t* positions,
                       double theta, int block_q, int block_k, int max_pos,
                       int B, int N, int H, int D, int dtype, int qk_precision,
-                      void* out, float* lse,
+                      int rope_layout, void* out, float* lse,
                       void* workspace, size_t workspace_bytes, void* stream);
 
 /* Backward. Given the forward's inputs, its out and lse, and dout (the
@@ -131,7 +141,7 @@ LWM_API int lwm_blockattn_bwd(const void* q, const void* k, const void* v,
                       const int32_t* segment_ids, const int32_t* positions,
                       double theta, int block_q, int block_k, int max_pos,
                       int B, int N, int H, int D, int dtype, int qk_precision,
-                      void* dq, void* dk, void* dv,
+                      int rope_layout, void* dq, void* dk, void* dv,
                       void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------
@@ -153,7 +163,7 @@ LWM_API size_t lwm_blockattn_fwd_block_workspace_size(int B, int Nq, int Nk,
  * lse = -inf.
  *   q      [B][Nq][H][D] bf16, un-rotated; rotated here by R(pos_q)
  *   k_rot  [B][Nk][H][D] bf16, keys already rotated (lwm_blockattn_rope_apply
- *          with their own positions)
+ *          with their own positions and the same rope_layout)
  *   v      [B][Nk][H][D] bf16
  *   seg_q  [B][Nq], pos_q [B][Nq], seg_k [B][Nk] int32; segment ids
  *          non-decreasing along the whole sequence
@@ -166,7 +176,8 @@ LWM_API int lwm_blockattn_fwd_block(const void* q, const void* k_rot,
                                     const int32_t* pos_q, const int32_t* seg_k,
                                     int q_off, int k_off, double theta,
                                     int max_pos, int B, int Nq, int Nk, int H,
-                                    int D, void* out, float* lse,
+                                    int D, int rope_layout, void* out,
+                                    float* lse,
                                     void* workspace, size_t workspace_bytes,
                                     void* stream);
 
@@ -219,13 +230,15 @@ LWM_API int lwm_blockattn_bwd_block(const void* q_rot, const void* k_rot,
 
 /* grad (bf16 [B][N][H][D]) from an fp32 accumulator of the same shape:
  * with positions (int32 [B][N]) and a table from lwm_blockattn_rope_table,
- * grad = R(-pos) acc / sqrt(D) (dq, dk); with positions == NULL,
- * grad = acc (dv). Async on stream. */
+ * grad = R(-pos) acc / sqrt(D) (dq, dk; pairs as rope_layout says, the
+ * layout the accumulator was built in); with positions == NULL, grad = acc
+ * (dv). Async on stream. */
 LWM_API int lwm_blockattn_grad_finish(const float* acc,
                                       const int32_t* positions,
                                       const float* rope_table, int max_pos,
                                       int B, int N, int H, int D, int dtype,
-                                      void* grad, void* stream);
+                                      int rope_layout, void* grad,
+                                      void* stream);
 
 /* Tile classifier (exported so it can be checked bit-exactly). For each
  * batch row b and query block t (Tq = ceil(N/block_q) blocks), key blocks
@@ -277,14 +290,16 @@ LWM_API int lwm_blockattn_version(void);
  * Decode (inference against a long KV cache).
  *
  * lwm_blockattn_rope_apply: x_rot = R(pos) x for a bf16 [B][N][H][D] tensor
- * (D == 128, interleaved pairs), using a table made by
+ * (D == 128, pairs as rope_layout says; x_rot keeps that layout), using a
+ * table made by
  * lwm_blockattn_rope_table for positions [0, max_pos). Rotating keys once as
  * they enter a cache lets decode read them as they are. Async on stream.
  * Returns LWM_OK or an error status (nothing launched on error). */
 LWM_API int lwm_blockattn_rope_apply(const void* x, const int32_t* positions,
                                      const float* rope_table, int max_pos,
                                      int B, int N, int H, int D, int dtype,
-                                     void* x_rot, void* stream);
+                                     int rope_layout, void* x_rot,
+                                     void* stream);
 
 /* Bytes of workspace lwm_blockattn_decode needs (per-chunk partial sums). */
 LWM_API size_t lwm_blockattn_decode_workspace_size(int B, int H, int D,
@@ -292,7 +307,8 @@ LWM_API size_t lwm_blockattn_decode_workspace_size(int B, int H, int D,
 
 /* One query token per (b, h) against a cache of L tokens.
  *   q        [B][H][D] bf16, un-rotated; rotated here by R(q_pos[b])
- *   k_rot    [B][L][H][D] bf16, keys already rotated (rope_apply)
+ *   k_rot    [B][L][H][D] bf16, keys already rotated (rope_apply, same
+ *            rope_layout)
  *   v        [B][L][H][D] bf16
  *   kv_start, kv_len [B] int32: the query sees cached keys
  *            [kv_start[b], kv_len[b]) (its own packed example: the query is
@@ -308,9 +324,10 @@ LWM_API int lwm_blockattn_decode(const void* q, const void* k_rot,
                                  const void* v, const int32_t* kv_start,
                                  const int32_t* kv_len, const int32_t* q_pos,
                                  const float* rope_table, int max_pos, int B,
-                                 int L, int H, int D, int dtype, void* out,
-                                 float* lse, void* workspace,
-                                 size_t workspace_bytes, void* stream);
+                                 int L, int H, int D, int dtype,
+                                 int rope_layout, void* out, float* lse,
+                                 void* workspace, size_t workspace_bytes,
+                                 void* stream);
 
 /* Self-test of the failure path: launches one small CTA that waits on an
  * mbarrier nobody arrives on, with the same bounded wait the attention
@@ -351,8 +368,8 @@ LWM_API int lwm_blockattn_fwd_noalloc(const void* q, const void* k,
                                       const int32_t* positions, double theta,
                                       int block_q, int block_k, int max_pos,
                                       int B, int N, int H, int D, int dtype,
-                                      int qk_precision, void* out,
-                                      float* lse, void* stream);
+                                      int qk_precision, int rope_layout,
+                                      void* out, float* lse, void* stream);
 
 #ifdef __cplusplus
 }

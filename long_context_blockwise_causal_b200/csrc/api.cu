@@ -145,6 +145,10 @@ int shape_status(int D, int block_q, int block_k) {
   return LWM_OK;
 }
 
+inline bool layout_ok(int rope_layout) {
+  return rope_layout == LWM_ROPE_INTERLEAVED || rope_layout == LWM_ROPE_HALF;
+}
+
 inline bool aligned16(const void* p) {
   return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
 }
@@ -188,7 +192,7 @@ int run_backward(BwdArgs a, const int32_t* seg_q, const int32_t* seg_k,
 int run_forward(const void* q, const void* k_rot, const void* k_rot_lo,
                 const void* v, const int32_t* seg_q, const int32_t* pos_q,
                 const int32_t* seg_k, int q_off, int k_off, int B, int Nq,
-                int Nk, int H, bool x3, void* out, float* lse,
+                int Nk, int H, bool x3, bool half, void* out, float* lse,
                 const Workspace& w, cudaStream_t st) {
   LWM_TRY(launch_cross_meta(seg_q, seg_k, B, Nq, Nk, q_off, k_off, w.row_lo,
                             w.row_hi, w.kv_lo, w.kv_hi, w.lo_max, w.hi_min,
@@ -204,6 +208,7 @@ int run_forward(const void* q, const void* k_rot, const void* k_rot_lo,
   a.order = w.order_fwd; a.counter = w.counter;
   a.B = B; a.Nq = Nq; a.Nk = Nk; a.H = H; a.k_off = k_off;
   a.qk_x3 = x3;
+  a.rope_half = half;
   a.status = status_word();
   if (!a.status) return LWM_ERR_CUDA;
   return cuda_status(launch_fwd_tc(a, st));
@@ -233,20 +238,22 @@ int lwm_blockattn_version(void) { return LWM_BLOCKATTN_VERSION; }
 
 int lwm_blockattn_rope_apply(const void* x, const int32_t* positions,
                              const float* rope_table, int max_pos, int B,
-                             int N, int H, int D, int dtype, void* x_rot,
-                             void* stream) {
+                             int N, int H, int D, int dtype, int rope_layout,
+                             void* x_rot, void* stream) {
   if (B < 0 || N < 0 || H < 0 || max_pos < 0 ||
       (int64_t(B) * N) >= (int64_t(1) << 31))
     return LWM_ERR_INVALID_ARG;
   if (D != kHeadDim) return LWM_ERR_UNSUPPORTED;
   if (dtype != LWM_DTYPE_BF16) return LWM_ERR_UNSUPPORTED;
+  if (!layout_ok(rope_layout)) return LWM_ERR_INVALID_ARG;
   if (int64_t(B) * N * H == 0) return LWM_OK;
   const void* ptrs[] = {x, positions, rope_table, x_rot};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return LWM_ERR_INVALID_ARG;
   if (max_pos < 1) return LWM_ERR_INVALID_ARG;
   return cuda_status(launch_rope_apply(x, positions, rope_table, B, N, H,
-                                       x_rot, nullptr,
+                                       rope_layout == LWM_ROPE_HALF, x_rot,
+                                       nullptr,
                                        static_cast<cudaStream_t>(stream)));
 }
 
@@ -261,12 +268,14 @@ int lwm_blockattn_decode(const void* q, const void* k_rot, const void* v,
                          const int32_t* kv_start, const int32_t* kv_len,
                          const int32_t* q_pos, const float* rope_table,
                          int max_pos, int B, int L, int H, int D, int dtype,
-                         void* out, float* lse, void* workspace,
-                         size_t workspace_bytes, void* stream) {
+                         int rope_layout, void* out, float* lse,
+                         void* workspace, size_t workspace_bytes,
+                         void* stream) {
   if (B < 0 || L < 0 || H < 0 || max_pos < 0 ||
       (int64_t(B) * L) >= (int64_t(1) << 31))
     return LWM_ERR_INVALID_ARG;
   if (D != kHeadDim || dtype != LWM_DTYPE_BF16) return LWM_ERR_UNSUPPORTED;
+  if (!layout_ok(rope_layout)) return LWM_ERR_INVALID_ARG;
   if (int64_t(B) * H == 0) return LWM_OK;
   const void* ptrs[] = {q, k_rot, v, kv_start, kv_len, q_pos, rope_table,
                         out, lse, workspace};
@@ -282,7 +291,8 @@ int lwm_blockattn_decode(const void* q, const void* k_rot, const void* v,
   float* part_acc =
       reinterpret_cast<float*>(ws + 2 * align_up(slots * sizeof(float)));
   return cuda_status(launch_decode(q, k_rot, v, kv_start, kv_len, q_pos,
-                                   rope_table, max_pos, B, L, H, out, lse,
+                                   rope_table, max_pos, B, L, H,
+                                   rope_layout == LWM_ROPE_HALF, out, lse,
                                    part_m, part_l, part_acc,
                                    static_cast<cudaStream_t>(stream)));
 }
@@ -326,10 +336,12 @@ int lwm_blockattn_fwd(const void* q, const void* k, const void* v,
                       const int32_t* segment_ids, const int32_t* positions,
                       double theta, int block_q, int block_k, int max_pos,
                       int B, int N, int H, int D, int dtype, int qk_precision,
-                      void* out, float* lse, void* workspace,
+                      int rope_layout, void* out, float* lse, void* workspace,
                       size_t workspace_bytes, void* stream) {
   if (!sizes_ok(B, N, H, D, block_q, block_k, max_pos))
     return LWM_ERR_INVALID_ARG;
+  if (!layout_ok(rope_layout)) return LWM_ERR_INVALID_ARG;
+  const bool half = rope_layout == LWM_ROPE_HALF;
   if (!(theta > 0.0) || !std::isfinite(theta)) return LWM_ERR_INVALID_ARG;
   if (dtype != LWM_DTYPE_BF16 && dtype != LWM_DTYPE_FP32)
     return LWM_ERR_INVALID_ARG;
@@ -353,14 +365,14 @@ int lwm_blockattn_fwd(const void* q, const void* k, const void* v,
     return cuda_status(launch_fwd_simt<float>(
         static_cast<const float*>(q), static_cast<const float*>(k),
         static_cast<const float*>(v), segment_ids, positions, w.table,
-        w.kv_lo, B, N, H, static_cast<float*>(out), lse, st));
+        w.kv_lo, B, N, H, half, static_cast<float*>(out), lse, st));
   }
   // keys are reused by every query block that sees them: rotate them once
-  LWM_TRY(launch_rope_apply(k, positions, w.table, B, N, H, w.k_rot,
+  LWM_TRY(launch_rope_apply(k, positions, w.table, B, N, H, half, w.k_rot,
                             w.k_rot_lo, st));
   return run_forward(q, w.k_rot, w.k_rot_lo, v, segment_ids, positions,
                      segment_ids, 0, 0, B, N, N, H,
-                     qk_precision == LWM_QK_BF16X3, out, lse, w, st);
+                     qk_precision == LWM_QK_BF16X3, half, out, lse, w, st);
 }
 
 size_t lwm_blockattn_fwd_block_workspace_size(int B, int Nq, int Nk, int H,
@@ -375,13 +387,14 @@ int lwm_blockattn_fwd_block(const void* q, const void* k_rot, const void* v,
                             const int32_t* seg_q, const int32_t* pos_q,
                             const int32_t* seg_k, int q_off, int k_off,
                             double theta, int max_pos, int B, int Nq, int Nk,
-                            int H, int D, void* out, float* lse,
-                            void* workspace, size_t workspace_bytes,
-                            void* stream) {
+                            int H, int D, int rope_layout, void* out,
+                            float* lse, void* workspace,
+                            size_t workspace_bytes, void* stream) {
   if (!sizes_ok(B, Nq, H, D, kBlock, kBlock, max_pos) || Nk < 0 ||
       q_off < 0 || k_off < 0 || (int64_t(B) * Nk) >= (int64_t(1) << 31))
     return LWM_ERR_INVALID_ARG;
   if (!(theta > 0.0) || !std::isfinite(theta)) return LWM_ERR_INVALID_ARG;
+  if (!layout_ok(rope_layout)) return LWM_ERR_INVALID_ARG;
   if (D != kHeadDim) return LWM_ERR_UNSUPPORTED;
   if (int64_t(B) * Nq * H == 0) return LWM_OK;
   if (max_pos < 1) return LWM_ERR_INVALID_ARG;
@@ -404,7 +417,8 @@ int lwm_blockattn_fwd_block(const void* q, const void* k_rot, const void* v,
   }
   LWM_TRY(launch_rope_table(theta, D, max_pos, w.table, st));
   return run_forward(q, k_rot, nullptr, v, seg_q, pos_q, seg_k, q_off, k_off,
-                     B, Nq, Nk, H, false, out, lse, w, st);
+                     B, Nq, Nk, H, false, rope_layout == LWM_ROPE_HALF, out,
+                     lse, w, st);
 }
 
 int lwm_blockattn_merge(void* out, float* lse, const void* out_part,
@@ -425,11 +439,14 @@ int lwm_blockattn_bwd(const void* q, const void* k, const void* v,
                       const int32_t* segment_ids, const int32_t* positions,
                       double theta, int block_q, int block_k, int max_pos,
                       int B, int N, int H, int D, int dtype, int qk_precision,
-                      void* dq, void* dk, void* dv, void* workspace,
+                      int rope_layout, void* dq, void* dk, void* dv,
+                      void* workspace,
                       size_t workspace_bytes, void* stream) {
   if (!sizes_ok(B, N, H, D, block_q, block_k, max_pos))
     return LWM_ERR_INVALID_ARG;
   if (!(theta > 0.0) || !std::isfinite(theta)) return LWM_ERR_INVALID_ARG;
+  if (!layout_ok(rope_layout)) return LWM_ERR_INVALID_ARG;
+  const bool half = rope_layout == LWM_ROPE_HALF;
   if (dtype != LWM_DTYPE_BF16 && dtype != LWM_DTYPE_FP32)
     return LWM_ERR_INVALID_ARG;
   if (qk_precision != LWM_QK_BF16 && qk_precision != LWM_QK_BF16X3)
@@ -458,11 +475,11 @@ int lwm_blockattn_bwd(const void* q, const void* k, const void* v,
     LWM_TRY(launch_bwd_simt<T>(
         static_cast<const T*>(q), static_cast<const T*>(k),
         static_cast<const T*>(v), static_cast<const T*>(dout), lse, w.delta,
-        segment_ids, positions, w.table, B, N, H, w.dq_acc,
+        segment_ids, positions, w.table, B, N, H, half, w.dq_acc,
         static_cast<T*>(dk), static_cast<T*>(dv), st));
     return cuda_status(launch_dq_convert<T>(w.dq_acc, positions, w.table, B,
-                                            N, H, scale, static_cast<T*>(dq),
-                                            st));
+                                            N, H, scale, half,
+                                            static_cast<T*>(dq), st));
   }
   using T = __nv_bfloat16;
   LWM_TRY(launch_bwd_delta<T>(static_cast<const T*>(out),
@@ -473,25 +490,26 @@ int lwm_blockattn_bwd(const void* q, const void* k, const void* v,
     LWM_TRY(launch_bwd_simt<T>(
         static_cast<const T*>(q), static_cast<const T*>(k),
         static_cast<const T*>(v), static_cast<const T*>(dout), lse, w.delta,
-        segment_ids, positions, w.table, B, N, H, w.dq_acc,
+        segment_ids, positions, w.table, B, N, H, half, w.dq_acc,
         static_cast<T*>(dk), static_cast<T*>(dv), st));
   } else {
     // queries and keys are both re-read inside the key-major sweep: rotate
     // them once
-    LWM_TRY(launch_rope_apply(q, positions, w.table, B, N, H, w.q_rot,
+    LWM_TRY(launch_rope_apply(q, positions, w.table, B, N, H, half, w.q_rot,
                               nullptr, st));
-    LWM_TRY(launch_rope_apply(k, positions, w.table, B, N, H, w.k_rot,
+    LWM_TRY(launch_rope_apply(k, positions, w.table, B, N, H, half, w.k_rot,
                               nullptr, st));
     BwdArgs a{};
     a.q_rot = w.q_rot; a.k_rot = w.k_rot; a.v = v; a.dout = dout;
     a.lse = lse; a.delta = w.delta; a.pos_k = positions; a.table = w.table;
     a.dq_acc = w.dq_acc; a.dk = dk; a.dv = dv;
-    a.B = B; a.Nq = N; a.Nk = N; a.H = H; a.q_off = 0;
+    a.B = B; a.Nq = N; a.Nk = N; a.H = H; a.q_off = 0; a.rope_half = half;
     s = run_backward(a, segment_ids, segment_ids, 0, w, st);
     if (s != LWM_OK) return s;
   }
   return cuda_status(launch_dq_convert<T>(w.dq_acc, positions, w.table, B, N,
-                                          H, scale, static_cast<T*>(dq), st));
+                                          H, scale, half, static_cast<T*>(dq),
+                                          st));
 }
 
 size_t lwm_blockattn_bwd_block_workspace_size(int B, int Nq, int Nk, int H,
@@ -550,10 +568,11 @@ int lwm_blockattn_bwd_delta(const void* out, const void* dout, int B, int N,
 
 int lwm_blockattn_grad_finish(const float* acc, const int32_t* positions,
                               const float* rope_table, int max_pos, int B,
-                              int N, int H, int D, int dtype, void* grad,
-                              void* stream) {
+                              int N, int H, int D, int dtype, int rope_layout,
+                              void* grad, void* stream) {
   if (B < 0 || N < 0 || H < 0 || max_pos < 0) return LWM_ERR_INVALID_ARG;
   if (D != kHeadDim || dtype != LWM_DTYPE_BF16) return LWM_ERR_UNSUPPORTED;
+  if (!layout_ok(rope_layout)) return LWM_ERR_INVALID_ARG;
   if (int64_t(B) * N * H == 0) return LWM_OK;
   if (!acc || !grad || !aligned16(acc) || !aligned16(grad))
     return LWM_ERR_INVALID_ARG;
@@ -561,7 +580,8 @@ int lwm_blockattn_grad_finish(const float* acc, const int32_t* positions,
   const float scale = positions ? 1.f / std::sqrt(float(D)) : 1.f;
   return cuda_status(launch_dq_convert<__nv_bfloat16>(
       acc, positions, rope_table, B, N, H, scale,
-      static_cast<__nv_bfloat16*>(grad), static_cast<cudaStream_t>(stream)));
+      rope_layout == LWM_ROPE_HALF, static_cast<__nv_bfloat16*>(grad),
+      static_cast<cudaStream_t>(stream)));
 }
 
 int lwm_blockattn_classify(const int32_t* segment_ids, int B, int N,

@@ -59,6 +59,53 @@ __global__ void rope_apply_kernel(const __nv_bfloat16* __restrict__ x,
   }
 }
 
+// Same for the rotate-half layout: pair k = (x[k], x[k + 64]). Item c of a
+// row rotates dims 8c .. 8c+7 with dims 64 + 8c .. 64 + 8c + 7
+// (frequencies 8c .. 8c+7) and writes them back in that layout.
+__global__ void rope_apply_half_kernel(const __nv_bfloat16* __restrict__ x,
+                                       const int32_t* __restrict__ pos,
+                                       const float2* __restrict__ table,
+                                       int64_t items, int H,
+                                       __nv_bfloat16* __restrict__ hi,
+                                       __nv_bfloat16* __restrict__ lo) {
+  constexpr int kItemsPerRow = kHeadDim / 16;
+  for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+       e < items; e += int64_t(gridDim.x) * blockDim.x) {
+    const int c = int(e % kItemsPerRow);
+    const int64_t row = e / kItemsPerRow;  // (b, n, h)
+    const int p = pos[row / H];
+    const float4* t = reinterpret_cast<const float4*>(
+        table + int64_t(p) * (kHeadDim / 2) + c * 8);
+    const int64_t i0 = row * (kHeadDim / 8) + c;   // uint4 index, first half
+    const int64_t i1 = i0 + kHeadDim / 16;         // second half
+    const uint4 wa = reinterpret_cast<const uint4*>(x)[i0];
+    const uint4 wb = reinterpret_cast<const uint4*>(x)[i1];
+    const uint32_t as[4] = {wa.x, wa.y, wa.z, wa.w};
+    const uint32_t bs[4] = {wb.x, wb.y, wb.z, wb.w};
+    uint32_t ha[4], hb[4], la[4], lb[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float4 cs = __ldg(t + k);  // pairs 8c + 2k, 8c + 2k + 1
+      const float a0 = bf16lo_to_f32(as[k]), a1 = bf16hi_to_f32(as[k]);
+      const float b0 = bf16lo_to_f32(bs[k]), b1 = bf16hi_to_f32(bs[k]);
+      const float ra0 = fmaf(a0, cs.x, -b0 * cs.y);
+      const float rb0 = fmaf(a0, cs.y, b0 * cs.x);
+      const float ra1 = fmaf(a1, cs.z, -b1 * cs.w);
+      const float rb1 = fmaf(a1, cs.w, b1 * cs.z);
+      ha[k] = pack_bf16x2(ra0, ra1);
+      hb[k] = pack_bf16x2(rb0, rb1);
+      la[k] = pack_bf16x2(ra0 - bf16lo_to_f32(ha[k]), ra1 - bf16hi_to_f32(ha[k]));
+      lb[k] = pack_bf16x2(rb0 - bf16lo_to_f32(hb[k]), rb1 - bf16hi_to_f32(hb[k]));
+    }
+    reinterpret_cast<uint4*>(hi)[i0] = make_uint4(ha[0], ha[1], ha[2], ha[3]);
+    reinterpret_cast<uint4*>(hi)[i1] = make_uint4(hb[0], hb[1], hb[2], hb[3]);
+    if (lo) {
+      reinterpret_cast<uint4*>(lo)[i0] = make_uint4(la[0], la[1], la[2], la[3]);
+      reinterpret_cast<uint4*>(lo)[i1] = make_uint4(lb[0], lb[1], lb[2], lb[3]);
+    }
+  }
+}
+
 // First index of the contiguous run holding row i (ids non-decreasing).
 __device__ __forceinline__ int run_start(const int32_t* __restrict__ seg,
                                          int i) {
@@ -457,28 +504,35 @@ template <typename T>
 __global__ void dq_convert_kernel(const float* __restrict__ acc,
                                   const int32_t* __restrict__ pos,
                                   const float2* __restrict__ table, int B,
-                                  int N, int H, float scale,
+                                  int N, int H, float scale, bool half,
                                   T* __restrict__ dq) {
   int64_t total = int64_t(B) * N * H * (kHeadDim / 2);
   for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
        e < total; e += int64_t(gridDim.x) * blockDim.x) {
-    int k = int(e % (kHeadDim / 2));
+    int k = int(e % (kHeadDim / 2));   // pair index
     int64_t bnh = e / (kHeadDim / 2);
     int64_t bn = bnh / H;
-    float2 x = reinterpret_cast<const float2*>(acc)[e];
-    x.x *= scale;
-    x.y *= scale;
+    // the pair's two elements: (2k, 2k+1) interleaved, (k, k+64) half
+    const int64_t i0 = bnh * kHeadDim + (half ? k : 2 * k);
+    const int64_t i1 = i0 + (half ? kHeadDim / 2 : 1);
+    float xa, xb;
+    if (half) {
+      xa = acc[i0] * scale;
+      xb = acc[i1] * scale;
+    } else {
+      const float2 x = reinterpret_cast<const float2*>(acc)[e];
+      xa = x.x * scale;
+      xb = x.y * scale;
+    }
     if (!pos) {  // plain conversion
-      dq[2 * e] = T(x.x);
-      dq[2 * e + 1] = T(x.y);
+      dq[i0] = T(xa);
+      dq[i1] = T(xb);
       continue;
     }
     float2 cs = table[int64_t(pos[bn]) * (kHeadDim / 2) + k];
     // inverse rotation: (a, b) -> (a c + b s, -a s + b c)
-    float a = x.x * cs.x + x.y * cs.y;
-    float c = x.y * cs.x - x.x * cs.y;
-    dq[2 * e] = T(a);
-    dq[2 * e + 1] = T(c);
+    dq[i0] = T(xa * cs.x + xb * cs.y);
+    dq[i1] = T(xb * cs.x - xa * cs.y);
   }
 }
 
@@ -512,13 +566,21 @@ cudaError_t launch_block_meta(const int32_t* seg, int B, int N, int bq, int bk,
 
 cudaError_t launch_rope_apply(const void* x, const int32_t* pos,
                               const float* table, int B, int N, int H,
-                              void* hi, void* lo, cudaStream_t st) {
+                              bool half, void* hi, void* lo, cudaStream_t st) {
   int64_t chunks = int64_t(B) * N * H * (kHeadDim / 8);
   if (chunks == 0) return cudaSuccess;
-  rope_apply_kernel<<<grid_for(chunks, 256, 148 * 16), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(x), pos,
-      reinterpret_cast<const float2*>(table), chunks, H,
-      static_cast<__nv_bfloat16*>(hi), static_cast<__nv_bfloat16*>(lo));
+  if (half) {
+    rope_apply_half_kernel<<<grid_for(chunks / 2, 256, 148 * 16), 256, 0,
+                             st>>>(
+        static_cast<const __nv_bfloat16*>(x), pos,
+        reinterpret_cast<const float2*>(table), chunks / 2, H,
+        static_cast<__nv_bfloat16*>(hi), static_cast<__nv_bfloat16*>(lo));
+  } else {
+    rope_apply_kernel<<<grid_for(chunks, 256, 148 * 16), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), pos,
+        reinterpret_cast<const float2*>(table), chunks, H,
+        static_cast<__nv_bfloat16*>(hi), static_cast<__nv_bfloat16*>(lo));
+  }
   note_launch();
   return cudaGetLastError();
 }
@@ -668,11 +730,12 @@ cudaError_t launch_bwd_delta(const T* out, const T* dout, int B, int N, int H,
 template <typename T>
 cudaError_t launch_dq_convert(const float* acc, const int32_t* pos,
                               const float* table, int B, int N, int H,
-                              float scale, T* dq, cudaStream_t st) {
+                              float scale, bool half, T* dq, cudaStream_t st) {
   int64_t n = int64_t(B) * N * H * (kHeadDim / 2);
   if (n == 0) return cudaSuccess;
   dq_convert_kernel<T><<<grid_for(n, 256, 148 * 32), 256, 0, st>>>(
-      acc, pos, reinterpret_cast<const float2*>(table), B, N, H, scale, dq);
+      acc, pos, reinterpret_cast<const float2*>(table), B, N, H, scale, half,
+      dq);
   note_launch();
   return cudaGetLastError();
 }
@@ -686,11 +749,12 @@ template cudaError_t launch_bwd_delta<float>(const float*, const float*, int,
 template cudaError_t launch_dq_convert<__nv_bfloat16>(const float*,
                                                       const int32_t*,
                                                       const float*, int, int,
-                                                      int, float,
+                                                      int, float, bool,
                                                       __nv_bfloat16*,
                                                       cudaStream_t);
 template cudaError_t launch_dq_convert<float>(const float*, const int32_t*,
                                               const float*, int, int, int,
-                                              float, float*, cudaStream_t);
+                                              float, bool, float*,
+                                              cudaStream_t);
 
 }  // namespace lwm

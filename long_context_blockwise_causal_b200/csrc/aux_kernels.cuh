@@ -11,10 +11,11 @@ cudaError_t launch_rope_table(double theta, int D, int max_pos, float* table,
                               cudaStream_t st);
 cudaError_t launch_block_meta(const int32_t* seg, int B, int N, int bq, int bk,
                               int32_t* kv_lo, int32_t* kv_hi, cudaStream_t st);
-// hi = R(pos) x in bf16, lo = residual (skipped when lo == nullptr).
+// hi = R(pos) x in bf16, lo = residual (skipped when lo == nullptr); pairs
+// (2k, 2k+1), or (k, k+64) when `half` (rotate-half layout, kept on output).
 cudaError_t launch_rope_apply(const void* x, const int32_t* pos,
                               const float* table, int B, int N, int H,
-                              void* hi, void* lo, cudaStream_t st);
+                              bool half, void* hi, void* lo, cudaStream_t st);
 // Per-row visible key ranges of queries [q_off, q_off+Nq) against keys
 // [k_off, k_off+Nk) (global indices), and per query block the key-block
 // range plus the shared row range used for the all-visible test.
@@ -58,23 +59,27 @@ cudaError_t launch_check_inputs(const int32_t* seg, const int32_t* pos, int B,
 template <typename T>
 cudaError_t launch_bwd_delta(const T* out, const T* dout, int B, int N, int H,
                              float* delta, cudaStream_t st);
-// dq = R(-pos) acc * scale in T; pos == nullptr: dq = acc * scale.
+// dq = R(-pos) acc * scale in T (pairs as in launch_rope_apply);
+// pos == nullptr: dq = acc * scale.
 template <typename T>
 cudaError_t launch_dq_convert(const float* acc, const int32_t* pos,
                               const float* table, int B, int N, int H,
-                              float scale, T* dq, cudaStream_t st);
+                              float scale, bool half, T* dq, cudaStream_t st);
 
 // CUDA-core kernels (fp32 arithmetic), any I/O type.
+// `half`: q and k in the rotate-half layout (dk written, and dq_acc
+// accumulated, in that layout too).
 template <typename T>
 cudaError_t launch_fwd_simt(const T* q, const T* k, const T* v,
                             const int32_t* seg, const int32_t* pos,
                             const float* table, const int32_t* kv_lo, int B,
-                            int N, int H, T* out, float* lse, cudaStream_t st);
+                            int N, int H, bool half, T* out, float* lse,
+                            cudaStream_t st);
 template <typename T>
 cudaError_t launch_bwd_simt(const T* q, const T* k, const T* v, const T* dout,
                             const float* lse, const float* delta,
                             const int32_t* seg, const int32_t* pos,
-                            const float* table, int B, int N, int H,
+                            const float* table, int B, int N, int H, bool half,
                             float* dq_acc, T* dk, T* dv, cudaStream_t st);
 
 }  // namespace lwm

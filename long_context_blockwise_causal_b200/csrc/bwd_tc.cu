@@ -72,6 +72,7 @@ struct BwdParams {
   float* dv_acc;
   int* status;
   int B, Nq, Nk, H, Tk, G, q_off, total_items;
+  int rope_half;
   float scale_log2, scale;
 };
 
@@ -359,6 +360,44 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       const float4* trow = reinterpret_cast<const float4*>(
           p.table + int64_t(valid_k ? __ldg(p.pos_k + rowbase + kj) : 0) *
                         (kHeadDim / 2));
+      if (p.rope_half) {
+        // pair k = (dim k, dim k + 64): columns c*32.. with (c+2)*32..
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t va[32], vb[32];
+          tmem_ld32(tD + lane_off + c * 32, va);
+          tmem_ld32(tD + lane_off + (c + 2) * 32, vb);
+          tmem_wait_ld();
+          if (!seen)
+#pragma unroll
+            for (int x = 0; x < 32; ++x) va[x] = vb[x] = 0u;
+          if (valid_k) {
+            uint32_t oa[16], ob[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {  // pairs c*32 + 2e, 2e + 1
+              const float4 cs = __ldg(trow + c * 16 + e);
+              const float a0 = __uint_as_float(va[2 * e]) * p.scale;
+              const float a1 = __uint_as_float(va[2 * e + 1]) * p.scale;
+              const float b0 = __uint_as_float(vb[2 * e]) * p.scale;
+              const float b1 = __uint_as_float(vb[2 * e + 1]) * p.scale;
+              // R(-pos): (a, b) -> (a c + b s, b c - a s)
+              oa[e] = pack_bf16x2(fmaf(a0, cs.x, b0 * cs.y),
+                                  fmaf(a1, cs.z, b1 * cs.w));
+              ob[e] = pack_bf16x2(fmaf(b0, cs.x, -a0 * cs.y),
+                                  fmaf(b1, cs.z, -a1 * cs.w));
+            }
+            uint4* da = reinterpret_cast<uint4*>(p.dk + orow + c * 32);
+            uint4* db = reinterpret_cast<uint4*>(p.dk + orow + (c + 2) * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              da[e] = make_uint4(oa[4 * e], oa[4 * e + 1], oa[4 * e + 2],
+                                 oa[4 * e + 3]);
+              db[e] = make_uint4(ob[4 * e], ob[4 * e + 1], ob[4 * e + 2],
+                                 ob[4 * e + 3]);
+            }
+          }
+        }
+      } else {
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t v[32];
@@ -387,6 +426,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           for (int e = 0; e < 4; ++e)
             dst[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
         }
+      }
       }
       }
       tc_fence_before();
@@ -673,6 +713,7 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t st) {
   p.Nk = a.Nk;
   p.H = a.H;
   p.q_off = a.q_off;
+  p.rope_half = a.rope_half ? 1 : 0;
   p.Tk = (a.Nk + kBlock - 1) / kBlock;
   // one head per scheduling round: the fp32 dQ accumulator, Q~ and dO of
   // a head (16 + 8 + 8 MB at 32K) then stay L2-resident while ~148 key

@@ -29,7 +29,7 @@ decode_split_kernel(const __nv_bfloat16* __restrict__ q,
                     const int32_t* __restrict__ kv_len,
                     const int32_t* __restrict__ q_pos,
                     const float2* __restrict__ table, int max_pos, int L,
-                    int H, int splits, float scale_log2,
+                    int H, int splits, bool half, float scale_log2,
                     float* __restrict__ part_m, float* __restrict__ part_l,
                     float* __restrict__ part_acc) {
   __shared__ float qs[kHeadDim];
@@ -44,15 +44,16 @@ decode_split_kernel(const __nv_bfloat16* __restrict__ q,
   const int c0 = start + split * chunk;
   const int c1 = min(c0 + chunk, len);
   const int64_t slot = (int64_t(b) * H + h) * splits + split;
-  // rotated query, fp32, in shared memory (R(pos) on interleaved pairs)
+  // rotated query, fp32, in shared memory, in the layout of the keys: pair
+  // t is dims (2t, 2t+1), or (t, t+64) in the rotate-half layout
   if (t < kHeadDim / 2) {
-    const __nv_bfloat162 x2 = reinterpret_cast<const __nv_bfloat162*>(
-        q + (int64_t(b) * H + h) * kHeadDim)[t];
+    const __nv_bfloat16* qr = q + (int64_t(b) * H + h) * kHeadDim;
+    const int i0 = half ? t : 2 * t, i1 = half ? t + kHeadDim / 2 : 2 * t + 1;
     const int pq = max(0, min(q_pos[b], max_pos - 1));
     const float2 cs = table[int64_t(pq) * (kHeadDim / 2) + t];
-    const float a = __low2float(x2), c = __high2float(x2);
-    qs[2 * t] = (a * cs.x - c * cs.y) * scale_log2;
-    qs[2 * t + 1] = (a * cs.y + c * cs.x) * scale_log2;
+    const float a = __bfloat162float(qr[i0]), c = __bfloat162float(qr[i1]);
+    qs[i0] = (a * cs.x - c * cs.y) * scale_log2;
+    qs[i1] = (a * cs.y + c * cs.x) * scale_log2;
   }
   __syncthreads();
   float m = -INFINITY, l = 0.f, acc = 0.f;
@@ -145,8 +146,8 @@ int decode_splits(int L) {
 cudaError_t launch_decode(const void* q, const void* k_rot, const void* v,
                           const int32_t* kv_start, const int32_t* kv_len,
                           const int32_t* q_pos, const float* table,
-                          int max_pos, int B, int L, int H, void* out,
-                          float* lse, float* part_m, float* part_l,
+                          int max_pos, int B, int L, int H, bool half,
+                          void* out, float* lse, float* part_m, float* part_l,
                           float* part_acc, cudaStream_t st) {
   if (B == 0 || H == 0) return cudaSuccess;
   const int splits = decode_splits(L);
@@ -155,7 +156,7 @@ cudaError_t launch_decode(const void* q, const void* k_rot, const void* v,
       static_cast<const __nv_bfloat16*>(q),
       static_cast<const __nv_bfloat16*>(k_rot),
       static_cast<const __nv_bfloat16*>(v), kv_start, kv_len, q_pos,
-      reinterpret_cast<const float2*>(table), max_pos, L, H, splits,
+      reinterpret_cast<const float2*>(table), max_pos, L, H, splits, half,
       kLog2e / sqrtf(float(kHeadDim)), part_m, part_l, part_acc);
   note_launch();
   cudaError_t e = cudaGetLastError();

@@ -78,6 +78,7 @@ struct FwdParams {
   float* lse;
   int* status;
   int B, Nq, Nk, H, Tq, U, G, k_off;
+  int rope_half;  // Q in the rotate-half layout
   int total_items;
   float scale_log2;
 };
@@ -180,6 +181,73 @@ __device__ __forceinline__ void rope_row(uint8_t* tile, uint8_t* lo_dst,
       if (X3)
         *reinterpret_cast<uint4*>(lo_dst + off) =
             make_uint4(lo_out[0], lo_out[1], lo_out[2], lo_out[3]);
+    }
+  }
+}
+
+// The same for the rotate-half layout: pair k is (dim k, dim k + 64), so
+// the 16-byte slot lc of d chunk 0 pairs with slot lc of d chunk 1 (same
+// swizzled offset, 16 KB apart); slot lc holds pairs 8 lc .. 8 lc + 7. The
+// rotated values stay in that layout (the keys were rotated in it too).
+template <bool X3>
+__device__ __forceinline__ void rope_row_half(uint8_t* tile, uint8_t* lo_dst,
+                                              const float4* __restrict__ trow,
+                                              float4 (&cs)[8], int r,
+                                              bool valid) {
+  if (!valid) {
+    if (X3) {
+#pragma unroll
+      for (int c = 0; c < 16; ++c)
+        *reinterpret_cast<uint4*>(lo_dst + (c >> 3) * kHalfTileBytes +
+                                  r * 128 + (((c & 7) ^ (r & 7)) << 4)) =
+            make_uint4(0, 0, 0, 0);
+    }
+    return;
+  }
+#pragma unroll
+  for (int qt = 0; qt < 4; ++qt) {  // cs: pairs 16 qt .. 16 qt + 15
+    if (qt > 0) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) cs[e] = __ldg(trow + qt * 8 + e);
+    }
+#pragma unroll
+    for (int cl = 0; cl < 2; ++cl) {
+      const int lc = 2 * qt + cl;
+      const int off0 = r * 128 + ((lc ^ (r & 7)) << 4);
+      const int off1 = off0 + kHalfTileBytes;
+      const uint4 w0 = *reinterpret_cast<uint4*>(tile + off0);
+      const uint4 w1 = *reinterpret_cast<uint4*>(tile + off1);
+      const uint32_t a[4] = {w0.x, w0.y, w0.z, w0.w};
+      const uint32_t b[4] = {w1.x, w1.y, w1.z, w1.w};
+      uint32_t ha[4], hb[4], la[4], lb[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float4 t = cs[4 * cl + e];  // pairs 8 lc + 2e, 8 lc + 2e + 1
+        const float a0 = bf16lo_to_f32(a[e]), a1 = bf16hi_to_f32(a[e]);
+        const float b0 = bf16lo_to_f32(b[e]), b1 = bf16hi_to_f32(b[e]);
+        const float ra0 = fmaf(a0, t.x, -b0 * t.y);
+        const float rb0 = fmaf(a0, t.y, b0 * t.x);
+        const float ra1 = fmaf(a1, t.z, -b1 * t.w);
+        const float rb1 = fmaf(a1, t.w, b1 * t.z);
+        ha[e] = pack_bf16x2(ra0, ra1);
+        hb[e] = pack_bf16x2(rb0, rb1);
+        if (X3) {
+          la[e] = pack_bf16x2(ra0 - bf16lo_to_f32(ha[e]),
+                              ra1 - bf16hi_to_f32(ha[e]));
+          lb[e] = pack_bf16x2(rb0 - bf16lo_to_f32(hb[e]),
+                              rb1 - bf16hi_to_f32(hb[e]));
+        }
+      }
+      *reinterpret_cast<uint4*>(tile + off0) =
+          make_uint4(ha[0], ha[1], ha[2], ha[3]);
+      *reinterpret_cast<uint4*>(tile + off1) =
+          make_uint4(hb[0], hb[1], hb[2], hb[3]);
+      if (X3) {
+        *reinterpret_cast<uint4*>(lo_dst + off0) =
+            make_uint4(la[0], la[1], la[2], la[3]);
+        *reinterpret_cast<uint4*>(lo_dst + off1) =
+            make_uint4(lb[0], lb[1], lb[2], lb[3]);
+      }
     }
   }
 }
@@ -468,8 +536,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         qcount[s]++;
-        rope_row<X3>(smem + C::kQ + s * kTileBytes,
-                     smem + C::kQlo + s * kTileBytes, trow, cs0, r, valid);
+        if (p.rope_half)
+          rope_row_half<X3>(smem + C::kQ + s * kTileBytes,
+                            smem + C::kQlo + s * kTileBytes, trow, cs0, r,
+                            valid);
+        else
+          rope_row<X3>(smem + C::kQ + s * kTileBytes,
+                       smem + C::kQlo + s * kTileBytes, trow, cs0, r, valid);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(C::bQReady + s));
@@ -798,6 +871,7 @@ static cudaError_t launch_fwd_impl(const FwdArgs& a, cudaStream_t st) {
   p.Nk = a.Nk;
   p.H = a.H;
   p.k_off = a.k_off;
+  p.rope_half = a.rope_half ? 1 : 0;
   p.Tq = (a.Nq + kBlock - 1) / kBlock;
   p.U = (p.Tq + kFwdBlocksPerUnit - 1) / kFwdBlocksPerUnit;
   // heads interleaved per scheduling round: 2 keeps the K/V of the heads

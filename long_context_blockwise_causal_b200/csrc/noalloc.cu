@@ -61,8 +61,8 @@ int lwm_blockattn_fwd_noalloc(const void* q, const void* k, const void* v,
                               const int32_t* positions, double theta,
                               int block_q, int block_k, int max_pos, int B,
                               int N, int H, int D, int dtype,
-                              int qk_precision, void* out, float* lse,
-                              void* stream) {
+                              int qk_precision, int rope_layout, void* out,
+                              float* lse, void* stream) {
   const size_t need = lwm_blockattn_fwd_workspace_size(
       B, N, H, D, block_q, block_k, max_pos, dtype, qk_precision);
   if (need == 0) return LWM_ERR_INVALID_ARG;
@@ -71,8 +71,8 @@ int lwm_blockattn_fwd_noalloc(const void* q, const void* k, const void* v,
   if (!scratch) return LWM_ERR_CUDA;
   return lwm_blockattn_fwd(q, k, v, segment_ids, positions, theta, block_q,
                            block_k, max_pos, B, N, H, D, dtype, qk_precision,
-                           out, lse, scratch, lwm::kNoAllocScratchBytes,
-                           stream);
+                           rope_layout, out, lse, scratch,
+                           lwm::kNoAllocScratchBytes, stream);
 }
 
 }  // extern "C"

@@ -6,10 +6,11 @@
 // mask every pair ("LWM：突破 100 万 Token 的开源大模型", 概述 (b)), and RoPE
 // rotates q and k as they are loaded.
 //
-// Thread layout: 4 threads per row; thread `part` owns the 16 interleaved
-// pairs k = 4*i + part (dims 2k, 2k+1), so a RoPE pair never straddles
-// threads and the 4 threads of a row read 4 consecutive float2 of a
-// shared-memory row (conflict free).
+// Thread layout: 4 threads per row; thread `part` owns the 16 RoPE pairs
+// k = 4*i + part (dims 2k, 2k+1; for q and k in the rotate-half layout the
+// pair is dims k, k+64), so a pair never straddles threads and the 4
+// threads of a row read 4 consecutive float2 of a shared-memory row
+// (conflict free). Values, outputs and their gradients keep (2k, 2k+1).
 #include "aux_kernels.cuh"
 
 namespace lwm {
@@ -44,6 +45,24 @@ __device__ __forceinline__ void st_pair<__nv_bfloat16>(__nv_bfloat16* p,
   *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
 }
 
+// RoPE pair k of a head row: (2k, 2k+1), or (k, k+64) in the rotate-half
+// layout.
+template <typename T>
+__device__ __forceinline__ float2 ld_rpair(const T* row, int k, bool half) {
+  if (!half) return ld_pair(row + 2 * k);
+  return make_float2(float(row[k]), float(row[k + kHeadDim / 2]));
+}
+template <typename T>
+__device__ __forceinline__ void st_rpair(T* row, int k, bool half, float a,
+                                         float b) {
+  if (!half) {
+    st_pair(row + 2 * k, a, b);
+  } else {
+    row[k] = T(a);
+    row[k + kHeadDim / 2] = T(b);
+  }
+}
+
 __device__ __forceinline__ float2 rot(float2 x, float2 cs, float sign) {
   float s = sign * cs.y;
   return make_float2(x.x * cs.x - x.y * s, x.x * s + x.y * cs.x);
@@ -62,7 +81,7 @@ fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
                 const int32_t* __restrict__ pos,
                 const float2* __restrict__ table,
                 const int32_t* __restrict__ kv_lo, int N, int H,
-                float scale_log2, T* __restrict__ out,
+                bool half, float scale_log2, T* __restrict__ out,
                 float* __restrict__ lse) {
   __shared__ float2 Ks[kKeys][kPairs];
   __shared__ float2 Vs[kKeys][kPairs];
@@ -83,7 +102,7 @@ fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
       int kk = 4 * e + part;
-      float2 x = valid ? ld_pair(qp + 2 * kk) : make_float2(0.f, 0.f);
+      float2 x = valid ? ld_rpair(qp, kk, half) : make_float2(0.f, 0.f);
       qv[e] = rot(x, table[int64_t(p) * kPairs + kk], 1.f);
       acc[e] = make_float2(0.f, 0.f);
     }
@@ -100,10 +119,10 @@ fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
       int key = e / kPairs, kk = e % kPairs, j = k0 + key;
       float2 kx = make_float2(0.f, 0.f), vx = kx;
       if (j < N) {
-        int64_t off = ((rowbase + j) * H + h) * kHeadDim + 2 * kk;
-        kx = rot(ld_pair(k + off), table[int64_t(pos[rowbase + j]) * kPairs + kk],
-                 1.f);
-        vx = ld_pair(v + off);
+        int64_t off = ((rowbase + j) * H + h) * kHeadDim;
+        kx = rot(ld_rpair(k + off, kk, half),
+                 table[int64_t(pos[rowbase + j]) * kPairs + kk], 1.f);
+        vx = ld_pair(v + off + 2 * kk);
       }
       Ks[key][kk] = kx;
       Vs[key][kk] = vx;
@@ -167,7 +186,7 @@ bwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
                 const float* __restrict__ lse, const float* __restrict__ delta,
                 const int32_t* __restrict__ seg,
                 const int32_t* __restrict__ pos,
-                const float2* __restrict__ table, int N, int H,
+                const float2* __restrict__ table, int N, int H, bool half,
                 float scale_log2, float scale, float* __restrict__ dq_acc,
                 T* __restrict__ dk, T* __restrict__ dv) {
   extern __shared__ float4 smem_f4[];
@@ -194,7 +213,7 @@ bwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
       int kk = 4 * e + part;
-      float2 x = valid ? ld_pair(k + off + 2 * kk) : make_float2(0.f, 0.f);
+      float2 x = valid ? ld_rpair(k + off, kk, half) : make_float2(0.f, 0.f);
       kv[e] = rot(x, table[int64_t(p) * kPairs + kk], 1.f);
       Ks[key][kk] = kv[e];
       vv[e] = valid ? ld_pair(v + off + 2 * kk) : make_float2(0.f, 0.f);
@@ -213,10 +232,10 @@ bwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
       int r = e / kPairs, kk = e % kPairs, i = i0 + r;
       float2 qx = make_float2(0.f, 0.f), gx = qx;
       if (i < N) {
-        int64_t off = ((rowbase + i) * H + h) * kHeadDim + 2 * kk;
-        qx = rot(ld_pair(q + off), table[int64_t(pos[rowbase + i]) * kPairs + kk],
-                 1.f);
-        gx = ld_pair(dout + off);
+        int64_t off = ((rowbase + i) * H + h) * kHeadDim;
+        qx = rot(ld_rpair(q + off, kk, half),
+                 table[int64_t(pos[rowbase + i]) * kPairs + kk], 1.f);
+        gx = ld_pair(dout + off + 2 * kk);
       }
       Qs[r][kk] = qx;
       Gs[r][kk] = gx;
@@ -273,12 +292,15 @@ bwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
             a[e].y = fmaf(w, kx.y, a[e].y);
           }
         }
-        float* dst = dq_acc + ((rowbase + i) * H + h) * kHeadDim + 2 * c;
+        // dq~ pairs in the layout q came in (converted by dq_convert)
+        float* dst = dq_acc + ((rowbase + i) * H + h) * kHeadDim;
+        const int second = half ? kHeadDim / 2 : 1;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           if (a[e].x != 0.f || a[e].y != 0.f) {
-            atomicAdd(dst + 2 * e, a[e].x);
-            atomicAdd(dst + 2 * e + 1, a[e].y);
+            const int first = half ? c + e : 2 * (c + e);
+            atomicAdd(dst + first, a[e].x);
+            atomicAdd(dst + first + second, a[e].y);
           }
         }
       }
@@ -292,7 +314,7 @@ bwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
     int kk = 4 * e + part;
     float2 g = make_float2(gk[e].x * scale, gk[e].y * scale);
     float2 r = rot(g, table[int64_t(p) * kPairs + kk], -1.f);
-    st_pair(dk + off + 2 * kk, r.x, r.y);
+    st_rpair(dk + off, kk, half, r.x, r.y);
     st_pair(dv + off + 2 * kk, gv[e].x, gv[e].y);
   }
 }
@@ -309,13 +331,14 @@ template <typename T>
 cudaError_t launch_fwd_simt(const T* q, const T* k, const T* v,
                             const int32_t* seg, const int32_t* pos,
                             const float* table, const int32_t* kv_lo, int B,
-                            int N, int H, T* out, float* lse, cudaStream_t st) {
+                            int N, int H, bool half, T* out, float* lse,
+                            cudaStream_t st) {
   if (B == 0 || N == 0 || H == 0) return cudaSuccess;
   dim3 grid((N + kRows - 1) / kRows, H, B);
   float scale_log2 = kLog2e / sqrtf(float(kHeadDim));
   fwd_simt_kernel<T><<<grid, kThreads, 0, st>>>(
       q, k, v, seg, pos, reinterpret_cast<const float2*>(table), kv_lo, N, H,
-      scale_log2, out, lse);
+      half, scale_log2, out, lse);
   note_launch();
   return cudaGetLastError();
 }
@@ -325,7 +348,8 @@ cudaError_t launch_bwd_simt(const T* q, const T* k, const T* v, const T* dout,
                             const float* lse, const float* delta,
                             const int32_t* seg, const int32_t* pos,
                             const float* table, int B, int N, int H,
-                            float* dq_acc, T* dk, T* dv, cudaStream_t st) {
+                            bool half, float* dq_acc, T* dk, T* dv,
+                            cudaStream_t st) {
   if (B == 0 || N == 0 || H == 0) return cudaSuccess;
   size_t smem = bwd_smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(
@@ -336,8 +360,8 @@ cudaError_t launch_bwd_simt(const T* q, const T* k, const T* v, const T* dout,
   float scale = 1.f / sqrtf(float(kHeadDim));
   bwd_simt_kernel<T><<<grid, kThreads, smem, st>>>(
       q, k, v, dout, lse, delta, seg, pos,
-      reinterpret_cast<const float2*>(table), N, H, kLog2e * scale, scale,
-      dq_acc, dk, dv);
+      reinterpret_cast<const float2*>(table), N, H, half, kLog2e * scale,
+      scale, dq_acc, dk, dv);
   note_launch();
   return cudaGetLastError();
 }
@@ -346,22 +370,23 @@ template cudaError_t launch_fwd_simt<float>(const float*, const float*,
                                             const float*, const int32_t*,
                                             const int32_t*, const float*,
                                             const int32_t*, int, int, int,
-                                            float*, float*, cudaStream_t);
+                                            bool, float*, float*,
+                                            cudaStream_t);
 template cudaError_t launch_fwd_simt<__nv_bfloat16>(
     const __nv_bfloat16*, const __nv_bfloat16*, const __nv_bfloat16*,
     const int32_t*, const int32_t*, const float*, const int32_t*, int, int,
-    int, __nv_bfloat16*, float*, cudaStream_t);
+    int, bool, __nv_bfloat16*, float*, cudaStream_t);
 template cudaError_t launch_bwd_simt<float>(const float*, const float*,
                                             const float*, const float*,
                                             const float*, const float*,
                                             const int32_t*, const int32_t*,
                                             const float*, int, int, int,
-                                            float*, float*, float*,
+                                            bool, float*, float*, float*,
                                             cudaStream_t);
 template cudaError_t launch_bwd_simt<__nv_bfloat16>(
     const __nv_bfloat16*, const __nv_bfloat16*, const __nv_bfloat16*,
     const __nv_bfloat16*, const float*, const float*, const int32_t*,
-    const int32_t*, const float*, int, int, int, float*, __nv_bfloat16*,
-    __nv_bfloat16*, cudaStream_t);
+    const int32_t*, const float*, int, int, int, bool, float*,
+    __nv_bfloat16*, __nv_bfloat16*, cudaStream_t);
 
 }  // namespace lwm

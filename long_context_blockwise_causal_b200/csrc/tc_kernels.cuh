@@ -36,6 +36,7 @@ struct FwdArgs {
   int32_t* counter;        // zeroed work counter (units handed out in order)
   int B, Nq, Nk, H, k_off;
   bool qk_x3;
+  bool rope_half;          // q (and k_rot) in the rotate-half layout
   int* status;
 };
 
@@ -71,6 +72,7 @@ struct BwdArgs {
   float* dk_acc;           // [B][Nk][H][D] fp32 accumulators
   float* dv_acc;
   int B, Nq, Nk, H, q_off;
+  bool rope_half;          // rotate-half layout (dk's R(-pos) pairs)
   int* status;
 };
 

@@ -22,6 +22,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, \
     ERR_TIMEOUT, ERR_PRECONDITION = range(7)
 DTYPE_BF16, DTYPE_FP32 = 0, 1
 QK_BF16, QK_BF16X3 = 0, 1
+ROPE_INTERLEAVED, ROPE_HALF = 0, 1
 TILE_EMPTY, TILE_PARTIAL, TILE_FULL = 0, 1, 2
 BLOCK = 128
 HEAD_DIM = 128
@@ -35,11 +36,11 @@ _SIGS = {
     "lwm_blockattn_fwd_workspace_size": (_sz, [_i] * 9),
     "lwm_blockattn_bwd_workspace_size": (_sz, [_i] * 9),
     "lwm_blockattn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _d, _i, _i, _i,
-                               _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _sz,
-                               _vp]),
+                               _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp,
+                               _sz, _vp]),
     "lwm_blockattn_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _d,
-                               _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp,
-                               _vp, _vp, _sz, _vp]),
+                               _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
+                               _vp, _vp, _vp, _sz, _vp]),
     "lwm_blockattn_classify": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp,
                                     _vp]),
     "lwm_blockattn_rope_table": (_i, [_d, _i, _i, _vp, _vp]),
@@ -51,17 +52,18 @@ _SIGS = {
     "lwm_blockattn_kernel_launches": (ctypes.c_uint64, []),
     "lwm_blockattn_selftest_wait_timeout": (_i, [ctypes.c_uint64, _vp]),
     "lwm_blockattn_rope_apply": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
-                                      _vp, _vp]),
+                                      _i, _vp, _vp]),
     "lwm_blockattn_decode_workspace_size": (_sz, [_i, _i, _i, _i]),
     "lwm_blockattn_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i,
-                                  _i, _i, _i, _i, _vp, _vp, _vp, _sz, _vp]),
+                                  _i, _i, _i, _i, _i, _vp, _vp, _vp, _sz,
+                                  _vp]),
     "lwm_blockattn_fwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _d, _i, _i,
-                                       _i, _i, _i, _i, _i, _i, _i, _vp, _vp,
-                                       _vp]),
+                                       _i, _i, _i, _i, _i, _i, _i, _i, _vp,
+                                       _vp, _vp]),
     "lwm_blockattn_fwd_block_workspace_size": (_sz, [_i] * 6),
     "lwm_blockattn_fwd_block": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i,
-                                     _d, _i, _i, _i, _i, _i, _i, _vp, _vp,
-                                     _vp, _sz, _vp]),
+                                     _d, _i, _i, _i, _i, _i, _i, _i, _vp,
+                                     _vp, _vp, _sz, _vp]),
     "lwm_blockattn_merge": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                  _vp]),
     "lwm_blockattn_bwd_delta": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp,
@@ -71,7 +73,7 @@ _SIGS = {
                                      _i, _i, _i, _i, _i, _i, _i, _vp, _vp,
                                      _vp, _vp, _sz, _vp]),
     "lwm_blockattn_grad_finish": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
-                                       _vp, _vp]),
+                                       _i, _vp, _vp]),
 }
 
 
@@ -141,6 +143,14 @@ def _qk_code(qk_precision) -> int:
     raise ValueError(f"qk_precision {qk_precision!r}")
 
 
+def _layout_code(rope_layout) -> int:
+    if rope_layout in (ROPE_INTERLEAVED, "interleaved"):
+        return ROPE_INTERLEAVED
+    if rope_layout in (ROPE_HALF, "half", "rotate_half"):
+        return ROPE_HALF
+    raise ValueError(f"rope_layout {rope_layout!r}")
+
+
 def _need_cuda(*ts):
     for t in ts:
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
@@ -173,8 +183,10 @@ def _workspace(nbytes, device, workspace):
 
 def fwd(q, k, v, segment_ids, positions, theta, max_pos=None,
         qk_precision="bf16", out=None, lse=None, workspace=None,
-        stream=None, block_q=BLOCK, block_k=BLOCK):
-    """Forward pass. Returns (out [B,N,H,D] in q's dtype, lse [B,H,N] fp32)."""
+        stream=None, block_q=BLOCK, block_k=BLOCK, rope_layout="interleaved"):
+    """Forward pass. Returns (out [B,N,H,D] in q's dtype, lse [B,H,N] fp32).
+    ``rope_layout``: "interleaved" pairs (2k, 2k+1) or "half" (k, k+D/2),
+    the rotate-half layout of Hugging Face Llama checkpoints."""
     _need_cuda(q, k, v, segment_ids, positions, out, lse, workspace)
     B, N, H, D = q.shape
     if max_pos is None:
@@ -189,15 +201,15 @@ def fwd(q, k, v, segment_ids, positions, theta, max_pos=None,
     st = lib().lwm_blockattn_fwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(segment_ids), _ptr(positions),
         float(theta), block_q, block_k, int(max_pos), B, N, H, D,
-        _dtype_code(q), _qk_code(qk_precision), _ptr(out), _ptr(lse),
-        _ptr(ws), ws.numel(), _stream(stream))
+        _dtype_code(q), _qk_code(qk_precision), _layout_code(rope_layout),
+        _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream))
     _check(st, "lwm_blockattn_fwd")
     return out, lse
 
 
 def fwd_noalloc(q, k, v, segment_ids, positions, theta, max_pos,
                 qk_precision="bf16", out=None, lse=None, stream=None,
-                block_q=BLOCK, block_k=BLOCK):
+                block_q=BLOCK, block_k=BLOCK, rope_layout="interleaved"):
     """Forward through lwm_blockattn_fwd_noalloc: the library's own fixed
     scratch array replaces the workspace (see the header for its limits).
     ``out``/``lse`` are allocated here only if the caller passes none."""
@@ -210,16 +222,18 @@ def fwd_noalloc(q, k, v, segment_ids, positions, theta, max_pos,
     st = lib().lwm_blockattn_fwd_noalloc(
         _ptr(q), _ptr(k), _ptr(v), _ptr(segment_ids), _ptr(positions),
         float(theta), block_q, block_k, int(max_pos), B, N, H, D,
-        _dtype_code(q), _qk_code(qk_precision), _ptr(out), _ptr(lse),
-        _stream(stream))
+        _dtype_code(q), _qk_code(qk_precision), _layout_code(rope_layout),
+        _ptr(out), _ptr(lse), _stream(stream))
     _check(st, "lwm_blockattn_fwd_noalloc")
     return out, lse
 
 
 def bwd(q, k, v, out, dout, lse, segment_ids, positions, theta,
         max_pos=None, qk_precision="bf16", dq=None, dk=None, dv=None,
-        workspace=None, stream=None, block_q=BLOCK, block_k=BLOCK):
-    """Backward pass. Returns (dq, dk, dv) in q's dtype."""
+        workspace=None, stream=None, block_q=BLOCK, block_k=BLOCK,
+        rope_layout="interleaved"):
+    """Backward pass. Returns (dq, dk, dv) in q's dtype (dq, dk in the
+    layout q and k came in)."""
     _need_cuda(q, k, v, out, dout, lse, segment_ids, positions, dq, dk, dv,
                workspace)
     B, N, H, D = q.shape
@@ -235,7 +249,8 @@ def bwd(q, k, v, out, dout, lse, segment_ids, positions, theta,
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
         _ptr(segment_ids), _ptr(positions), float(theta), block_q, block_k,
         int(max_pos), B, N, H, D, _dtype_code(q), _qk_code(qk_precision),
-        _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(), _stream(stream))
+        _layout_code(rope_layout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
+        ws.numel(), _stream(stream))
     _check(st, "lwm_blockattn_bwd")
     return dq, dk, dv
 
@@ -246,7 +261,8 @@ def fwd_block_workspace_size(B, Nq, Nk, H, max_pos, D=HEAD_DIM) -> int:
 
 
 def fwd_block(q, k_rot, v, seg_q, pos_q, seg_k, q_off, k_off, theta,
-              max_pos, out=None, lse=None, workspace=None, stream=None):
+              max_pos, out=None, lse=None, workspace=None, stream=None,
+              rope_layout="interleaved"):
     """Partial forward of query rows [q_off, q_off+Nq) against the rotated
     key / value rows [k_off, k_off+Nk) of the same packed sequence (one step
     of a ring). Returns (out [B,Nq,H,D] bf16, lse [B,H,Nq] fp32); rows that
@@ -263,7 +279,8 @@ def fwd_block(q, k_rot, v, seg_q, pos_q, seg_k, q_off, k_off, theta,
     st = lib().lwm_blockattn_fwd_block(
         _ptr(q), _ptr(k_rot), _ptr(v), _ptr(seg_q), _ptr(pos_q), _ptr(seg_k),
         int(q_off), int(k_off), float(theta), int(max_pos), B, Nq, Nk, H, D,
-        _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream))
+        _layout_code(rope_layout), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+        _stream(stream))
     _check(st, "lwm_blockattn_fwd_block")
     return out, lse
 
@@ -317,7 +334,8 @@ def bwd_block(q_rot, k_rot, v, dout, lse, delta, seg_q, seg_k, q_off, k_off,
     return dq_acc, dk_acc, dv_acc
 
 
-def grad_finish(acc, positions=None, table=None, out=None, stream=None):
+def grad_finish(acc, positions=None, table=None, out=None, stream=None,
+                rope_layout="interleaved"):
     """bf16 gradient from an fp32 accumulator: R(-pos) acc / sqrt(D) when
     positions are given (dq, dk), else acc (dv)."""
     _need_cuda(acc, positions, table, out)
@@ -327,7 +345,7 @@ def grad_finish(acc, positions=None, table=None, out=None, stream=None):
     st = lib().lwm_blockattn_grad_finish(
         _ptr(acc), _ptr(positions), _ptr(table),
         0 if table is None else table.shape[0], B, N, H, D, DTYPE_BF16,
-        _ptr(out), _stream(stream))
+        _layout_code(rope_layout), _ptr(out), _stream(stream))
     _check(st, "lwm_blockattn_grad_finish")
     return out
 
@@ -360,14 +378,16 @@ def rope_table(theta, max_pos, D=HEAD_DIM, device="cuda", stream=None):
     return t
 
 
-def rope_apply(x, positions, table, stream=None, out=None):
-    """R(pos) x (bf16 [B,N,H,D]) with a table from rope_table()."""
+def rope_apply(x, positions, table, stream=None, out=None,
+               rope_layout="interleaved"):
+    """R(pos) x (bf16 [B,N,H,D]) with a table from rope_table(), pairs as
+    ``rope_layout`` says (the output keeps that layout)."""
     _need_cuda(x, positions, table, out)
     B, N, H, D = x.shape
     out = torch.empty_like(x) if out is None else out
     st = lib().lwm_blockattn_rope_apply(
         _ptr(x), _ptr(positions), _ptr(table), table.shape[0], B, N, H, D,
-        _dtype_code(x), _ptr(out), _stream(stream))
+        _dtype_code(x), _layout_code(rope_layout), _ptr(out), _stream(stream))
     _check(st, "lwm_blockattn_rope_apply")
     return out
 
@@ -377,7 +397,7 @@ def decode_workspace_size(B, H, L, D=HEAD_DIM) -> int:
 
 
 def decode(q, k_rot, v, kv_start, kv_len, q_pos, table, out=None, lse=None,
-           workspace=None, stream=None):
+           workspace=None, stream=None, rope_layout="interleaved"):
     """One query token per (b, h) [B,H,D] against a cache of rotated keys
     and values [B,L,H,D]; returns (out [B,H,D], lse [B,H])."""
     _need_cuda(q, k_rot, v, kv_start, kv_len, q_pos, table, out, lse,
@@ -391,7 +411,8 @@ def decode(q, k_rot, v, kv_start, kv_len, q_pos, table, out=None, lse=None,
     st = lib().lwm_blockattn_decode(
         _ptr(q), _ptr(k_rot), _ptr(v), _ptr(kv_start), _ptr(kv_len),
         _ptr(q_pos), _ptr(table), table.shape[0], B, L, H, D, _dtype_code(q),
-        _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream))
+        _layout_code(rope_layout), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+        _stream(stream))
     _check(st, "lwm_blockattn_decode")
     return out, lse
 

@@ -56,18 +56,22 @@ def causally_visible(q_off: int, nq: int, k_off: int, nk: int) -> bool:
 class CudaBackend:
     """The ring's calls on this library's kernels (bf16, D = 128)."""
 
-    def __init__(self, theta: float, max_pos: int, device=None):
+    def __init__(self, theta: float, max_pos: int, device=None,
+                 rope_layout="interleaved"):
         self.theta = float(theta)
         self.max_pos = int(max_pos)
+        self.layout = rope_layout
         self.table = ops.rope_table(self.theta, self.max_pos,
                                     device=device or "cuda")
 
     def rotate(self, k, positions):
-        return ops.rope_apply(k, positions, self.table)
+        return ops.rope_apply(k, positions, self.table,
+                              rope_layout=self.layout)
 
     def partial(self, q, k_rot, v, seg_q, pos_q, seg_k, q_off, k_off):
         return ops.fwd_block(q, k_rot, v, seg_q, pos_q, seg_k, q_off, k_off,
-                             self.theta, self.max_pos)
+                             self.theta, self.max_pos,
+                             rope_layout=self.layout)
 
     def merge(self, out, lse, out_part, lse_part):
         return ops.merge(out, lse, out_part, lse_part)
@@ -92,7 +96,8 @@ class CudaBackend:
                       k_off, dq_acc, dk_acc, dv_acc)
 
     def finish(self, acc, positions):
-        return ops.grad_finish(acc, positions, self.table)
+        return ops.grad_finish(acc, positions, self.table,
+                               rope_layout=self.layout)
 
     def finish_v(self, acc):
         return ops.grad_finish(acc)

@@ -30,7 +30,8 @@ RoPE pairs, theta^(-2k/D) frequencies in fp64, causal mask on token index,
 natural-log logsumexp) are listed in the module docstrings that use them.
 
 Modules:
-  rope       -- RoPE frequencies, angles and rotation.
+  rope       -- RoPE frequencies, angles and rotation (interleaved pairs and
+                the rotate-half layout, with the permutation between them).
   attention  -- dense fp64 forward/backward (row-blocked), sampled rows.
   blockwise  -- CPU online-softmax restatement in ring order (invariance pin).
   ring       -- partial attention over a key block, the log-sum-exp merge and
@@ -38,7 +39,10 @@ Modules:
   classify   -- tile classification (brute force and a counting form).
 """
 
-from .rope import rope_inv_freq, rope_angles, rope_rotate  # noqa: F401
+from .rope import (  # noqa: F401
+    rope_inv_freq, rope_angles, rope_rotate, rope_rotate_half,
+    half_to_interleaved, interleaved_to_half,
+)
 from .attention import (  # noqa: F401
     allowed_mask, attn_fwd, attn_fwd_rows, attn_bwd, attn_bwd_rows,
     attn_bwd_cols, SOFTMAX_SCALE_RULE,

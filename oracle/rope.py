@@ -54,3 +54,38 @@ def rope_rotate(x, positions, theta: float, sign: int = 1) -> np.ndarray:
     out[..., 0::2] = a * c - b * s
     out[..., 1::2] = a * s + b * c
     return out
+
+
+def rope_rotate_half(x, positions, theta: float, sign: int = 1) -> np.ndarray:
+    """RoPE in the rotate-half layout: pair k is (x[k], x[k + D/2]) with the
+    same frequency theta ** (-2k / D); this is how Hugging Face Llama
+    checkpoints (the PyTorch form of the models, "LWM：突破 100 万 Token 的开
+    源大模型", 脚本运行说明) lay out q and k."""
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    ang = float(sign) * rope_angles(positions, theta, d)
+    c = np.cos(ang)
+    s = np.sin(ang)
+    a = x[..., : d // 2]
+    b = x[..., d // 2:]
+    out = np.empty_like(x)
+    out[..., : d // 2] = a * c - b * s
+    out[..., d // 2:] = a * s + b * c
+    return out
+
+
+def half_to_interleaved(x) -> np.ndarray:
+    """Permute the last axis from the rotate-half layout to the interleaved
+    one: out[2k] = x[k], out[2k+1] = x[k + D/2]."""
+    x = np.asarray(x)
+    d = x.shape[-1]
+    out = np.empty_like(x)
+    out[..., 0::2] = x[..., : d // 2]
+    out[..., 1::2] = x[..., d // 2:]
+    return out
+
+
+def interleaved_to_half(x) -> np.ndarray:
+    """Inverse of half_to_interleaved."""
+    x = np.asarray(x)
+    return np.concatenate([x[..., 0::2], x[..., 1::2]], axis=-1)

@@ -64,7 +64,7 @@ def test_workspace_sizes_grow_with_inputs():
 def _fwd_raw(**kw):
     args = dict(q=1 << 20, k=1 << 20, v=1 << 20, seg=1 << 20, pos=1 << 20,
                 theta=1e4, bq=128, bk=128, max_pos=16, B=1, N=16, H=1, D=128,
-                dtype=0, qkp=0, out=1 << 20, lse=1 << 20, ws=1 << 20,
+                dtype=0, qkp=0, layout=0, out=1 << 20, lse=1 << 20, ws=1 << 20,
                 wsb=1 << 40, stream=None)
     args.update(kw)
     v = lambda x: None if x is None else ctypes.c_void_p(x)
@@ -72,7 +72,8 @@ def _fwd_raw(**kw):
         v(args["q"]), v(args["k"]), v(args["v"]), v(args["seg"]),
         v(args["pos"]), args["theta"], args["bq"], args["bk"],
         args["max_pos"], args["B"], args["N"], args["H"], args["D"],
-        args["dtype"], args["qkp"], v(args["out"]), v(args["lse"]),
+        args["dtype"], args["qkp"], args["layout"], v(args["out"]),
+        v(args["lse"]),
         v(args["ws"]), args["wsb"], v(args["stream"]))
 
 
@@ -85,6 +86,7 @@ def _fwd_raw(**kw):
     ({"theta": float("nan")}, ops.ERR_INVALID_ARG),
     ({"dtype": 7}, ops.ERR_INVALID_ARG),
     ({"qkp": 5}, ops.ERR_INVALID_ARG),
+    ({"layout": 2}, ops.ERR_INVALID_ARG),
     ({"N": -1}, ops.ERR_INVALID_ARG),
     ({"max_pos": 0}, ops.ERR_INVALID_ARG),
     ({"D": 64}, ops.ERR_UNSUPPORTED),
@@ -104,11 +106,14 @@ def test_bwd_and_classify_reject_bad_arguments():
     v = ctypes.c_void_p
     p = v(1 << 20)
     st = L.lwm_blockattn_bwd(p, p, p, p, p, p, p, p, 1e4, 128, 128, 16, 1, 16,
-                             1, 128, 0, 0, p, p, None, p, 1 << 40, None)
+                             1, 128, 0, 0, 0, p, p, None, p, 1 << 40, None)
     assert st == ops.ERR_INVALID_ARG  # dv is NULL
     st = L.lwm_blockattn_bwd(p, p, p, p, p, p, p, p, 1e4, 128, 128, 16, 1, 16,
-                             1, 128, 0, 0, p, p, p, p, 10, None)
+                             1, 128, 0, 0, 0, p, p, p, p, 10, None)
     assert st == ops.ERR_WORKSPACE
+    st = L.lwm_blockattn_bwd(p, p, p, p, p, p, p, p, 1e4, 128, 128, 16, 1, 16,
+                             1, 128, 0, 0, 3, p, p, p, p, 1 << 40, None)
+    assert st == ops.ERR_INVALID_ARG  # unknown RoPE layout
     assert L.lwm_blockattn_classify(p, 1, 16, 128, 48, p, p, None,
                                     None) == ops.ERR_UNSUPPORTED
     assert L.lwm_blockattn_classify(None, 1, 16, 128, 128, p, p, None,
@@ -119,3 +124,51 @@ def test_bwd_and_classify_reject_bad_arguments():
         ops.ERR_INVALID_ARG
     assert L.lwm_blockattn_rope_table(1e4, 127, 10, p, None) == \
         ops.ERR_INVALID_ARG
+
+
+def test_ring_and_layout_entry_points_reject_bad_arguments():
+    L = ops.lib()
+    v = ctypes.c_void_p
+    p = v(1 << 20)
+    big = 1 << 40
+    # fwd_block: null q, unknown layout, misaligned seg_k
+    assert L.lwm_blockattn_fwd_block(None, p, p, p, p, p, 0, 0, 1e4, 16, 1, 16,
+                                     16, 1, 128, 0, p, p, p, big,
+                                     None) == ops.ERR_INVALID_ARG
+    assert L.lwm_blockattn_fwd_block(p, p, p, p, p, p, 0, 0, 1e4, 16, 1, 16,
+                                     16, 1, 128, 9, p, p, p, big,
+                                     None) == ops.ERR_INVALID_ARG
+    assert L.lwm_blockattn_fwd_block(p, p, p, p, p, v((1 << 20) + 4), 0, 0,
+                                     1e4, 16, 1, 16, 16, 1, 128, 0, p, p, p,
+                                     big, None) == ops.ERR_INVALID_ARG
+    assert L.lwm_blockattn_fwd_block(p, p, p, p, p, p, -1, 0, 1e4, 16, 1, 16,
+                                     16, 1, 128, 0, p, p, p, big,
+                                     None) == ops.ERR_INVALID_ARG
+    # bwd_block: null accumulator; D != 128
+    assert L.lwm_blockattn_bwd_block(p, p, p, p, p, p, p, p, 0, 0, 1, 16, 16,
+                                     1, 128, p, None, p, p, big,
+                                     None) == ops.ERR_INVALID_ARG
+    assert L.lwm_blockattn_bwd_block(p, p, p, p, p, p, p, p, 0, 0, 1, 16, 16,
+                                     1, 64, p, p, p, p, big,
+                                     None) == ops.ERR_UNSUPPORTED
+    # merge / bwd_delta: fp32 I/O is not offered
+    assert L.lwm_blockattn_merge(p, p, p, p, 1, 16, 1, 128, 1,
+                                 None) == ops.ERR_UNSUPPORTED
+    assert L.lwm_blockattn_bwd_delta(p, p, 1, 16, 1, 128, 1, p,
+                                     None) == ops.ERR_UNSUPPORTED
+    # grad_finish: positions without a table
+    assert L.lwm_blockattn_grad_finish(p, p, None, 16, 1, 16, 1, 128, 0, 0,
+                                       p, None) == ops.ERR_INVALID_ARG
+    # rope_apply and decode: unknown layout
+    assert L.lwm_blockattn_rope_apply(p, p, p, 16, 1, 16, 1, 128, 0, 5, p,
+                                      None) == ops.ERR_INVALID_ARG
+    assert L.lwm_blockattn_decode(p, p, p, p, p, p, p, 16, 1, 16, 1, 128, 0,
+                                  5, p, p, p, big,
+                                  None) == ops.ERR_INVALID_ARG
+    # empty problems launch nothing and succeed
+    assert L.lwm_blockattn_fwd_block(None, None, None, None, None, None, 0, 0,
+                                     1e4, 16, 1, 0, 16, 1, 128, 0, None, None,
+                                     None, 0, None) == ops.OK
+    assert L.lwm_blockattn_bwd_block(None, None, None, None, None, None, None,
+                                     None, 0, 0, 1, 16, 0, 1, 128, None, None,
+                                     None, None, 0, None) == ops.OK

@@ -405,3 +405,50 @@ def test_sampled_backward_rows_and_cols_equal_full_backward():
                                   row_block=7)
     np.testing.assert_allclose(dk, full["dk"][0, rows, 0], atol=1e-12)
     np.testing.assert_allclose(dv, full["dv"][0, rows, 0], atol=1e-12)
+
+
+# ------------------------------------------------- rotate-half layout pins
+
+def test_rope_rotate_half_matches_transformers_llama():
+    d, n, theta = 128, 64, 1e6
+    rng = np.random.default_rng(30)
+    x = rng.standard_normal((n, d))
+    pos = rng.integers(0, 300, n)
+    # fp32 frequencies inside transformers: angle error <= 300 * 2^-24
+    np.testing.assert_allclose(orope.rope_rotate_half(x, pos, theta),
+                               _hf_rope(x, pos, theta), atol=1e-4, rtol=0)
+
+
+def test_rotate_half_is_interleaved_rope_under_the_permutation():
+    d, n, theta = 128, 50, 5e7
+    rng = np.random.default_rng(31)
+    x = rng.standard_normal((3, n, d))
+    pos = rng.integers(0, 10 ** 6, n)
+    for sign in (1, -1):
+        via = orope.interleaved_to_half(
+            orope.rope_rotate(orope.half_to_interleaved(x), pos, theta, sign))
+        np.testing.assert_allclose(orope.rope_rotate_half(x, pos, theta, sign),
+                                   via, atol=1e-12, rtol=0)
+    y = rng.standard_normal((4, d))
+    assert np.array_equal(orope.interleaved_to_half(orope.half_to_interleaved(y)), y)
+    assert np.array_equal(orope.half_to_interleaved(y)[:, 1], y[:, d // 2])
+
+
+def test_attention_in_rotate_half_layout_equals_permuted_interleaved():
+    # scores only see dot products of q and k rotated in one layout, so
+    # attention on rotate-half inputs equals the oracle on permuted inputs
+    q, k, v, seg, pos = rand_case(32, N=90, H=2, D=16)
+    theta = 1e4
+    out, lse = oracle.attn_fwd(orope.half_to_interleaved(q),
+                               orope.half_to_interleaved(k), v, seg, pos,
+                               theta)
+    b, h = 0, 1
+    qr = orope.rope_rotate_half(q[b, :, h], pos[b], theta)
+    kr = orope.rope_rotate_half(k[b, :, h], pos[b], theta)
+    rows = np.arange(90)
+    s = np.where(oracle.allowed_mask(seg[b], rows, rows), qr @ kr.T / 4.0,
+                 -np.inf)
+    ref_lse = np.log(np.exp(s - s.max(1, keepdims=True)).sum(1)) + s.max(1)
+    ref_out = np.exp(s - ref_lse[:, None]) @ v[b, :, h]
+    np.testing.assert_allclose(out[b, :, h], ref_out, atol=1e-12)
+    np.testing.assert_allclose(lse[b, h], ref_lse, atol=1e-12)

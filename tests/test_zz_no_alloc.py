@@ -66,5 +66,6 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(cuda_dev):
     fake = ctypes.c_void_p(1 << 20)
     st = ops.lib().lwm_blockattn_fwd_noalloc(
         fake, fake, fake, fake, fake, 5e7, 128, 128, 262144, 1, 262144, 32,
-        128, ops.DTYPE_BF16, ops.QK_BF16, fake, fake, None)
+        128, ops.DTYPE_BF16, ops.QK_BF16, ops.ROPE_INTERLEAVED, fake, fake,
+        None)
     assert st == ops.ERR_WORKSPACE
