@@ -307,6 +307,147 @@ def bench_decode(args):
     print(json.dumps(line), flush=True)
 
 
+FFN_METRIC = ("blockwise SwiGLU FFN TFLOP/s (3 projections, chunked over "
+              "tokens) at 1 B200; % of bf16 tensor peak")
+
+
+def ffn_oracle_sample(t_host, budget_s):
+    """Time the fp64 oracle MLP on the first R tokens (full weights), R
+    sized so one run takes about budget_s. Returns (TFLOP/s, info)."""
+    import oracle
+    from threadpoolctl import threadpool_info
+    w = {k: v.float().numpy().astype(np.float64) for k, v in t_host.items()
+         if k != "x"}
+    x = t_host["x"]
+    Dm, F = x.shape[1], w["w_gate"].shape[0]
+
+    def run(R):
+        xs = x[:R].float().numpy().astype(np.float64)
+        t0 = time.perf_counter()
+        oracle.swiglu_mlp(xs, w["w_gate"], w["w_up"], w["w_down"])
+        return time.perf_counter() - t0
+
+    R = 32
+    dt = run(R)
+    R = int(min(x.shape[0], max(32, R * max(budget_s, 0.1) / max(dt, 1e-3))))
+    dt = run(R)
+    threads = max((i.get("num_threads", 1) for i in threadpool_info()),
+                  default=1)
+    info = {"sample": f"oracle SwiGLU MLP (fp64 numpy) on the first {R} "
+                      f"tokens, full {Dm}x{F} weights; FLOP of those rows / "
+                      f"wall time",
+            "cores": int(threads), "host_cores": os.cpu_count(),
+            "seconds": dt}
+    return wl.ffn_flops(R, Dm, F) / dt / 1e12, info
+
+
+def bench_ffn(args):
+    """Blockwise FFN: three dense projections on the tensor cores."""
+    w = wl.FFN_WORKLOADS[args.workload]
+    flop = wl.ffn_flops(w.T, w.Dm, w.F)
+    cfg = {"workload": w.name, "T": w.T, "Dm": w.Dm, "F": w.F,
+           "chunk": w.chunk, "weights": "N(0, 0.02^2) bf16",
+           "l2": "inputs and weights larger than L2 (no flush)"}
+    if args.impl == "reference":
+        if int(os.environ.get("RANK", "0")) != 0:
+            return
+        t_host = wl.make_ffn_inputs(w.T, w.Dm, w.F, args.seed, device="cpu",
+                                    w_std=w.w_std)
+        vals, secs = [], []
+        for i in range(args.warmup + args.steps):
+            tf, info = ffn_oracle_sample(t_host, args.ref_budget)
+            if i >= args.warmup:
+                vals.append(tf)
+                secs.append(info["seconds"])
+        value = float(np.mean(vals))
+        print(json.dumps({
+            "impl": "reference", "metric": FFN_METRIC, "value": value,
+            "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": float(np.mean(secs)) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "config": cfg,
+            "cpu_baseline": {"kind": "oracle", "value": value,
+                             "unit": "TFLOP/s", "cores": info["cores"],
+                             "sample": info["sample"]},
+            "e2e": {"value": value, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+            flush=True)
+        return
+    from long_context_blockwise_causal_b200 import ops
+    dev = torch.device("cuda", 0)
+    t = wl.make_ffn_inputs(w.T, w.Dm, w.F, args.seed, device=dev,
+                           w_std=w.w_std)
+    y = torch.empty_like(t["x"])
+    ws = torch.empty(ops.ffn_workspace_size(w.chunk, w.F), dtype=torch.uint8,
+                     device=dev)
+    step = lambda: ops.ffn_fwd(t["x"], t["w_gate"], t["w_up"], t["w_down"],
+                               chunk=w.chunk, y=y, workspace=ws)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev)
+    clocks.start()
+    time.sleep(0.3)
+    l0 = ops.kernel_launches()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    launches = ops.kernel_launches() - l0
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    tflops = flop / (ms / 1e3) / 1e12
+    pk = peaks()
+    line = {"metric": FFN_METRIC, "value": tflops, "unit": "TFLOP/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": cfg, "tokens_per_s": w.T / (ms / 1e3),
+            "roofline": {"bound": "tensor", "kernel": "mlp_gemm_kernel",
+                         "achieved": tflops, "peak": pk["bf16_tflops_sustained"],
+                         "unit": "TFLOP/s",
+                         "frac": tflops / pk["bf16_tflops_sustained"],
+                         "frac_of_burst_peak": tflops / pk["bf16_tflops"],
+                         "traffic": None,
+                         "peak_kind": f"bf16 sustained ({pk['source']})"},
+            "gpu_launches": int(launches), "device_status": ops.last_status(),
+            "clocks": clk}
+    if not args.no_e2e:
+        # through the public call with host buffers: x in, y out per step
+        xh = t["x"].cpu().pin_memory()
+        yh = torch.empty_like(xh).pin_memory()
+        xd = torch.empty_like(t["x"])
+
+        def e2e_step():
+            xd.copy_(xh, non_blocking=True)
+            ops.ffn_fwd(xd, t["w_gate"], t["w_up"], t["w_down"],
+                        chunk=w.chunk, y=y, workspace=ws)
+            yh.copy_(y, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1) / args.steps
+        nb = xh.numel() * xh.element_size()
+        line["e2e"] = {"value": flop / (ems / 1e3) / 1e12, "unit": "TFLOP/s",
+                       "ms_per_step": ems, "h2d_bytes_per_step": nb,
+                       "d2h_bytes_per_step": nb}
+    if not args.no_cpu_baseline:
+        t_host = {k: v.cpu() for k, v in t.items()}
+        tf, info = ffn_oracle_sample(t_host, args.cpu_budget)
+        line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s",
+                                "kind": "oracle", **info}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -314,7 +455,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="text32k",
-                    choices=sorted(wl.WORKLOADS) + sorted(DECODE_WORKLOADS))
+                    choices=sorted(wl.WORKLOADS) + sorted(DECODE_WORKLOADS)
+                    + sorted(wl.FFN_WORKLOADS))
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--N", type=int, default=None,
                     help="override the workload's sequence length (profiling)")
@@ -335,6 +477,9 @@ def main():
     if args.workload in DECODE_WORKLOADS:
         if args.impl != "reference":
             bench_decode(args)
+        return
+    if args.workload in wl.FFN_WORKLOADS:
+        bench_ffn(args)
         return
     if args.impl == "reference":
         # host cores only: rank 0 runs the oracle, other ranks have no work

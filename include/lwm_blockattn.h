@@ -240,6 +240,32 @@ LWM_API int lwm_blockattn_grad_finish(const float* acc,
                                       int rope_layout, void* grad,
                                       void* stream);
 
+/* ---------------------------------------------------------------------
+ * Blockwise feed-forward network: the Llama-2 SwiGLU MLP of the blockwise
+ * transformer, run over the tokens in chunks so that only one chunk's
+ * intermediate activations exist at a time ("LWM：突破 100 万 Token 的开源大
+ * 模型", 配置参数: scan_mlp with scan_mlp_chunk_size 8192; the Llama-2-7B
+ * backbone, "Inside Large World Model", Core Architecture).
+ *
+ * Bytes of workspace lwm_blockffn_fwd needs: one chunk's intermediate,
+ * chunk x F bf16 (chunk clipped to T by the caller or not: the larger is
+ * safe). */
+LWM_API size_t lwm_blockffn_workspace_size(int chunk, int F);
+
+/* y = (silu(x Wg^T) * (x Wu^T)) Wd^T over T tokens, `chunk` tokens at a
+ * time.
+ *   x      [T][Dm] bf16            y [T][Dm] bf16 (written)
+ *   w_gate, w_up [F][Dm] bf16, w_down [Dm][F] bf16 (nn.Linear layout:
+ *          row = output feature)
+ * silu(h) = h / (1 + e^-h); products accumulate in fp32 on the tensor
+ * cores; the intermediate is rounded to bf16 once. Dm and F multiples of
+ * 64; only LWM_DTYPE_BF16. Async on stream; nothing launched on error. */
+LWM_API int lwm_blockffn_fwd(const void* x, const void* w_gate,
+                             const void* w_up, const void* w_down, int T,
+                             int Dm, int F, int chunk, int dtype, void* y,
+                             void* workspace, size_t workspace_bytes,
+                             void* stream);
+
 /* Tile classifier (exported so it can be checked bit-exactly). For each
  * batch row b and query block t (Tq = ceil(N/block_q) blocks), key blocks
  * j (Tk = ceil(N/block_k)):

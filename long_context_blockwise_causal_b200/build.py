@@ -18,7 +18,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "liblwm_blockattn.so")
 SOURCES = ["api.cu", "aux_kernels.cu", "simt.cu", "fwd_tc.cu", "bwd_tc.cu",
-           "noalloc.cu", "decode.cu"]
+           "noalloc.cu", "decode.cu", "mlp.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
          "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr",

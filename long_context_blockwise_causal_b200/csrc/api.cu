@@ -7,6 +7,7 @@
 
 #include "aux_kernels.cuh"
 #include "decode.cuh"
+#include "mlp.cuh"
 #include "tc_kernels.cuh"
 
 namespace lwm {
@@ -582,6 +583,43 @@ int lwm_blockattn_grad_finish(const float* acc, const int32_t* positions,
       acc, positions, rope_table, B, N, H, scale,
       rope_layout == LWM_ROPE_HALF, static_cast<__nv_bfloat16*>(grad),
       static_cast<cudaStream_t>(stream)));
+}
+
+size_t lwm_blockffn_workspace_size(int chunk, int F) {
+  if (chunk < 1 || F < 1) return 0;
+  return align_up(size_t(chunk) * F * 2);
+}
+
+int lwm_blockffn_fwd(const void* x, const void* w_gate, const void* w_up,
+                     const void* w_down, int T, int Dm, int F, int chunk,
+                     int dtype, void* y, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  if (T < 0 || Dm < 1 || F < 1 || chunk < 1) return LWM_ERR_INVALID_ARG;
+  if (dtype != LWM_DTYPE_BF16 || Dm % 64 != 0 || F % 64 != 0)
+    return LWM_ERR_UNSUPPORTED;
+  if (T == 0) return LWM_OK;
+  if (int64_t(T) * std::max(Dm, F) >= (int64_t(1) << 40))
+    return LWM_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, w_gate, w_up, w_down, y, workspace};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return LWM_ERR_INVALID_ARG;
+  const int c = std::min(chunk, T);
+  if (workspace_bytes < lwm_blockffn_workspace_size(c, F))
+    return LWM_ERR_WORKSPACE;
+  int* status = status_word();
+  if (!status) return LWM_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const char* xb = static_cast<const char*>(x);
+  char* yb = static_cast<char*>(y);
+  // one chunk of tokens at a time: only [chunk][F] of intermediate is live
+  for (int t0 = 0; t0 < T; t0 += c) {
+    const int m = std::min(c, T - t0);
+    LWM_TRY(launch_mlp_up(xb + size_t(t0) * Dm * 2, w_gate, w_up, m, Dm, F,
+                          workspace, status, st));
+    LWM_TRY(launch_mlp_down(workspace, w_down, m, F, Dm,
+                            yb + size_t(t0) * Dm * 2, status, st));
+  }
+  return LWM_OK;
 }
 
 int lwm_blockattn_classify(const int32_t* segment_ids, int B, int N,

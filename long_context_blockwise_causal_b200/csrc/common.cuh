@@ -103,6 +103,15 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap,
       : "memory");
 }
 
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap,
+                                            uint32_t bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::"
+      "complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(tmap), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_store_4d(const void* tmap, uint32_t src,
                                              int c0, int c1, int c2, int c3) {
   asm volatile(
@@ -282,6 +291,11 @@ __device__ __forceinline__ float bf16lo_to_f32(uint32_t w) {
 }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t w) {
   return __uint_as_float(w & 0xFFFF0000u);
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 __device__ __forceinline__ float ex2(float x) {
   float y;

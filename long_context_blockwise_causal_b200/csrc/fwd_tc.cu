@@ -814,6 +814,24 @@ bool make_bnhd_map(CUtensorMap* m, const void* base, int B, int N, int H) {
   return r == CUDA_SUCCESS;
 }
 
+// Row-major bf16 [rows][cols] matrix as a 2-D map {cols, rows}; box 64
+// columns (128 bytes) x box_rows rows with the 128-byte swizzle.
+bool make_2d_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols,
+                 int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(cols) * 2};
+  cuuint32_t box[2] = {64, cuuint32_t(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // fp32 [B][N][H][128] tensor as a 4-D map {D, H, N, B}; box 32 x 1 x 32 x 1
 // (one 128-byte column chunk of 32 rows) with the 128-byte swizzle.
 bool make_bnhd_f32_map(CUtensorMap* m, const void* base, int B, int N,

@@ -84,6 +84,10 @@ bool make_bnhd_map(CUtensorMap* m, const void* base, int B, int N, int H);
 // 128-byte swizzle (used for the dQ reduce-add).
 bool make_bnhd_f32_map(CUtensorMap* m, const void* base, int B, int N,
                        int H);
+// Row-major bf16 [rows][cols] matrix as a 2-D map, box 64 x box_rows,
+// 128-byte swizzle (cols * 2 must be a multiple of 16 bytes).
+bool make_2d_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols,
+                 int box_rows);
 int sm_count();
 cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t st);
 

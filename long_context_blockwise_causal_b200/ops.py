@@ -74,6 +74,9 @@ _SIGS = {
                                      _vp, _vp, _sz, _vp]),
     "lwm_blockattn_grad_finish": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                                        _i, _vp, _vp]),
+    "lwm_blockffn_workspace_size": (_sz, [_i, _i]),
+    "lwm_blockffn_fwd": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp,
+                              _vp, _sz, _vp]),
 }
 
 
@@ -348,6 +351,27 @@ def grad_finish(acc, positions=None, table=None, out=None, stream=None,
         _layout_code(rope_layout), _ptr(out), _stream(stream))
     _check(st, "lwm_blockattn_grad_finish")
     return out
+
+
+def ffn_workspace_size(chunk, F) -> int:
+    return int(lib().lwm_blockffn_workspace_size(chunk, F))
+
+
+def ffn_fwd(x, w_gate, w_up, w_down, chunk=8192, y=None, workspace=None,
+            stream=None):
+    """Blockwise SwiGLU MLP: y = (silu(x Wg^T) * (x Wu^T)) Wd^T, `chunk`
+    tokens at a time. x [T, Dm]; Wg, Wu [F, Dm]; Wd [Dm, F]; bf16."""
+    _need_cuda(x, w_gate, w_up, w_down, y, workspace)
+    T, Dm = x.shape
+    F = w_gate.shape[0]
+    y = torch.empty_like(x) if y is None else y
+    c = max(1, min(int(chunk), T))
+    ws = _workspace(ffn_workspace_size(c, F), x.device, workspace)
+    st = lib().lwm_blockffn_fwd(
+        _ptr(x), _ptr(w_gate), _ptr(w_up), _ptr(w_down), T, Dm, F, int(chunk),
+        _dtype_code(x), _ptr(y), _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "lwm_blockffn_fwd")
+    return y
 
 
 def classify(segment_ids, block_q=BLOCK, block_k=BLOCK, with_class=True,

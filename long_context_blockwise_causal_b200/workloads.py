@@ -179,3 +179,46 @@ def make_inputs(w: Workload, seed: int, device="cpu", dtype=None,
         t["dout"] = random_tensor(shape, seed * 16 + 4, w.scale, dtype,
                                   device)
     return t
+
+
+# ------------------------------------------------ blockwise feed-forward
+@dataclass(frozen=True)
+class FfnWorkload:
+    """The Llama-2-7B MLP over T tokens in chunks of `chunk` (the pages'
+    scan_mlp_chunk_size); activations N(0,1), weights N(0, 0.02^2) (the
+    Llama initialiser's std), bf16."""
+    name: str
+    T: int
+    Dm: int
+    F: int
+    chunk: int
+    w_std: float = 0.02
+
+
+FFN_WORKLOADS = {
+    # one 32K-token sequence of LWM-Text-32K through one MLP block
+    "mlp32k": FfnWorkload("mlp32k", 32768, 4096, 11008, 8192),
+    # a single chunk (the unit the pages' scan_mlp processes)
+    "mlp8k": FfnWorkload("mlp8k", 8192, 4096, 11008, 8192),
+}
+
+
+def ffn_flops(T: int, Dm: int, F: int) -> int:
+    """Multiply-adds x2 of the three projections (the SwiGLU itself is
+    O(T F) and not counted)."""
+    return 2 * T * Dm * F * 3
+
+
+def make_ffn_inputs(T: int, Dm: int, F: int, seed: int, device="cpu",
+                    w_std: float = 0.02, dtype=None):
+    """x [T, Dm]; w_gate, w_up [F, Dm]; w_down [Dm, F] (nn.Linear layout)."""
+    import torch
+
+    dtype = torch.bfloat16 if dtype is None else dtype
+    s = seed * 16
+    return {
+        "x": random_tensor((1, T, Dm), s + 5, 1.0, dtype, device)[0],
+        "w_gate": random_tensor((1, F, Dm), s + 6, w_std, dtype, device)[0],
+        "w_up": random_tensor((1, F, Dm), s + 7, w_std, dtype, device)[0],
+        "w_down": random_tensor((1, Dm, F), s + 8, w_std, dtype, device)[0],
+    }

@@ -37,6 +37,7 @@ Modules:
   ring       -- partial attention over a key block, the log-sum-exp merge and
                 a P-device ring run in order (RingAttention).
   classify   -- tile classification (brute force and a counting form).
+  ffn        -- the blockwise (chunked) SwiGLU feed-forward network.
 """
 
 from .rope import (  # noqa: F401
@@ -51,6 +52,9 @@ from .blockwise import blockwise_fwd  # noqa: F401
 from .ring import (  # noqa: F401
     attn_fwd_partial, merge_partials, ring_chunks, ring_fwd, bwd_delta,
     attn_bwd_partial, ring_bwd,
+)
+from .ffn import (  # noqa: F401
+    silu, swiglu_intermediate, swiglu_mlp, blockwise_mlp,
 )
 from .classify import (  # noqa: F401
     classify_bruteforce, classify_count, TILE_EMPTY, TILE_PARTIAL, TILE_FULL,
