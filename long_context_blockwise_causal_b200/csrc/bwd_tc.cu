@@ -20,9 +20,10 @@
 // Queries and keys arrive pre-rotated (R(pos) q, R(pos) k); dK = R(-pos)
 // (dK~ / sqrt(D)) in the epilogue, dQ the same in the conversion kernel.
 //
-// Warps: 0-3 compute (thread = key row = TMEM lane), 4-7 dQ reduction and
-// per-block (lse, D) staging, 8 TMA producer, 9 tcgen05 issuer + TMEM
-// owner, 10-11 idle (complete the warpgroup for setmaxnreg).
+// Warps: 0-7 compute (thread = key row = TMEM lane; warps w and w + 4
+// share the lanes and split the 128 columns), 8-11 dQ reduction and
+// per-block (lse, D) staging, 12 TMA producer, 13 tcgen05 issuer + TMEM
+// owner, 14-15 idle (complete the warpgroup for setmaxnreg).
 #include <cuda.h>
 
 #include "aux_kernels.cuh"
@@ -31,10 +32,11 @@
 namespace lwm {
 namespace {
 
-constexpr int kThreadsBwd = 12 * 32;
-constexpr int kLaunchRegsBwd = 168;   // 65536 / 384, rounded down to 8
-constexpr int kRegsCompute = 240, kRegsDq = 160, kRegsMiscBwd = 104;
-static_assert(kRegsCompute + kRegsDq + kRegsMiscBwd == 3 * kLaunchRegsBwd,
+constexpr int kThreadsBwd = 16 * 32;
+constexpr int kLaunchRegsBwd = 128;   // 65536 / 512
+// two compute warpgroups, the dQ warpgroup, the producer/MMA warpgroup
+constexpr int kRegsCompute = 152, kRegsDq = 128, kRegsMiscBwd = 80;
+static_assert(2 * kRegsCompute + kRegsDq + kRegsMiscBwd == 4 * kLaunchRegsBwd,
               "register split must equal the launch allocation");
 constexpr int kTile = kBlock * kHeadDim * 2;   // 32 KB
 constexpr int kHalf = kTile / 2;
@@ -137,25 +139,25 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(bar(bAux1), 128);
     mbar_init(bar(bStFull), 1);
     mbar_init(bar(bDptFull), 1);
-    mbar_init(bar(bPFull), 4);
+    mbar_init(bar(bPFull), 8);
     mbar_init(bar(bDqFull), 1);
     mbar_init(bar(bDqEmpty), 4);
     mbar_init(bar(bAccFull), 1);
-    mbar_init(bar(bAccEmpty), 4);
+    mbar_init(bar(bAccEmpty), 8);
     mbar_init(bar(bDoneB), 1);
     mbar_init(bar(bItemFull0), 1);
     mbar_init(bar(bItemFull1), 1);
-    // consumers: 4 compute warps, 4 dQ warps, the MMA lane
-    mbar_init(bar(bItemEmpty0), 9);
-    mbar_init(bar(bItemEmpty1), 9);
+    // consumers: 8 compute warps, 4 dQ warps, the MMA lane
+    mbar_init(bar(bItemEmpty0), 13);
+    mbar_init(bar(bItemEmpty1), 13);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == 13) {
     tmem_alloc(smem_u32(tmem_holder), 512);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == 12 && lane == 0) {
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
@@ -169,11 +171,14 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t tA = tmem, tB = tmem + 128, tC = tmem + 256, tD = tmem + 384;
   const int nitems = p.total_items;
 
-  if (warp < 4) {
+  if (warp < 8) {
     // ---------------------------------------------------- compute (keys)
+    // two warps per TMEM lane quadrant: warp w owns key rows 32 (w % 4) ..
+    // +31 and the 64 query columns (or d columns) of half ch = w / 4
     regs_inc<kRegsCompute>();
-    const int r = warp * 32 + lane;  // key row of the block = TMEM lane
-    const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    const int q4 = warp & 3, ch = warp >> 2;
+    const int r = q4 * 32 + lane;  // key row of the block = TMEM lane
+    const uint32_t lane_off = uint32_t(q4 * 32) << 16;
     int g = 0, n = 0;
     bool ok = true;
     for (int u = 0; ok; ++u) {
@@ -208,23 +213,26 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int q0 = p.q_off + i * kBlock;  // global index of query 0
         // every key of the block seen by every query of the block
         const bool full = klo_max <= q0 && khi_min >= q0 + kBlock - 1;
-        const float* ls = aux_lse + st * 128;
-        const float* dl = aux_del + st * 128;
-        uint8_t* dsrow = smem + kSDS + r * 128;
+        const float* ls = aux_lse + st * 128 + ch * 64;
+        const float* dl = aux_del + st * 128 + ch * 64;
+        uint8_t* dsrow = smem + kSDS + ch * kHalf + r * 128;
+        // this warp's 64 query columns of S^T / dP^T start at column ch*64;
+        // its bf16 P^T and dS^T go to the first 32 of those columns (inside
+        // its own range, so the other half's loads are never overwritten)
+        const uint32_t colA = tA + lane_off + ch * 64;
+        const uint32_t colB = tB + lane_off + ch * 64;
         // phase 1 (while dP^T is still on the tensor pipe):
         // P^T = 2^(S^T c - lse log2 e), masked; bf16 copy over S^T
-        float pf[4][32];
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
+        float pf[2][32];
+        {
           uint32_t sv[2][32];
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc)
-            tmem_ld32(tA + lane_off + (2 * half + cc) * 32, sv[cc]);
+          for (int cc = 0; cc < 2; ++cc) tmem_ld32(colA + cc * 32, sv[cc]);
           tmem_wait_ld();
           if (!full) {
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
-              const int qb = q0 + (2 * half + cc) * 32;
+              const int qb = q0 + ch * 64 + cc * 32;
               const int lo = lo_k - qb, hi = hi_k - qb;
 #pragma unroll
               for (int x = 0; x < 32; ++x)
@@ -233,11 +241,10 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
 #pragma unroll
           for (int cc = 0; cc < 2; ++cc) {
-            const int c = 2 * half + cc;
             uint32_t pp[16];
 #pragma unroll
             for (int x = 0; x < 32; x += 4) {
-              const float4 l4 = *reinterpret_cast<const float4*>(ls + c * 32 + x);
+              const float4 l4 = *reinterpret_cast<const float4*>(ls + cc * 32 + x);
               const float2 t0 = fma2(make_float2(__uint_as_float(sv[cc][x]),
                                                  __uint_as_float(sv[cc][x + 1])),
                                      make_float2(p.scale_log2, p.scale_log2),
@@ -246,14 +253,14 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                  __uint_as_float(sv[cc][x + 3])),
                                      make_float2(p.scale_log2, p.scale_log2),
                                      make_float2(-l4.z, -l4.w));
-              pf[c][x] = ex2(t0.x);
-              pf[c][x + 1] = ex2(t0.y);
-              pf[c][x + 2] = ex2(t1.x);
-              pf[c][x + 3] = ex2(t1.y);
-              pp[x >> 1] = pack_bf16x2(pf[c][x], pf[c][x + 1]);
-              pp[(x >> 1) + 1] = pack_bf16x2(pf[c][x + 2], pf[c][x + 3]);
+              pf[cc][x] = ex2(t0.x);
+              pf[cc][x + 1] = ex2(t0.y);
+              pf[cc][x + 2] = ex2(t1.x);
+              pf[cc][x + 3] = ex2(t1.y);
+              pp[x >> 1] = pack_bf16x2(pf[cc][x], pf[cc][x + 1]);
+              pp[(x >> 1) + 1] = pack_bf16x2(pf[cc][x + 2], pf[cc][x + 3]);
             }
-            tmem_st16(tA + lane_off + c * 16, pp);
+            tmem_st16(colA + cc * 16, pp);
           }
         }
         // phase 2: dS^T = P^T (dP^T - D) once dP^T has landed
@@ -264,35 +271,31 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           break;
         }
         tc_fence_after();
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
+        {
           uint32_t dv[2][32];
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc)
-            tmem_ld32(tB + lane_off + (2 * half + cc) * 32, dv[cc]);
+          for (int cc = 0; cc < 2; ++cc) tmem_ld32(colB + cc * 32, dv[cc]);
           tmem_wait_ld();
 #pragma unroll
           for (int cc = 0; cc < 2; ++cc) {
-            const int c = 2 * half + cc;
             uint32_t pd[16];
 #pragma unroll
             for (int x = 0; x < 32; x += 4) {
-              const float4 d4 = *reinterpret_cast<const float4*>(dl + c * 32 + x);
-              const float ds0 = pf[c][x] * (__uint_as_float(dv[cc][x]) - d4.x);
-              const float ds1 = pf[c][x + 1] * (__uint_as_float(dv[cc][x + 1]) - d4.y);
-              const float ds2 = pf[c][x + 2] * (__uint_as_float(dv[cc][x + 2]) - d4.z);
-              const float ds3 = pf[c][x + 3] * (__uint_as_float(dv[cc][x + 3]) - d4.w);
+              const float4 d4 = *reinterpret_cast<const float4*>(dl + cc * 32 + x);
+              const float ds0 = pf[cc][x] * (__uint_as_float(dv[cc][x]) - d4.x);
+              const float ds1 = pf[cc][x + 1] * (__uint_as_float(dv[cc][x + 1]) - d4.y);
+              const float ds2 = pf[cc][x + 2] * (__uint_as_float(dv[cc][x + 2]) - d4.z);
+              const float ds3 = pf[cc][x + 3] * (__uint_as_float(dv[cc][x + 3]) - d4.w);
               pd[x >> 1] = pack_bf16x2(ds0, ds1);
               pd[(x >> 1) + 1] = pack_bf16x2(ds2, ds3);
             }
-            tmem_st16(tB + lane_off + c * 16, pd);
-            // dS row r, queries c*32 .. c*32+31: query half (c >> 1),
-            // 16-byte chunks (c & 1) * 4 .. +3 of that 128-byte row
+            tmem_st16(colB + cc * 16, pd);
+            // dS row r, queries ch*64 + cc*32 .. +31: the query half ch of
+            // the tile, 16-byte chunks cc*4 .. +3 of that 128-byte row
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int lc = (c & 1) * 4 + e;
-              *reinterpret_cast<uint4*>(dsrow + (c >> 1) * kHalf +
-                                        ((lc ^ (r & 7)) << 4)) =
+              const int lc = cc * 4 + e;
+              *reinterpret_cast<uint4*>(dsrow + ((lc ^ (r & 7)) << 4)) =
                   make_uint4(pd[4 * e], pd[4 * e + 1], pd[4 * e + 2],
                              pd[4 * e + 3]);
             }
@@ -315,17 +318,22 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       // a key block no query sees issued no MMA: its accumulators hold
       // nothing of this item (bf16 mode writes zeros, fp32 mode adds none)
       const bool seen = m.qlo <= m.qhi;
+      const float4* trow = reinterpret_cast<const float4*>(
+          p.table + int64_t(valid_k && p.pos_k ? __ldg(p.pos_k + rowbase + kj)
+                                               : 0) *
+                        (kHeadDim / 2));
       if (p.dk_acc) {
         // fp32 accumulators carried across calls: add dV and the unscaled,
-        // rotated dK~ (this thread owns key row kj of this launch)
+        // rotated dK~ (this thread owns key row kj, d columns ch*64 .. +63)
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 4; ++c) {
+          const int col = ch * 64 + (c & 1) * 32;
           uint32_t v[32];
-          tmem_ld32((c < 4 ? tC : tD) + lane_off + (c & 3) * 32, v);
+          tmem_ld32((c < 2 ? tC : tD) + lane_off + col, v);
           tmem_wait_ld();
           if (valid_k && seen) {
             float4* dst = reinterpret_cast<float4*>(
-                (c < 4 ? p.dv_acc : p.dk_acc) + orow + (c & 3) * 32);
+                (c < 2 ? p.dv_acc : p.dk_acc) + orow + col);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
               float4 a = dst[e];
@@ -338,35 +346,33 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
         }
       } else {
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tC + lane_off + c * 32, v);
-        tmem_wait_ld();
-        if (!seen)
-#pragma unroll
-          for (int x = 0; x < 32; ++x) v[x] = 0u;
-        if (valid_k) {
-          uint4* dst = reinterpret_cast<uint4*>(p.dv + orow + c * 32);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(
-                pack_bf16x2(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
-                pack_bf16x2(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
-                pack_bf16x2(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
-                pack_bf16x2(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
-        }
-      }
-      const float4* trow = reinterpret_cast<const float4*>(
-          p.table + int64_t(valid_k ? __ldg(p.pos_k + rowbase + kj) : 0) *
-                        (kHeadDim / 2));
-      if (p.rope_half) {
-        // pair k = (dim k, dim k + 64): columns c*32.. with (c+2)*32..
+        // dV: d columns ch*64 .. +63
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
+          const int col = ch * 64 + c * 32;
+          uint32_t v[32];
+          tmem_ld32(tC + lane_off + col, v);
+          tmem_wait_ld();
+          if (!seen)
+#pragma unroll
+            for (int x = 0; x < 32; ++x) v[x] = 0u;
+          if (valid_k) {
+            uint4* dst = reinterpret_cast<uint4*>(p.dv + orow + col);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              dst[e] = make_uint4(
+                  pack_bf16x2(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
+                  pack_bf16x2(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
+                  pack_bf16x2(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
+                  pack_bf16x2(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
+          }
+        }
+        if (p.rope_half) {
+          // pair k = (dim k, dim k + 64): this warp takes columns ch*32 ..
+          // +31 with (ch+2)*32 .. +31, i.e. pairs ch*32 .. ch*32 + 31
           uint32_t va[32], vb[32];
-          tmem_ld32(tD + lane_off + c * 32, va);
-          tmem_ld32(tD + lane_off + (c + 2) * 32, vb);
+          tmem_ld32(tD + lane_off + ch * 32, va);
+          tmem_ld32(tD + lane_off + (ch + 2) * 32, vb);
           tmem_wait_ld();
           if (!seen)
 #pragma unroll
@@ -374,8 +380,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           if (valid_k) {
             uint32_t oa[16], ob[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {  // pairs c*32 + 2e, 2e + 1
-              const float4 cs = __ldg(trow + c * 16 + e);
+            for (int e = 0; e < 16; ++e) {  // pairs ch*32 + 2e, 2e + 1
+              const float4 cs = __ldg(trow + ch * 16 + e);
               const float a0 = __uint_as_float(va[2 * e]) * p.scale;
               const float a1 = __uint_as_float(va[2 * e + 1]) * p.scale;
               const float b0 = __uint_as_float(vb[2 * e]) * p.scale;
@@ -386,8 +392,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
               ob[e] = pack_bf16x2(fmaf(b0, cs.x, -a0 * cs.y),
                                   fmaf(b1, cs.z, -a1 * cs.w));
             }
-            uint4* da = reinterpret_cast<uint4*>(p.dk + orow + c * 32);
-            uint4* db = reinterpret_cast<uint4*>(p.dk + orow + (c + 2) * 32);
+            uint4* da = reinterpret_cast<uint4*>(p.dk + orow + ch * 32);
+            uint4* db = reinterpret_cast<uint4*>(p.dk + orow + (ch + 2) * 32);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               da[e] = make_uint4(oa[4 * e], oa[4 * e + 1], oa[4 * e + 2],
@@ -396,49 +402,51 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                                  ob[4 * e + 3]);
             }
           }
-        }
-      } else {
+        } else {
+          // interleaved pairs (2k, 2k+1): d columns ch*64 .. +63
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tD + lane_off + c * 32, v);
-        tmem_wait_ld();
-        if (!seen)
+          for (int c = 0; c < 2; ++c) {
+            const int col = ch * 64 + c * 32;
+            uint32_t v[32];
+            tmem_ld32(tD + lane_off + col, v);
+            tmem_wait_ld();
+            if (!seen)
 #pragma unroll
-          for (int x = 0; x < 32; ++x) v[x] = 0u;
-        if (valid_k) {
-          uint32_t o[16];
+              for (int x = 0; x < 32; ++x) v[x] = 0u;
+            if (valid_k) {
+              uint32_t o[16];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {  // pairs c*16 + 2e, 2e+1
-            const float4 cs = __ldg(trow + c * 8 + e);
-            const float a0 = __uint_as_float(v[4 * e]) * p.scale;
-            const float b0 = __uint_as_float(v[4 * e + 1]) * p.scale;
-            const float a1 = __uint_as_float(v[4 * e + 2]) * p.scale;
-            const float b1 = __uint_as_float(v[4 * e + 3]) * p.scale;
-            // R(-pos): (a, b) -> (a c + b s, b c - a s)
-            o[2 * e] = pack_bf16x2(fmaf(a0, cs.x, b0 * cs.y),
-                                   fmaf(b0, cs.x, -a0 * cs.y));
-            o[2 * e + 1] = pack_bf16x2(fmaf(a1, cs.z, b1 * cs.w),
-                                       fmaf(b1, cs.z, -a1 * cs.w));
+              for (int e = 0; e < 8; ++e) {  // pairs col/2 + 2e, 2e+1
+                const float4 cs = __ldg(trow + col / 4 + e);
+                const float a0 = __uint_as_float(v[4 * e]) * p.scale;
+                const float b0 = __uint_as_float(v[4 * e + 1]) * p.scale;
+                const float a1 = __uint_as_float(v[4 * e + 2]) * p.scale;
+                const float b1 = __uint_as_float(v[4 * e + 3]) * p.scale;
+                // R(-pos): (a, b) -> (a c + b s, b c - a s)
+                o[2 * e] = pack_bf16x2(fmaf(a0, cs.x, b0 * cs.y),
+                                       fmaf(b0, cs.x, -a0 * cs.y));
+                o[2 * e + 1] = pack_bf16x2(fmaf(a1, cs.z, b1 * cs.w),
+                                           fmaf(b1, cs.z, -a1 * cs.w));
+              }
+              uint4* dst = reinterpret_cast<uint4*>(p.dk + orow + col);
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                dst[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2],
+                                    o[4 * e + 3]);
+            }
           }
-          uint4* dst = reinterpret_cast<uint4*>(p.dk + orow + c * 32);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
         }
-      }
-      }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(bAccEmpty));
       ++n;
     }
-  } else if (warp < 8) {
+  } else if (warp < 12) {
     // ---------------------------------------------------- dQ + staging
     regs_dec<kRegsDq>();
-    const int r = (warp - 4) * 32 + lane;  // query row = TMEM lane
-    const uint32_t lane_off = uint32_t((warp - 4) * 32) << 16;
+    const int r = (warp - 8) * 32 + lane;  // query row = TMEM lane
+    const uint32_t lane_off = uint32_t((warp - 8) * 32) << 16;
     int g = 0;
     bool ok = true;
     int pb = 0, ph = 0, pq0 = 0;  // the block whose dQ is pending
@@ -448,30 +456,38 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     // boxes, 128-byte swizzle), then a TMA reduce-add of each box into the
     // fp32 accumulator; the stage goes back to the producer after the
     // reduce has read it.
-    const int wq = warp - 4;
+    const int wq = warp - 8;
     int pst = 0;  // stage of the pending block
     auto flush = [&](int t) -> bool {
       bool w = mbar_wait(bar(bDqFull), t & 1, abort_flag, p.status, kWaitNs);
       w = __all_sync(0xffffffffu, w);
       if (!w) return false;
       tc_fence_after();
-      uint32_t v[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tB + lane_off + c * 32, v[c]);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(bDqEmpty));
       const int qoff = kSQ + pst * kTile, ooff = kSDO + pst * kTile;
+      // two 32-column chunks at a time (64 registers); TMEM is released
+      // once the last chunk is in registers
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int box = (c < 2 ? qoff : ooff) + (wq * 2 + (c & 1)) * 4096;
-        uint8_t* rowp = smem + box + lane * 128;
+      for (int c2 = 0; c2 < 4; c2 += 2) {
+        uint32_t v[2][32];
+        tmem_ld32(tB + lane_off + c2 * 32, v[0]);
+        tmem_ld32(tB + lane_off + (c2 + 1) * 32, v[1]);
+        tmem_wait_ld();
+        if (c2 == 2) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(bDqEmpty));
+        }
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          *reinterpret_cast<uint4*>(rowp + ((e ^ (lane & 7)) << 4)) =
-              make_uint4(v[c][4 * e], v[c][4 * e + 1], v[c][4 * e + 2],
-                         v[c][4 * e + 3]);
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = c2 + cc;
+          const int box = (c < 2 ? qoff : ooff) + (wq * 2 + (c & 1)) * 4096;
+          uint8_t* rowp = smem + box + lane * 128;
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            *reinterpret_cast<uint4*>(rowp + ((e ^ (lane & 7)) << 4)) =
+                make_uint4(v[cc][4 * e], v[cc][4 * e + 1], v[cc][4 * e + 2],
+                           v[cc][4 * e + 3]);
+        }
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -523,7 +539,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     // warps 8-11 share one register budget, then split: 8 producer,
     // 9 MMA, 10-11 idle
     regs_dec<kRegsMiscBwd>();
-    if (warp == 8) {
+    if (warp == 12) {
     // ---------------------------------------------------- TMA producer
     if (lane == 0) {
       int g = 0, n = 0;
@@ -578,7 +594,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_wait(bar(bQFull0 + (f & 1)), (f >> 1) & 1, nullptr, p.status,
                   kWaitNs);
     }
-    } else if (warp == 9) {
+    } else if (warp == 13) {
     // ---------------------------------------------------- tcgen05 issuer
     if (lane == 0) {
       const uint32_t idKK = idesc_bf16(128, 128, 0, 0);  // A, B K-major
@@ -633,14 +649,18 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                            kWaitNs);
           if (!ok) break;
           tc_fence_after();
+          // bf16 P^T / dS^T of queries 64.. sit 32 columns further on
+          // (each compute warp packs its half inside its own S^T columns)
 #pragma unroll
           for (int k = 0; k < 8; ++k)  // dV += P^T dO
-            mma_ts(tC, tA + 8 * k, sdesc_sw128(ob + 2048 * k, kHalf, 1024),
-                   idKM, (!first_q || k > 0) ? 1u : 0u);
+            mma_ts(tC, tA + 8 * k + (k >= 4 ? 32 : 0),
+                   sdesc_sw128(ob + 2048 * k, kHalf, 1024), idKM,
+                   (!first_q || k > 0) ? 1u : 0u);
 #pragma unroll
           for (int k = 0; k < 8; ++k)  // dK~ += dS^T Q~
-            mma_ts(tD, tB + 8 * k, sdesc_sw128(qb + 2048 * k, kHalf, 1024),
-                   idKM, (!first_q || k > 0) ? 1u : 0u);
+            mma_ts(tD, tB + 8 * k + (k >= 4 ? 32 : 0),
+                   sdesc_sw128(qb + 2048 * k, kHalf, 1024), idKM,
+                   (!first_q || k > 0) ? 1u : 0u);
 #pragma unroll
           for (int k = 0; k < 8; ++k)  // dQ~ = dS K~, into B after dK read it
             mma_ss(tB, sdesc_sw128(sbase + kSDS + 2048 * k, kHalf, 1024),
@@ -671,7 +691,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

@@ -355,20 +355,27 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::bItemEmpty + (n & 1)));
       if (it < 0) break;
-      Item m = get_item(p, it);
-      if (!m.present[s]) continue;
+      const Item m = get_item(p, it);
+      // this warp's sub-tile as scalars: s is a run-time value, and an
+      // array indexed by it would live in local memory (reloaded after
+      // every asm statement of the tile loop)
+      const bool my_present = s ? m.present[1] : m.present[0];
+      const int my_t = s ? m.t[1] : m.t[0];
+      const int my_lo = s ? m.lo[1] : m.lo[0];
+      const int my_hi = s ? m.hi[1] : m.hi[0];
+      if (!my_present) continue;
       const int64_t rowbase = int64_t(m.b) * p.Nq;
-      const int q0 = m.t[s] * kBlock;
+      const int q0 = my_t * kBlock;
       const int i = q0 + r;
       const bool valid = i < p.Nq;
       // allowed keys of this row (global indices): lo_i <= key <= hi_i
       const int lo_i = valid ? __ldg(p.row_lo + rowbase + i) : 1;
       const int hi_i = valid ? __ldg(p.row_hi + rowbase + i) : 0;
-      const int lo_max = __ldg(p.lo_max + m.b * p.Tq + m.t[s]);
-      const int hi_min = __ldg(p.hi_min + m.b * p.Tq + m.t[s]);
+      const int lo_max = __ldg(p.lo_max + m.b * p.Tq + my_t);
+      const int hi_min = __ldg(p.hi_min + m.b * p.Tq + my_t);
       float m_used = -INFINITY, l = 0.f;
       bool first = true;
-      for (int j = m.hi[s]; j >= m.lo[s] && ok; --j) {
+      for (int j = my_hi; j >= my_lo && ok; --j) {
         ok = mbar_wait(bar(C::bSFull + s), sc & 1, abort_flag, p.status,
                        kWaitLimitNs);
         ok = __all_sync(0xffffffffu, ok);
@@ -524,7 +531,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (it < 0) break;
       Item m = get_item(p, it);
       const int64_t rowbase = int64_t(m.b) * p.Nq;
-      for (int s = 0; s < 2 && ok; ++s) {
+            for (int s = 0; s < 2 && ok; ++s) {
         if (!m.present[s]) continue;
         float4 cs0[8];
         bool valid;
@@ -570,6 +577,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_arrive(bar(C::bItemFull + (n & 1)));
         if (it < 0) break;
         Item m = get_item(p, it);
+        #pragma unroll
         for (int s = 0; s < 2 && ok; ++s) {
           if (!m.present[s]) continue;
           if (qfill[s] > 0)
@@ -671,6 +679,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             if (!ok) break;
             tc_fence_after();
           }
+          #pragma unroll
           for (int s = 0; s < 2 && ok; ++s) {
             if (prev >= 0 && active(m, s, prev)) {
               ok = mbar_wait(bar(C::bPFull + s), pc[s] & 1, abort_flag,
@@ -741,6 +750,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         // a sub-tile that sees no key block issued no MMA: its Q tile is
         // still consumed here, so the rotation is done with it before the
         // epilogue stages the (zero) output in the same buffer
+        #pragma unroll
         for (int s = 0; s < 2 && ok; ++s)
           if (m.present[s] && !qwaited[s]) {
             ok = mbar_wait(bar(C::bQReady + s), qc[s] & 1, abort_flag,
@@ -748,6 +758,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             qc[s]++;
           }
         if (!ok) break;
+        #pragma unroll
         for (int s = 0; s < 2; ++s)
           if (m.present[s]) {
             mma_commit(bar(C::bOFull + s));
