@@ -167,6 +167,8 @@ LWM_API size_t lwm_blockattn_fwd_block_workspace_size(int B, int Nq, int Nk,
  *   v      [B][Nk][H][D] bf16
  *   seg_q  [B][Nq], pos_q [B][Nq], seg_k [B][Nk] int32; segment ids
  *          non-decreasing along the whole sequence
+ *   rope_table  the table of lwm_blockattn_rope_table for (theta, max_pos),
+ *          reused across the calls of a ring; NULL: built in the workspace
  *   out    [B][Nq][H][D] bf16, lse [B][H][Nq] fp32 (natural log), written
  *          (not accumulated): fold them into a running result with
  *          lwm_blockattn_merge.
@@ -175,9 +177,9 @@ LWM_API int lwm_blockattn_fwd_block(const void* q, const void* k_rot,
                                     const void* v, const int32_t* seg_q,
                                     const int32_t* pos_q, const int32_t* seg_k,
                                     int q_off, int k_off, double theta,
-                                    int max_pos, int B, int Nq, int Nk, int H,
-                                    int D, int rope_layout, void* out,
-                                    float* lse,
+                                    int max_pos, const float* rope_table,
+                                    int B, int Nq, int Nk, int H, int D,
+                                    int rope_layout, void* out, float* lse,
                                     void* workspace, size_t workspace_bytes,
                                     void* stream);
 

@@ -387,7 +387,8 @@ size_t lwm_blockattn_fwd_block_workspace_size(int B, int Nq, int Nk, int H,
 int lwm_blockattn_fwd_block(const void* q, const void* k_rot, const void* v,
                             const int32_t* seg_q, const int32_t* pos_q,
                             const int32_t* seg_k, int q_off, int k_off,
-                            double theta, int max_pos, int B, int Nq, int Nk,
+                            double theta, int max_pos,
+                            const float* rope_table, int B, int Nq, int Nk,
                             int H, int D, int rope_layout, void* out,
                             float* lse, void* workspace,
                             size_t workspace_bytes, void* stream) {
@@ -416,7 +417,12 @@ int lwm_blockattn_fwd_block(const void* q, const void* k_rot, const void* v,
     LWM_TRY(launch_fill(lse, -INFINITY, size_t(B) * H * Nq, st));
     return LWM_OK;
   }
-  LWM_TRY(launch_rope_table(theta, D, max_pos, w.table, st));
+  if (rope_table) {
+    if (!aligned16(rope_table)) return LWM_ERR_INVALID_ARG;
+    w.table = const_cast<float*>(rope_table);
+  } else {
+    LWM_TRY(launch_rope_table(theta, D, max_pos, w.table, st));
+  }
   return run_forward(q, k_rot, nullptr, v, seg_q, pos_q, seg_k, q_off, k_off,
                      B, Nq, Nk, H, false, rope_layout == LWM_ROPE_HALF, out,
                      lse, w, st);

@@ -62,8 +62,8 @@ _SIGS = {
                                        _vp, _vp]),
     "lwm_blockattn_fwd_block_workspace_size": (_sz, [_i] * 6),
     "lwm_blockattn_fwd_block": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i,
-                                     _d, _i, _i, _i, _i, _i, _i, _i, _vp,
-                                     _vp, _vp, _sz, _vp]),
+                                     _d, _i, _vp, _i, _i, _i, _i, _i, _i,
+                                     _vp, _vp, _vp, _sz, _vp]),
     "lwm_blockattn_merge": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                  _vp]),
     "lwm_blockattn_bwd_delta": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp,
@@ -265,14 +265,16 @@ def fwd_block_workspace_size(B, Nq, Nk, H, max_pos, D=HEAD_DIM) -> int:
 
 def fwd_block(q, k_rot, v, seg_q, pos_q, seg_k, q_off, k_off, theta,
               max_pos, out=None, lse=None, workspace=None, stream=None,
-              rope_layout="interleaved"):
+              rope_layout="interleaved", table=None):
     """Partial forward of query rows [q_off, q_off+Nq) against the rotated
     key / value rows [k_off, k_off+Nk) of the same packed sequence (one step
     of a ring). Returns (out [B,Nq,H,D] bf16, lse [B,H,Nq] fp32); rows that
     see no key get (0, -inf)."""
-    _need_cuda(q, k_rot, v, seg_q, pos_q, seg_k, out, lse, workspace)
+    _need_cuda(q, k_rot, v, seg_q, pos_q, seg_k, out, lse, workspace, table)
     B, Nq, H, D = q.shape
     Nk = k_rot.shape[1]
+    if table is not None and table.shape[0] < max_pos:
+        raise ValueError("rope table shorter than max_pos")
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
@@ -281,9 +283,9 @@ def fwd_block(q, k_rot, v, seg_q, pos_q, seg_k, q_off, k_off, theta,
                     q.device, workspace)
     st = lib().lwm_blockattn_fwd_block(
         _ptr(q), _ptr(k_rot), _ptr(v), _ptr(seg_q), _ptr(pos_q), _ptr(seg_k),
-        int(q_off), int(k_off), float(theta), int(max_pos), B, Nq, Nk, H, D,
-        _layout_code(rope_layout), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
-        _stream(stream))
+        int(q_off), int(k_off), float(theta), int(max_pos), _ptr(table), B,
+        Nq, Nk, H, D, _layout_code(rope_layout), _ptr(out), _ptr(lse),
+        _ptr(ws), ws.numel(), _stream(stream))
     _check(st, "lwm_blockattn_fwd_block")
     return out, lse
 

@@ -132,17 +132,17 @@ def test_ring_and_layout_entry_points_reject_bad_arguments():
     p = v(1 << 20)
     big = 1 << 40
     # fwd_block: null q, unknown layout, misaligned seg_k
-    assert L.lwm_blockattn_fwd_block(None, p, p, p, p, p, 0, 0, 1e4, 16, 1, 16,
-                                     16, 1, 128, 0, p, p, p, big,
+    assert L.lwm_blockattn_fwd_block(None, p, p, p, p, p, 0, 0, 1e4, 16, None, 1,
+                                     16, 16, 1, 128, 0, p, p, p, big,
                                      None) == ops.ERR_INVALID_ARG
-    assert L.lwm_blockattn_fwd_block(p, p, p, p, p, p, 0, 0, 1e4, 16, 1, 16,
+    assert L.lwm_blockattn_fwd_block(p, p, p, p, p, p, 0, 0, 1e4, 16, None, 1, 16,
                                      16, 1, 128, 9, p, p, p, big,
                                      None) == ops.ERR_INVALID_ARG
     assert L.lwm_blockattn_fwd_block(p, p, p, p, p, v((1 << 20) + 4), 0, 0,
-                                     1e4, 16, 1, 16, 16, 1, 128, 0, p, p, p,
-                                     big, None) == ops.ERR_INVALID_ARG
-    assert L.lwm_blockattn_fwd_block(p, p, p, p, p, p, -1, 0, 1e4, 16, 1, 16,
-                                     16, 1, 128, 0, p, p, p, big,
+                                     1e4, 16, None, 1, 16, 16, 1, 128, 0, p,
+                                     p, p, big, None) == ops.ERR_INVALID_ARG
+    assert L.lwm_blockattn_fwd_block(p, p, p, p, p, p, -1, 0, 1e4, 16, None, 1,
+                                     16, 16, 1, 128, 0, p, p, p, big,
                                      None) == ops.ERR_INVALID_ARG
     # bwd_block: null accumulator; D != 128
     assert L.lwm_blockattn_bwd_block(p, p, p, p, p, p, p, p, 0, 0, 1, 16, 16,
@@ -167,8 +167,8 @@ def test_ring_and_layout_entry_points_reject_bad_arguments():
                                   None) == ops.ERR_INVALID_ARG
     # empty problems launch nothing and succeed
     assert L.lwm_blockattn_fwd_block(None, None, None, None, None, None, 0, 0,
-                                     1e4, 16, 1, 0, 16, 1, 128, 0, None, None,
-                                     None, 0, None) == ops.OK
+                                     1e4, 16, None, 1, 0, 16, 1, 128, 0, None,
+                                     None, None, 0, None) == ops.OK
     assert L.lwm_blockattn_bwd_block(None, None, None, None, None, None, None,
                                      None, 0, 0, 1, 16, 0, 1, 128, None, None,
                                      None, None, 0, None) == ops.OK

@@ -340,3 +340,43 @@ def test_ring_of_one_backward_equals_full_backward(cuda_dev):
         scale = a.float().abs().max().item()
         err = (a.float() - b.float()).abs().max().item()
         assert err <= 2 ** -7 * scale, f"{name}: {err}"
+
+
+@pytest.mark.parametrize("P", [2, 4])
+def test_simulated_zigzag_ring_matches_dense_oracle(cuda_dev, P):
+    t = _with_dout(_case(1500, 2, 1, 31), 32)
+    mp = int(t["positions"].max()) + 1
+    be = ring.CudaBackend(t["theta"], mp)
+    out, lse = ring.simulate_ring_fwd(t["q"], t["k"], t["v"],
+                                      t["segment_ids"], t["positions"], P, be,
+                                      layout="zigzag")
+    dq, dk, dv = ring.simulate_ring_bwd(t["q"], t["k"], t["v"], out,
+                                        t["dout"], lse, t["segment_ids"],
+                                        t["positions"], P, be,
+                                        layout="zigzag")
+    torch.cuda.synchronize()
+    assert ops.last_status() == ops.OK
+    ref = oracle.attn_bwd(t["q"], t["k"], t["v"], t["dout"],
+                          t["segment_ids"], t["positions"], t["theta"])
+    assert np.abs(out.float().cpu().numpy() - ref["out"]).max() <= OUT_TOL
+    assert np.abs(lse.cpu().numpy() - ref["lse"]).max() <= LSE_TOL
+    for name, g in (("dq", dq), ("dk", dk), ("dv", dv)):
+        err = np.abs(g.float().cpu().numpy() - ref[name]).max()
+        assert err <= BWD_REL * np.abs(ref[name]).max(), f"{name}: {err}"
+
+
+def test_partial_with_caller_table_is_identical(cuda_dev):
+    # the ring passes one table to every step; the result must not change
+    t = _case(900, 2, 1, 33)
+    mp = int(t["positions"].max()) + 1
+    table = ops.rope_table(t["theta"], mp)
+    qs, ks = slice(450, 900), slice(0, 450)
+    c = lambda x, s: x[:, s].contiguous()
+    k_rot = ops.rope_apply(c(t["k"], ks), c(t["positions"], ks), table)
+    args = (c(t["q"], qs), k_rot, c(t["v"], ks), c(t["segment_ids"], qs),
+            c(t["positions"], qs), c(t["segment_ids"], ks), 450, 0,
+            t["theta"], mp)
+    o1, l1 = ops.fwd_block(*args)
+    o2, l2 = ops.fwd_block(*args, table=table)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)

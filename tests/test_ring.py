@@ -82,13 +82,72 @@ def test_simulated_ring_backward_with_oracle_steps_equals_dense(P):
         np.testing.assert_allclose(got.numpy(), ref[name], atol=1e-11)
 
 
+def test_zigzag_parts_cover_the_sequence_once():
+    for N, P in [(200, 3), (1 << 15, 8), (17, 4), (8, 4)]:
+        got = sorted(pt for r in range(P) for pt in ring.ring_parts(N, P, r,
+                                                                    "zigzag"))
+        off = 0
+        for o, n in got:
+            assert o == off
+            off += n
+        assert off == N
+        # rank r holds chunk r and its mirror 2P-1-r
+        for r in range(P):
+            (a, _), (b, _) = ring.ring_parts(N, P, r, "zigzag")
+            assert (a, b) == (ring.ring_chunk(N, 2 * P, r)[0],
+                              ring.ring_chunk(N, 2 * P, 2 * P - 1 - r)[0])
+
+
+def _causal_pairs(parts, N, P, layout):
+    """Visible (query, key) pairs of one causal sequence a rank computes."""
+    tot = 0
+    for q_off, nq in parts:
+        for src in range(P):
+            for k_off, nk in ring.ring_parts(N, P, src, layout):
+                for i in range(q_off, q_off + nq):
+                    tot += max(0, min(i, k_off + nk - 1) - k_off + 1)
+    return tot
+
+
+def test_zigzag_balances_the_causal_ring():
+    N, P = 512, 4
+    work = {lay: [_causal_pairs(ring.ring_parts(N, P, r, lay), N, P, lay)
+                  for r in range(P)] for lay in ring.LAYOUTS}
+    total = N * (N + 1) // 2
+    for lay in ring.LAYOUTS:
+        assert sum(work[lay]) == total
+    c, z = work["contiguous"], work["zigzag"]
+    assert max(c) / min(c) > 5          # the plain ring: last rank >> first
+    assert max(z) / min(z) < 1.01       # zigzag: equal shares
+
+
+@pytest.mark.parametrize("P", [1, 2, 3, 4])
+def test_simulated_zigzag_ring_with_oracle_steps_equals_dense(P):
+    t = _inputs(N=150, seed=9)
+    g = torch.Generator().manual_seed(4)
+    dout = torch.randn(t["q"].shape, generator=g, dtype=torch.float64)
+    ref = oracle.attn_bwd(t["q"], t["k"], t["v"], dout, t["segment_ids"],
+                          t["positions"], THETA)
+    be = OracleBackend(THETA)
+    ro, rl = ring.simulate_ring_fwd(t["q"], t["k"], t["v"], t["segment_ids"],
+                                    t["positions"], P, be, layout="zigzag")
+    np.testing.assert_allclose(ro.numpy(), ref["out"], atol=1e-12)
+    np.testing.assert_allclose(rl.numpy(), ref["lse"], atol=1e-12)
+    dq, dk, dv = ring.simulate_ring_bwd(
+        t["q"].double(), t["k"].double(), t["v"].double(),
+        torch.from_numpy(ref["out"]), dout, torch.from_numpy(ref["lse"]),
+        t["segment_ids"], t["positions"], P, be, layout="zigzag")
+    for got, name in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        np.testing.assert_allclose(got.numpy(), ref[name], atol=1e-11)
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
         return s.getsockname()[1]
 
 
-def _worker(rank, world, port, q):
+def _worker(rank, world, port, q, layout="contiguous"):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port),
                       WORLD_SIZE=str(world), RANK=str(rank),
                       LOCAL_RANK=str(rank))
@@ -96,44 +155,67 @@ def _worker(rank, world, port, q):
     ldist.init_from_env("gloo", timeout_s=60)
     t = _inputs()
     N = t["q"].shape[1]
-    off, n = ring.ring_chunk(N, world, rank)
-    sl = slice(off, off + n)
+    parts = ring.ring_parts(N, world, rank, layout)
+
+    def mine(x):  # this rank's tokens: its parts, concatenated
+        return torch.cat([x[:, o:o + n] for o, n in parts], dim=1)
+
+    def mine_h(x):  # the same along the last axis of [B, H, N]
+        return torch.cat([x[:, :, o:o + n] for o, n in parts], dim=2)
+
     out, lse = ring.ring_fwd(
-        t["q"][:, sl].contiguous(), t["k"][:, sl].contiguous(),
-        t["v"][:, sl].contiguous(), t["segment_ids"][:, sl].contiguous(),
-        t["positions"][:, sl].contiguous(), N, OracleBackend(THETA))
+        mine(t["q"]), mine(t["k"]), mine(t["v"]), mine(t["segment_ids"]),
+        mine(t["positions"]), N, OracleBackend(THETA), layout=layout)
     g = torch.Generator().manual_seed(3)
     dout = torch.randn(t["q"].shape, generator=g, dtype=torch.float64)
     grads = ring.ring_bwd(
-        t["q"][:, sl].double().contiguous(), t["k"][:, sl].double().contiguous(),
-        t["v"][:, sl].double().contiguous(), out, dout[:, sl].contiguous(),
-        lse, t["segment_ids"][:, sl].contiguous(),
-        t["positions"][:, sl].contiguous(), N, OracleBackend(THETA))
+        mine(t["q"]).double(), mine(t["k"]).double(), mine(t["v"]).double(),
+        out, mine(dout), lse, mine(t["segment_ids"]), mine(t["positions"]),
+        N, OracleBackend(THETA), layout=layout)
     outs = [None] * world
     torch.distributed.all_gather_object(
-        outs, (out.numpy(), lse.numpy()) + tuple(x.numpy() for x in grads))
+        outs, (parts, out.numpy(), lse.numpy())
+        + tuple(x.numpy() for x in grads))
     if rank == 0:
+        # put every rank's parts back in global order
+        def glob(i, axis):
+            full = None
+            for o in outs:
+                x, off = o[i], 0
+                for po, pn in o[0]:
+                    sl = [slice(None)] * x.ndim
+                    sl[axis] = slice(off, off + pn)
+                    if full is None:
+                        shape = list(x.shape)
+                        shape[axis] = N
+                        full = np.zeros(shape)
+                    fs = [slice(None)] * x.ndim
+                    fs[axis] = slice(po, po + pn)
+                    full[tuple(fs)] = x[tuple(sl)]
+                    off += pn
+            return full
+        outs = [(glob(1, 1), glob(2, 2), glob(3, 1), glob(4, 1), glob(5, 1))]
         ref = oracle.attn_bwd(t["q"], t["k"], t["v"], dout,
                               t["segment_ids"], t["positions"], THETA)
-        errs = [float(np.abs(np.concatenate([o[0] for o in outs], axis=1)
-                             - ref["out"]).max()),
-                float(np.abs(np.concatenate([o[1] for o in outs], axis=2)
-                             - ref["lse"]).max())]
+        o = outs[0]
+        errs = [float(np.abs(o[0] - ref["out"]).max()),
+                float(np.abs(o[1] - ref["lse"]).max())]
         for i, name in ((2, "dq"), (3, "dk"), (4, "dv")):
-            errs.append(float(np.abs(np.concatenate([o[i] for o in outs],
-                                                    axis=1)
-                                     - ref[name]).max()))
+            errs.append(float(np.abs(o[i] - ref[name]).max()))
         q.put(errs)
     torch.distributed.barrier()
     torch.distributed.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
-def test_ring_forward_and_backward_over_gloo_ranks_equals_dense(world):
+@pytest.mark.parametrize("world,layout", [(2, "contiguous"),
+                                          (3, "contiguous"), (2, "zigzag"),
+                                          (3, "zigzag")])
+def test_ring_forward_and_backward_over_gloo_ranks_equals_dense(world,
+                                                                layout):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, q))
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q, layout))
              for r in range(world)]
     for p in procs:
         p.start()
