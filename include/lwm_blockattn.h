@@ -268,6 +268,25 @@ LWM_API int lwm_blockffn_fwd(const void* x, const void* w_gate,
                              void* workspace, size_t workspace_bytes,
                              void* stream);
 
+/* Bytes of workspace lwm_blockffn_bwd needs: one chunk's bf16 dact, dh,
+ * dg and act, 4 x chunk x F x 2 bytes. */
+LWM_API size_t lwm_blockffn_bwd_workspace_size(int chunk, int F);
+
+/* Backward of lwm_blockffn_fwd, chunk by chunk with h and g recomputed:
+ *   dact = dy Wd, dh = dact * g * silu'(h), dg = dact * silu(h),
+ *   dx = dh Wg + dg Wu (bf16 [T][Dm], written),
+ *   dw_gate = sum_chunks dh^T x, dw_up = dg^T x ([F][Dm] fp32),
+ *   dw_down = dy^T act ([Dm][F] fp32), all three written (zeroed first).
+ * dy [T][Dm] bf16. dact, dh, dg and act are rounded to bf16 once; the
+ * products accumulate in fp32. Dm, F multiples of 64; bf16 only. Async on
+ * stream. */
+LWM_API int lwm_blockffn_bwd(const void* x, const void* w_gate,
+                             const void* w_up, const void* w_down,
+                             const void* dy, int T, int Dm, int F, int chunk,
+                             int dtype, void* dx, float* dw_gate,
+                             float* dw_up, float* dw_down, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
 /* Tile classifier (exported so it can be checked bit-exactly). For each
  * batch row b and query block t (Tq = ceil(N/block_q) blocks), key blocks
  * j (Tk = ceil(N/block_k)):

@@ -628,6 +628,57 @@ int lwm_blockffn_fwd(const void* x, const void* w_gate, const void* w_up,
   return LWM_OK;
 }
 
+size_t lwm_blockffn_bwd_workspace_size(int chunk, int F) {
+  if (chunk < 1 || F < 1) return 0;
+  // dact [c][F], dh|dg [c][2F], act [c][F], all bf16
+  return 3 * align_up(size_t(chunk) * F * 2) + align_up(size_t(chunk) * F * 2);
+}
+
+int lwm_blockffn_bwd(const void* x, const void* w_gate, const void* w_up,
+                     const void* w_down, const void* dy, int T, int Dm, int F,
+                     int chunk, int dtype, void* dx, float* dw_gate,
+                     float* dw_up, float* dw_down, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  if (T < 0 || Dm < 1 || F < 1 || chunk < 1) return LWM_ERR_INVALID_ARG;
+  if (dtype != LWM_DTYPE_BF16 || Dm % 64 != 0 || F % 64 != 0)
+    return LWM_ERR_UNSUPPORTED;
+  const void* ptrs[] = {w_gate, w_up, w_down, dw_gate, dw_up, dw_down};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return LWM_ERR_INVALID_ARG;
+  if (int64_t(T) * std::max(Dm, F) >= (int64_t(1) << 40))
+    return LWM_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the weight gradients are sums over every token: start from zero
+  LWM_TRY(cudaMemsetAsync(dw_gate, 0, size_t(F) * Dm * 4, st));
+  LWM_TRY(cudaMemsetAsync(dw_up, 0, size_t(F) * Dm * 4, st));
+  LWM_TRY(cudaMemsetAsync(dw_down, 0, size_t(F) * Dm * 4, st));
+  if (T == 0) return LWM_OK;
+  const void* ptrs2[] = {x, dy, dx, workspace};
+  for (const void* p : ptrs2)
+    if (!p || !aligned16(p)) return LWM_ERR_INVALID_ARG;
+  const int c = std::min(chunk, T);
+  if (workspace_bytes < lwm_blockffn_bwd_workspace_size(c, F))
+    return LWM_ERR_WORKSPACE;
+  int* status = status_word();
+  if (!status) return LWM_ERR_CUDA;
+  char* ws = static_cast<char*>(workspace);
+  const size_t one = align_up(size_t(c) * F * 2);
+  void* dact = ws;
+  void* dhg = ws + one;
+  void* act = ws + 3 * one;
+  const char* xb = static_cast<const char*>(x);
+  const char* dyb = static_cast<const char*>(dy);
+  char* dxb = static_cast<char*>(dx);
+  for (int t0 = 0; t0 < T; t0 += c) {
+    const int m = std::min(c, T - t0);
+    const size_t off = size_t(t0) * Dm * 2;
+    LWM_TRY(launch_mlp_bwd_chunk(xb + off, w_gate, w_up, w_down, dyb + off,
+                                 m, Dm, F, dact, dhg, act, dxb + off, dw_gate,
+                                 dw_up, dw_down, status, st));
+  }
+  return LWM_OK;
+}
+
 int lwm_blockattn_classify(const int32_t* segment_ids, int B, int N,
                            int block_q, int block_k, int32_t* kv_lo,
                            int32_t* kv_hi, uint8_t* tile_class,

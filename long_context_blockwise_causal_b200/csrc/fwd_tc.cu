@@ -829,10 +829,17 @@ bool make_bnhd_map(CUtensorMap* m, const void* base, int B, int N, int H) {
 // columns (128 bytes) x box_rows rows with the 128-byte swizzle.
 bool make_2d_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols,
                  int box_rows) {
+  return make_2d_map_strided(m, base, rows, cols, cols, box_rows);
+}
+
+// The same for a [rows][cols] window of a wider matrix (row stride ld
+// elements).
+bool make_2d_map_strided(CUtensorMap* m, const void* base, int64_t rows,
+                         int64_t cols, int64_t ld, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
-  cuuint64_t strides[1] = {cuuint64_t(cols) * 2};
+  cuuint64_t strides[1] = {cuuint64_t(ld) * 2};
   cuuint32_t box[2] = {64, cuuint32_t(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,

@@ -88,6 +88,8 @@ bool make_bnhd_f32_map(CUtensorMap* m, const void* base, int B, int N,
 // 128-byte swizzle (cols * 2 must be a multiple of 16 bytes).
 bool make_2d_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols,
                  int box_rows);
+bool make_2d_map_strided(CUtensorMap* m, const void* base, int64_t rows,
+                         int64_t cols, int64_t ld, int box_rows);
 int sm_count();
 cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t st);
 

@@ -77,6 +77,9 @@ _SIGS = {
     "lwm_blockffn_workspace_size": (_sz, [_i, _i]),
     "lwm_blockffn_fwd": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp,
                               _vp, _sz, _vp]),
+    "lwm_blockffn_bwd_workspace_size": (_sz, [_i, _i]),
+    "lwm_blockffn_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
+                              _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
 }
 
 
@@ -374,6 +377,34 @@ def ffn_fwd(x, w_gate, w_up, w_down, chunk=8192, y=None, workspace=None,
         _dtype_code(x), _ptr(y), _ptr(ws), ws.numel(), _stream(stream))
     _check(st, "lwm_blockffn_fwd")
     return y
+
+
+def ffn_bwd_workspace_size(chunk, F) -> int:
+    return int(lib().lwm_blockffn_bwd_workspace_size(chunk, F))
+
+
+def ffn_bwd(x, w_gate, w_up, w_down, dy, chunk=8192, dx=None, dw_gate=None,
+            dw_up=None, dw_down=None, workspace=None, stream=None):
+    """Backward of ffn_fwd: returns (dx bf16 [T, Dm], dWg, dWu fp32 [F, Dm],
+    dWd fp32 [Dm, F]); h and g are recomputed chunk by chunk."""
+    _need_cuda(x, w_gate, w_up, w_down, dy, dx, dw_gate, dw_up, dw_down,
+               workspace)
+    T, Dm = x.shape
+    F = w_gate.shape[0]
+    dev = x.device
+    dx = torch.empty_like(x) if dx is None else dx
+    f32 = dict(dtype=torch.float32, device=dev)
+    dw_gate = torch.empty((F, Dm), **f32) if dw_gate is None else dw_gate
+    dw_up = torch.empty((F, Dm), **f32) if dw_up is None else dw_up
+    dw_down = torch.empty((Dm, F), **f32) if dw_down is None else dw_down
+    c = max(1, min(int(chunk), T))
+    ws = _workspace(ffn_bwd_workspace_size(c, F), dev, workspace)
+    st = lib().lwm_blockffn_bwd(
+        _ptr(x), _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(dy), T, Dm, F,
+        int(chunk), _dtype_code(x), _ptr(dx), _ptr(dw_gate), _ptr(dw_up),
+        _ptr(dw_down), _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "lwm_blockffn_bwd")
+    return dx, dw_gate, dw_up, dw_down
 
 
 def classify(segment_ids, block_q=BLOCK, block_k=BLOCK, with_class=True,

@@ -54,7 +54,8 @@ from .ring import (  # noqa: F401
     attn_bwd_partial, ring_bwd,
 )
 from .ffn import (  # noqa: F401
-    silu, swiglu_intermediate, swiglu_mlp, blockwise_mlp,
+    silu, swiglu_intermediate, swiglu_mlp, blockwise_mlp, silu_grad,
+    swiglu_mlp_bwd,
 )
 from .classify import (  # noqa: F401
     classify_bruteforce, classify_count, TILE_EMPTY, TILE_PARTIAL, TILE_FULL,

@@ -42,3 +42,26 @@ def blockwise_mlp(x, w_gate, w_up, w_down, chunk):
     if not parts:
         return np.zeros((0, _f64(w_down).shape[0]))
     return np.concatenate(parts, axis=0)
+
+
+def silu_grad(h):
+    """d silu / dh = s (1 + h (1 - s)) with s the logistic sigmoid."""
+    h = np.asarray(h, dtype=np.float64)
+    s = 1.0 / (1.0 + np.exp(-h))
+    return s * (1.0 + h * (1.0 - s))
+
+
+def swiglu_mlp_bwd(x, w_gate, w_up, w_down, dy):
+    """Chain rule of swiglu_mlp. Returns dict with dx [T, Dm], dw_gate,
+    dw_up [F, Dm], dw_down [Dm, F] and the intermediates act, dact, dh, dg
+    [T, F]."""
+    x, wg, wu, wd, dy = (_f64(t) for t in (x, w_gate, w_up, w_down, dy))
+    h = x @ wg.T
+    g = x @ wu.T
+    act = silu(h) * g
+    dact = dy @ wd
+    dh = dact * g * silu_grad(h)
+    dg = dact * silu(h)
+    return {"dx": dh @ wg + dg @ wu, "dw_gate": dh.T @ x, "dw_up": dg.T @ x,
+            "dw_down": dy.T @ act, "act": act, "dact": dact, "dh": dh,
+            "dg": dg}

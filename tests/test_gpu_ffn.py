@@ -75,3 +75,99 @@ def test_ffn_llama_shape_sampled_rows(cuda_dev):
     rows = np.unique(np.r_[0, w.chunk - 1, w.chunk, w.T - 1,
                            rng.integers(0, w.T, 28)])
     _bound_check(y, {k: v for k, v in t.items()}, rows=rows)
+
+
+# ------------------------------------------------------------ backward
+
+def _bwd_inputs(T, Dm, F, seed, w_std=0.05):
+    t = wl.make_ffn_inputs(T, Dm, F, seed=seed, device="cuda", w_std=w_std)
+    g = torch.Generator(device="cuda").manual_seed(seed * 16 + 9)
+    t["dy"] = torch.randn((T, Dm), generator=g, device="cuda").to(torch.bfloat16)
+    return t
+
+
+def _host64(t):
+    return {k: v.float().cpu().numpy().astype(np.float64) for k, v in t.items()}
+
+
+def _check_bwd_full(t, got):
+    """Every element within twice the rounding bound of the bf16
+    intermediates: dact, dh, dg and act are rounded once (2^-9 relative),
+    and dh, dg also carry dact's rounding; dx is rounded once more."""
+    h = _host64(t)
+    ref = oracle.swiglu_mlp_bwd(h["x"], h["w_gate"], h["w_up"], h["w_down"],
+                                h["dy"])
+    A = np.abs
+    u = 2.0 ** -9
+    bounds = {
+        "dx": 2 * (u * A(ref["dx"]) + 2 * u * (A(ref["dh"]) @ A(h["w_gate"])
+                                              + A(ref["dg"]) @ A(h["w_up"]))),
+        "dw_gate": 2 * 2 * u * (A(ref["dh"]).T @ A(h["x"])),
+        "dw_up": 2 * 2 * u * (A(ref["dg"]).T @ A(h["x"])),
+        "dw_down": 2 * u * (A(h["dy"]).T @ A(ref["act"])),
+    }
+    for name, g in zip(("dx", "dw_gate", "dw_up", "dw_down"), got):
+        gg = g.float().cpu().numpy()
+        err = np.abs(gg - ref[name])
+        tol = bounds[name] + 1e-6
+        assert np.all(err <= tol), (name, float((err / tol).max()))
+
+
+@pytest.mark.parametrize("T,Dm,F,chunk", [(1000, 256, 640, 384),
+                                          (129, 128, 128, 8192),
+                                          (300, 192, 320, 64)])
+def test_ffn_backward_matches_oracle(cuda_dev, T, Dm, F, chunk):
+    t = _bwd_inputs(T, Dm, F, seed=4)
+    got = ops.ffn_bwd(t["x"], t["w_gate"], t["w_up"], t["w_down"], t["dy"],
+                      chunk=chunk)
+    torch.cuda.synchronize()
+    assert ops.last_status() == ops.OK
+    _check_bwd_full(t, got)
+
+
+def test_ffn_backward_chunking_changes_only_weight_sum_order(cuda_dev):
+    # dx rows depend on their own token only: identical bits for any chunk;
+    # the weight gradients are sums over chunks, equal up to fp32 order
+    t = _bwd_inputs(1100, 256, 384, seed=5)
+    a = ops.ffn_bwd(t["x"], t["w_gate"], t["w_up"], t["w_down"], t["dy"],
+                    chunk=256)
+    b = ops.ffn_bwd(t["x"], t["w_gate"], t["w_up"], t["w_down"], t["dy"],
+                    chunk=1100)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b[0])
+    for x, y in zip(a[1:], b[1:]):
+        assert (x - y).abs().max().item() <= 1e-5 * y.abs().max().item()
+
+
+def test_ffn_backward_llama_shape_sampled(cuda_dev):
+    # one 8192-token chunk of the Llama-2-7B MLP: dx on sampled rows, the
+    # weight gradients on sampled rows, each computed by the oracle over
+    # every token
+    w = wl.FFN_WORKLOADS["mlp8k"]
+    t = _bwd_inputs(w.T, w.Dm, w.F, seed=6, w_std=w.w_std)
+    dx, dwg, dwu, dwd = ops.ffn_bwd(t["x"], t["w_gate"], t["w_up"],
+                                    t["w_down"], t["dy"], chunk=w.chunk)
+    torch.cuda.synchronize()
+    assert ops.last_status() == ops.OK
+    h = _host64(t)
+    rng = np.random.default_rng(7)
+    rows = np.unique(np.r_[0, w.T - 1, rng.integers(0, w.T, 14)])
+    ref = oracle.swiglu_mlp_bwd(h["x"][rows], h["w_gate"], h["w_up"],
+                                h["w_down"], h["dy"][rows])
+    err = np.abs(dx.float().cpu().numpy()[rows] - ref["dx"])
+    assert err.max() <= 2 ** -6 * np.abs(ref["dx"]).max()
+    fr = np.unique(np.r_[0, w.F - 1, rng.integers(0, w.F, 6)])
+    dr = np.unique(np.r_[0, w.Dm - 1, rng.integers(0, w.Dm, 6)])
+    x, dy = h["x"], h["dy"]
+    hg = x @ h["w_gate"][fr].T          # [T, |fr|]
+    gg = x @ h["w_up"][fr].T
+    dact = dy @ h["w_down"][:, fr]
+    dh = dact * gg * oracle.silu_grad(hg)
+    dg = dact * oracle.silu(hg)
+    for got, ref_rows in ((dwg, dh.T @ x), (dwu, dg.T @ x)):
+        g_ = got.cpu().numpy()[fr]
+        assert np.abs(g_ - ref_rows).max() <= 2 ** -6 * np.abs(ref_rows).max()
+    act = oracle.swiglu_intermediate(x, h["w_gate"], h["w_up"])
+    ref_d = dy[:, dr].T @ act
+    g_ = dwd.cpu().numpy()[dr]
+    assert np.abs(g_ - ref_d).max() <= 2 ** -6 * np.abs(ref_d).max()
