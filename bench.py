@@ -307,8 +307,9 @@ def bench_decode(args):
     print(json.dumps(line), flush=True)
 
 
-FFN_METRIC = ("blockwise SwiGLU FFN TFLOP/s (3 projections, chunked over "
-              "tokens) at 1 B200; % of bf16 tensor peak")
+FFN_METRIC = ("blockwise SwiGLU FFN TFLOP/s, forward + backward (3 + 8 "
+              "products of T x Dm x F: the backward recomputes x Wg^T and "
+              "x Wu^T per chunk) at 1 B200; % of bf16 tensor peak")
 
 
 def ffn_oracle_sample(t_host, budget_s):
@@ -323,8 +324,10 @@ def ffn_oracle_sample(t_host, budget_s):
 
     def run(R):
         xs = x[:R].float().numpy().astype(np.float64)
+        dy = np.ones((R, Dm))
         t0 = time.perf_counter()
         oracle.swiglu_mlp(xs, w["w_gate"], w["w_up"], w["w_down"])
+        oracle.swiglu_mlp_bwd(xs, w["w_gate"], w["w_up"], w["w_down"], dy)
         return time.perf_counter() - t0
 
     R = 32
@@ -333,18 +336,20 @@ def ffn_oracle_sample(t_host, budget_s):
     dt = run(R)
     threads = max((i.get("num_threads", 1) for i in threadpool_info()),
                   default=1)
-    info = {"sample": f"oracle SwiGLU MLP (fp64 numpy) on the first {R} "
-                      f"tokens, full {Dm}x{F} weights; FLOP of those rows / "
-                      f"wall time",
+    info = {"sample": f"oracle SwiGLU MLP forward + backward (fp64 numpy) "
+                      f"on the first {R} tokens, full {Dm}x{F} weights; "
+                      f"FLOP of those rows (3 + 8 products) / wall time",
             "cores": int(threads), "host_cores": os.cpu_count(),
             "seconds": dt}
-    return wl.ffn_flops(R, Dm, F) / dt / 1e12, info
+    return wl.ffn_flops(R, Dm, F) // 3 * 11 / dt / 1e12, info
 
 
 def bench_ffn(args):
     """Blockwise FFN: three dense projections on the tensor cores."""
     w = wl.FFN_WORKLOADS[args.workload]
-    flop = wl.ffn_flops(w.T, w.Dm, w.F)
+    f_fwd = wl.ffn_flops(w.T, w.Dm, w.F)          # 3 products
+    f_bwd = f_fwd // 3 * 8                         # 8 products
+    flop = f_fwd + f_bwd
     cfg = {"workload": w.name, "T": w.T, "Dm": w.Dm, "F": w.F,
            "chunk": w.chunk, "weights": "N(0, 0.02^2) bf16",
            "l2": "inputs and weights larger than L2 (no flush)"}
@@ -378,39 +383,63 @@ def bench_ffn(args):
     t = wl.make_ffn_inputs(w.T, w.Dm, w.F, args.seed, device=dev,
                            w_std=w.w_std)
     y = torch.empty_like(t["x"])
+    g = torch.Generator(device=dev).manual_seed(args.seed * 16 + 9)
+    dy = torch.randn(t["x"].shape, generator=g, device=dev).to(torch.bfloat16)
     ws = torch.empty(ops.ffn_workspace_size(w.chunk, w.F), dtype=torch.uint8,
                      device=dev)
-    step = lambda: ops.ffn_fwd(t["x"], t["w_gate"], t["w_up"], t["w_down"],
-                               chunk=w.chunk, y=y, workspace=ws)
+    wsb = torch.empty(ops.ffn_bwd_workspace_size(w.chunk, w.F),
+                      dtype=torch.uint8, device=dev)
+    grads = (torch.empty_like(t["x"]),
+             torch.empty((w.F, w.Dm), dtype=torch.float32, device=dev),
+             torch.empty((w.F, w.Dm), dtype=torch.float32, device=dev),
+             torch.empty((w.Dm, w.F), dtype=torch.float32, device=dev))
+    fwd = lambda: ops.ffn_fwd(t["x"], t["w_gate"], t["w_up"], t["w_down"],
+                              chunk=w.chunk, y=y, workspace=ws)
+    bwd = lambda: ops.ffn_bwd(t["x"], t["w_gate"], t["w_up"], t["w_down"],
+                              dy, chunk=w.chunk, dx=grads[0],
+                              dw_gate=grads[1], dw_up=grads[2],
+                              dw_down=grads[3], workspace=wsb)
     for _ in range(args.warmup):
-        step()
+        fwd()
+        bwd()
     torch.cuda.synchronize()
     clocks = ClockSampler(dev)
     clocks.start()
     time.sleep(0.3)
     l0 = ops.kernel_launches()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    t_f = t_b = 0.0
     for _ in range(args.steps):
-        step()
-    e1.record()
-    torch.cuda.synchronize()
+        ev[0].record()
+        fwd()
+        ev[1].record()
+        bwd()
+        ev[2].record()
+        torch.cuda.synchronize()
+        t_f += ev[0].elapsed_time(ev[1])
+        t_b += ev[1].elapsed_time(ev[2])
     launches = ops.kernel_launches() - l0
     clk = clocks.stop()
-    ms = e0.elapsed_time(e1) / args.steps
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    ms = (t_f + t_b) / args.steps
+    ms_f, ms_b = t_f / args.steps, t_b / args.steps
     tflops = flop / (ms / 1e3) / 1e12
+    tf_b = f_bwd / (ms_b / 1e3) / 1e12
     pk = peaks()
     line = {"metric": FFN_METRIC, "value": tflops, "unit": "TFLOP/s",
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": cfg, "tokens_per_s": w.T / (ms / 1e3),
-            "roofline": {"bound": "tensor", "kernel": "mlp_gemm_kernel",
-                         "achieved": tflops, "peak": pk["bf16_tflops_sustained"],
+            "fwd": {"ms": ms_f, "tflops": f_fwd / (ms_f / 1e3) / 1e12},
+            "bwd": {"ms": ms_b, "tflops": tf_b},
+            "roofline": {"bound": "tensor",
+                         "kernel": "mlp_gemm_kernel (backward launches)",
+                         "achieved": tf_b, "peak": pk["bf16_tflops_sustained"],
                          "unit": "TFLOP/s",
-                         "frac": tflops / pk["bf16_tflops_sustained"],
-                         "frac_of_burst_peak": tflops / pk["bf16_tflops"],
+                         "frac": tf_b / pk["bf16_tflops_sustained"],
+                         "frac_of_burst_peak": tf_b / pk["bf16_tflops"],
                          "traffic": None,
                          "peak_kind": f"bf16 sustained ({pk['source']})"},
             "gpu_launches": int(launches), "device_status": ops.last_status(),
@@ -421,11 +450,20 @@ def bench_ffn(args):
         yh = torch.empty_like(xh).pin_memory()
         xd = torch.empty_like(t["x"])
 
+        dyh = dy.cpu().pin_memory()
+        dyd = torch.empty_like(dy)
+        dxh = torch.empty_like(xh).pin_memory()
+
         def e2e_step():
             xd.copy_(xh, non_blocking=True)
+            dyd.copy_(dyh, non_blocking=True)
             ops.ffn_fwd(xd, t["w_gate"], t["w_up"], t["w_down"],
                         chunk=w.chunk, y=y, workspace=ws)
+            ops.ffn_bwd(xd, t["w_gate"], t["w_up"], t["w_down"], dyd,
+                        chunk=w.chunk, dx=grads[0], dw_gate=grads[1],
+                        dw_up=grads[2], dw_down=grads[3], workspace=wsb)
             yh.copy_(y, non_blocking=True)
+            dxh.copy_(grads[0], non_blocking=True)
 
         for _ in range(2):
             e2e_step()
@@ -438,8 +476,10 @@ def bench_ffn(args):
         ems = e0.elapsed_time(e1) / args.steps
         nb = xh.numel() * xh.element_size()
         line["e2e"] = {"value": flop / (ems / 1e3) / 1e12, "unit": "TFLOP/s",
-                       "ms_per_step": ems, "h2d_bytes_per_step": nb,
-                       "d2h_bytes_per_step": nb}
+                       "ms_per_step": ems, "h2d_bytes_per_step": 2 * nb,
+                       "d2h_bytes_per_step": 2 * nb,
+                       "note": "x and dy in, y and dx out per step; weights "
+                               "and weight gradients stay on the device"}
     if not args.no_cpu_baseline:
         t_host = {k: v.cpu() for k, v in t.items()}
         tf, info = ffn_oracle_sample(t_host, args.cpu_budget)

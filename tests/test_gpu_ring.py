@@ -371,7 +371,9 @@ def test_partial_with_caller_table_is_identical(cuda_dev):
     mp = int(t["positions"].max()) + 1
     table = ops.rope_table(t["theta"], mp)
     qs, ks = slice(450, 900), slice(0, 450)
-    c = lambda x, s: x[:, s].contiguous()
+    # each piece in its own allocation (the library wants 16-byte aligned
+    # pointers, which slices of a B = 1 tensor need not be)
+    c = lambda x, s: x[:, s].clone(memory_format=torch.contiguous_format)
     k_rot = ops.rope_apply(c(t["k"], ks), c(t["positions"], ks), table)
     args = (c(t["q"], qs), k_rot, c(t["v"], ks), c(t["segment_ids"], qs),
             c(t["positions"], qs), c(t["segment_ids"], ks), 450, 0,
