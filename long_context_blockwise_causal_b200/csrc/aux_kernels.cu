@@ -499,40 +499,73 @@ __global__ void bwd_delta_kernel(const T* __restrict__ out,
   }
 }
 
-// dq = R(-pos) * dq_acc, rounded to T; one thread per (row, pair).
-template <typename T>
+// Four consecutive values of T from floats (one 8- or 16-byte store).
+__device__ __forceinline__ void store4(__nv_bfloat16* p, float a, float b,
+                                       float c, float d) {
+  *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(a, b),
+                                            pack_bf16x2(c, d));
+}
+__device__ __forceinline__ void store4(float* p, float a, float b, float c,
+                                       float d) {
+  *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
+}
+
+// dq = R(-pos) * dq_acc * scale, rounded to T (pos == nullptr: no
+// rotation). One thread per four RoPE pairs of a (b, n, h) row: pairs
+// 4u .. 4u+3, which are the values 8u .. 8u+7 in the interleaved layout and
+// 4u .. 4u+3 with 64+4u .. 64+4u+3 in the rotate-half layout.
+template <typename T, bool HALF>
 __global__ void dq_convert_kernel(const float* __restrict__ acc,
                                   const int32_t* __restrict__ pos,
-                                  const float2* __restrict__ table, int B,
-                                  int N, int H, float scale, bool half,
+                                  const float4* __restrict__ table, int B,
+                                  int N, int H, float scale,
                                   T* __restrict__ dq) {
-  int64_t total = int64_t(B) * N * H * (kHeadDim / 2);
+  constexpr int kQuads = kHeadDim / 8;  // groups of 4 pairs per row
+  const int64_t total = int64_t(B) * N * H * kQuads;
   for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
        e < total; e += int64_t(gridDim.x) * blockDim.x) {
-    int k = int(e % (kHeadDim / 2));   // pair index
-    int64_t bnh = e / (kHeadDim / 2);
-    int64_t bn = bnh / H;
-    // the pair's two elements: (2k, 2k+1) interleaved, (k, k+64) half
-    const int64_t i0 = bnh * kHeadDim + (half ? k : 2 * k);
-    const int64_t i1 = i0 + (half ? kHeadDim / 2 : 1);
-    float xa, xb;
-    if (half) {
-      xa = acc[i0] * scale;
-      xb = acc[i1] * scale;
+    const int u = int(e % kQuads);
+    const int64_t bnh = e / kQuads;
+    const int64_t row = bnh * kHeadDim;
+    // a[i], b[i]: the two elements of pair 4u + i
+    float a[4], b[4];
+    if (HALF) {
+      const float4 x = *reinterpret_cast<const float4*>(acc + row + 4 * u);
+      const float4 y = *reinterpret_cast<const float4*>(acc + row + 64 + 4 * u);
+      a[0] = x.x; a[1] = x.y; a[2] = x.z; a[3] = x.w;
+      b[0] = y.x; b[1] = y.y; b[2] = y.z; b[3] = y.w;
     } else {
-      const float2 x = reinterpret_cast<const float2*>(acc)[e];
-      xa = x.x * scale;
-      xb = x.y * scale;
+      const float4 x = *reinterpret_cast<const float4*>(acc + row + 8 * u);
+      const float4 y = *reinterpret_cast<const float4*>(acc + row + 8 * u + 4);
+      a[0] = x.x; b[0] = x.y; a[1] = x.z; b[1] = x.w;
+      a[2] = y.x; b[2] = y.y; a[3] = y.z; b[3] = y.w;
     }
-    if (!pos) {  // plain conversion
-      dq[i0] = T(xa);
-      dq[i1] = T(xb);
-      continue;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      a[i] *= scale;
+      b[i] *= scale;
     }
-    float2 cs = table[int64_t(pos[bn]) * (kHeadDim / 2) + k];
-    // inverse rotation: (a, b) -> (a c + b s, -a s + b c)
-    dq[i0] = T(xa * cs.x + xb * cs.y);
-    dq[i1] = T(xb * cs.x - xa * cs.y);
+    if (pos) {
+      // inverse rotation: (a, b) -> (a c + b s, -a s + b c)
+      const float4* t = table + int64_t(pos[bnh / H]) * (kHeadDim / 4) + 2 * u;
+      const float4 c01 = t[0], c23 = t[1];
+      const float cs[4] = {c01.x, c01.z, c23.x, c23.z};
+      const float sn[4] = {c01.y, c01.w, c23.y, c23.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float ra = a[i] * cs[i] + b[i] * sn[i];
+        const float rb = b[i] * cs[i] - a[i] * sn[i];
+        a[i] = ra;
+        b[i] = rb;
+      }
+    }
+    if (HALF) {
+      store4(dq + row + 4 * u, a[0], a[1], a[2], a[3]);
+      store4(dq + row + 64 + 4 * u, b[0], b[1], b[2], b[3]);
+    } else {
+      store4(dq + row + 8 * u, a[0], b[0], a[1], b[1]);
+      store4(dq + row + 8 * u + 4, a[2], b[2], a[3], b[3]);
+    }
   }
 }
 
@@ -731,11 +764,15 @@ template <typename T>
 cudaError_t launch_dq_convert(const float* acc, const int32_t* pos,
                               const float* table, int B, int N, int H,
                               float scale, bool half, T* dq, cudaStream_t st) {
-  int64_t n = int64_t(B) * N * H * (kHeadDim / 2);
+  const int64_t n = int64_t(B) * N * H * (kHeadDim / 8);
   if (n == 0) return cudaSuccess;
-  dq_convert_kernel<T><<<grid_for(n, 256, 148 * 32), 256, 0, st>>>(
-      acc, pos, reinterpret_cast<const float2*>(table), B, N, H, scale, half,
-      dq);
+  const float4* t4 = reinterpret_cast<const float4*>(table);
+  if (half)
+    dq_convert_kernel<T, true><<<grid_for(n, 256, 148 * 32), 256, 0, st>>>(
+        acc, pos, t4, B, N, H, scale, dq);
+  else
+    dq_convert_kernel<T, false><<<grid_for(n, 256, 148 * 32), 256, 0, st>>>(
+        acc, pos, t4, B, N, H, scale, dq);
   note_launch();
   return cudaGetLastError();
 }
