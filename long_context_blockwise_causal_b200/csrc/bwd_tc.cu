@@ -48,7 +48,7 @@ constexpr int kSK = 0, kSV = kTile, kSQ = 2 * kTile, kSDO = 4 * kTile,
               kSBars = kSAux + 4 * 128 * 4;
 enum {
   bKVFull = 0, bKVEmpty, bQFull0, bQFull1, bQEmpty0, bQEmpty1, bAux0, bAux1,
-  bStFull, bDptFull, bPFull, bDqFull, bDqEmpty, bAccFull, bAccEmpty, bDoneB, bDsFree,
+  bStFull, bDptFull, bPFull, bDqFull, bDqEmpty, bAccFull, bAccEmpty, bDoneB,
   bItemFull0, bItemFull1, bItemEmpty0, bItemEmpty1, kNumBarsB
 };
 constexpr int kSMisc = kSBars + kNumBarsB * 8;
@@ -95,13 +95,6 @@ __device__ __forceinline__ BItem get_bitem(const BwdParams& p, int it) {
   m.qlo = p.q_lo[unit];
   m.qhi = p.q_hi[unit];
   return m;
-}
-
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b,
-                                           float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr),
-               "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
 }
 
 __global__ void __launch_bounds__(kThreadsBwd, 1)
