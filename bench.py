@@ -44,6 +44,18 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
                   "bf16_tflops_sustained": 1400.0}
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or None
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -592,6 +604,11 @@ def main():
                            with_dout=w.backward)
     B, N, H, D = t["q"].shape
     pairs_per_head = wl.visible_pairs(t["lengths"])
+    # tile pairs the kernels execute (key blocks in each query block's
+    # [kv_lo, kv_hi], 128 x 128 pairs each) over the visible pairs
+    lo_, hi_, _ = ops.classify(t["segment_ids"], with_class=False)
+    executed_ratio = float(((hi_ - lo_ + 1).clamp(min=0).sum().item())
+                           * 128 * 128 / max(1, pairs_per_head))
     fwd_flop = 4.0 * D * pairs_per_head * H
     bwd_flop = 10.0 * D * pairs_per_head * H if w.backward else 0.0
     strong = args.shard == "heads" and ws > 1
@@ -718,7 +735,12 @@ def main():
         tf, info = oracle_sample(w, t_host, args.cpu_budget, w.backward)
         cpu = {"value": tf, "unit": "TFLOP/s", "cores": info["cores"],
                "kind": "oracle", "sample": info["sample"],
-               "seconds": info["seconds"], "host_cores": info["host_cores"]}
+               "seconds": info["seconds"], "host_cores": info["host_cores"],
+               "cpu_model": cpu_model(),
+               "extrapolated_full_step_s":
+                   (fwd_flop + bwd_flop) / (tf * 1e12) if tf > 0 else None,
+               "extrapolated_note": "extrapolated: the whole step's "
+                                    "mask-aware FLOP at the sampled rate"}
 
     if rank == 0:
         pk = peaks()
@@ -741,6 +763,7 @@ def main():
                        "theta": w.theta, "qk_precision": qkp,
                        "segments": w.segments,
                        "visible_pairs_per_head": pairs_per_head,
+                       "executed_tile_pairs_over_visible": executed_ratio,
                        "l2": "inputs larger than L2 (no flush)"
                        if 3 * t["q"].numel() * 2 > 126e6 else
                        "inputs smaller than L2 (re-read from L2)",
