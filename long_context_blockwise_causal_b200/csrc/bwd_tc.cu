@@ -21,9 +21,10 @@
 // (dK~ / sqrt(D)) in the epilogue, dQ the same in the conversion kernel.
 //
 // Warps: 0-7 compute (thread = key row = TMEM lane; warps w and w + 4
-// share the lanes and split the 128 columns), 8-11 dQ reduction and
-// per-block (lse, D) staging, 12 TMA producer, 13 tcgen05 issuer + TMEM
-// owner, 14-15 idle (complete the warpgroup for setmaxnreg).
+// share the lanes and split the 128 columns; they also move each block's
+// dQ out of TMEM into shared memory right after its MMA), 8-11 dQ
+// reduce-add and per-block (lse, D) staging, 12 TMA producer, 13 tcgen05
+// issuer + TMEM owner, 14-15 idle (complete the warpgroup for setmaxnreg).
 #include <cuda.h>
 
 #include "aux_kernels.cuh"
@@ -49,7 +50,7 @@ constexpr int kSK = 0, kSV = kTile, kSQ = 2 * kTile, kSDO = 4 * kTile,
 enum {
   bKVFull = 0, bKVEmpty, bQFull0, bQFull1, bQEmpty0, bQEmpty1, bAux0, bAux1,
   bStFull, bDptFull, bPFull, bDqFull, bDqEmpty, bAccFull, bAccEmpty, bDoneB,
-  bItemFull0, bItemFull1, bItemEmpty0, bItemEmpty1, kNumBarsB
+  bItemFull0, bItemFull1, bItemEmpty0, bItemEmpty1, bDqStaged, kNumBarsB
 };
 constexpr int kSMisc = kSBars + kNumBarsB * 8;
 constexpr int kSmemBwd = kSMisc + 16;   // tmem addr, abort, 2 work slots
@@ -134,7 +135,9 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(bar(bDptFull), 1);
     mbar_init(bar(bPFull), 8);
     mbar_init(bar(bDqFull), 1);
-    mbar_init(bar(bDqEmpty), 4);
+    // the compute warps drain dQ from TMEM into the stage buffers
+    mbar_init(bar(bDqEmpty), 8);
+    mbar_init(bar(bDqStaged), 8);
     mbar_init(bar(bAccFull), 1);
     mbar_init(bar(bAccEmpty), 8);
     mbar_init(bar(bDoneB), 1);
@@ -299,6 +302,40 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(bPFull));
+        // dQ~ of this block: once its MMA is done (it follows dV and dK),
+        // this warp moves its 64 d columns out of TMEM (then TMEM is free
+        // for the next dP^T) into the block's own Q~ / dO stage buffers,
+        // which its MMAs no longer read, as two 32-column 4 KB boxes
+        // (128-byte swizzle) of its 32 rows; the dQ warps reduce-add them
+        ok = mbar_wait(bar(bDqFull), g & 1, abort_flag, p.status, kWaitNs);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        {
+          uint32_t dqv[2][32];
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc)
+            tmem_ld32(tB + lane_off + ch * 64 + cc * 32, dqv[cc]);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(bDqEmpty));
+          const int qoff = kSQ + st * kTile, ooff = kSDO + st * kTile;
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            const int c = 2 * ch + cc;  // 32-column chunk of d
+            const int box = (c < 2 ? qoff : ooff) + (q4 * 2 + (c & 1)) * 4096;
+            uint8_t* rowp = smem + box + lane * 128;
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              *reinterpret_cast<uint4*>(rowp + ((e ^ (lane & 7)) << 4)) =
+                  make_uint4(dqv[cc][4 * e], dqv[cc][4 * e + 1],
+                             dqv[cc][4 * e + 2], dqv[cc][4 * e + 3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(bDqStaged));
+        }
         ++g;
       }
       if (!ok) break;
@@ -438,52 +475,24 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   } else if (warp < 12) {
     // ---------------------------------------------------- dQ + staging
     regs_dec<kRegsDq>();
-    const int r = (warp - 8) * 32 + lane;  // query row = TMEM lane
-    const uint32_t lane_off = uint32_t((warp - 8) * 32) << 16;
+    const int r = (warp - 8) * 32 + lane;  // query row of the block
     int g = 0;
     bool ok = true;
     int pb = 0, ph = 0, pq0 = 0;  // the block whose dQ is pending
-    // dQ of block t: TMEM -> registers (then TMEM is free for the next
-    // dP^T), registers -> the block's own Q~ and dO stage buffers, which
-    // its MMAs no longer read (this warp's 32 rows as four 32-column 4 KB
-    // boxes, 128-byte swizzle), then a TMA reduce-add of each box into the
-    // fp32 accumulator; the stage goes back to the producer after the
-    // reduce has read it.
+    // dQ of block t, staged by the compute warps in the block's own Q~ and
+    // dO stage buffers (this warp's 32 rows as four 32-column 4 KB boxes,
+    // 128-byte swizzle): a TMA reduce-add of each box into the fp32
+    // accumulator; the stage goes back to the producer after the reduce
+    // has read it.
     const int wq = warp - 8;
     int pst = 0;  // stage of the pending block
     auto flush = [&](int t) -> bool {
-      bool w = mbar_wait(bar(bDqFull), t & 1, abort_flag, p.status, kWaitNs);
+      // the compute warps have staged dQ of block t in its stage buffers
+      bool w = mbar_wait(bar(bDqStaged), t & 1, abort_flag, p.status,
+                         kWaitNs);
       w = __all_sync(0xffffffffu, w);
       if (!w) return false;
-      tc_fence_after();
       const int qoff = kSQ + pst * kTile, ooff = kSDO + pst * kTile;
-      // two 32-column chunks at a time (64 registers); TMEM is released
-      // once the last chunk is in registers
-#pragma unroll
-      for (int c2 = 0; c2 < 4; c2 += 2) {
-        uint32_t v[2][32];
-        tmem_ld32(tB + lane_off + c2 * 32, v[0]);
-        tmem_ld32(tB + lane_off + (c2 + 1) * 32, v[1]);
-        tmem_wait_ld();
-        if (c2 == 2) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(bDqEmpty));
-        }
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int c = c2 + cc;
-          const int box = (c < 2 ? qoff : ooff) + (wq * 2 + (c & 1)) * 4096;
-          uint8_t* rowp = smem + box + lane * 128;
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            *reinterpret_cast<uint4*>(rowp + ((e ^ (lane & 7)) << 4)) =
-                make_uint4(v[cc][4 * e], v[cc][4 * e + 1], v[cc][4 * e + 2],
-                           v[cc][4 * e + 3]);
-        }
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
       if (lane == 0) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
