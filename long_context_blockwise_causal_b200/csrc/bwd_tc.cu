@@ -50,7 +50,8 @@ constexpr int kSK = 0, kSV = kTile, kSQ = 2 * kTile, kSDO = 4 * kTile,
 enum {
   bKVFull = 0, bKVEmpty, bQFull0, bQFull1, bQEmpty0, bQEmpty1, bAux0, bAux1,
   bStFull, bDptFull, bPFull, bDqFull, bDqEmpty, bAccFull, bAccEmpty, bDoneB,
-  bItemFull0, bItemFull1, bItemEmpty0, bItemEmpty1, bDqStaged, kNumBarsB
+  bItemFull0, bItemFull1, bItemEmpty0, bItemEmpty1, bDqStaged, bDsFull,
+  kNumBarsB
 };
 constexpr int kSMisc = kSBars + kNumBarsB * 8;
 constexpr int kSmemBwd = kSMisc + 16;   // tmem addr, abort, 2 work slots
@@ -134,6 +135,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(bar(bStFull), 1);
     mbar_init(bar(bDptFull), 1);
     mbar_init(bar(bPFull), 8);
+    mbar_init(bar(bDsFull), 8);
     mbar_init(bar(bDqFull), 1);
     // the compute warps drain dQ from TMEM into the stage buffers
     mbar_init(bar(bDqEmpty), 8);
@@ -217,7 +219,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         // its own range, so the other half's loads are never overwritten)
         const uint32_t colA = tA + lane_off + ch * 64;
         const uint32_t colB = tB + lane_off + ch * 64;
-        // phase 1 (while dP^T is still on the tensor pipe):
+        // phase 1 (while dP^T is still on the tensor pipe; its end lets dV
+        // start while phase 2 runs):
         // P^T = 2^(S^T c - lse log2 e), masked; bf16 copy over S^T
         float pf[2][32];
         {
@@ -259,6 +262,11 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             tmem_st16(colA + cc * 16, pp);
           }
         }
+        // P^T is in TMEM: dV runs on the tensor pipe while dS is formed
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(bPFull));
         // phase 2: dS^T = P^T (dP^T - D) once dP^T has landed
         ok = mbar_wait(bar(bDptFull), g & 1, abort_flag, p.status, kWaitNs);
         ok = __all_sync(0xffffffffu, ok);
@@ -301,7 +309,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(bPFull));
+        if (lane == 0) mbar_arrive(bar(bDsFull));
         // dQ~ of this block: once its MMA is done (it follows dV and dK),
         // this warp moves its 64 d columns out of TMEM (then TMEM is free
         // for the next dP^T) into the block's own Q~ / dO stage buffers,
@@ -658,6 +666,9 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             mma_ts(tC, tA + 8 * k + (k >= 4 ? 32 : 0),
                    sdesc_sw128(ob + 2048 * k, kHalf, 1024), idKM,
                    (!first_q || k > 0) ? 1u : 0u);
+          ok = mbar_wait(bar(bDsFull), g & 1, abort_flag, p.status, kWaitNs);
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll
           for (int k = 0; k < 8; ++k)  // dK~ += dS^T Q~
             mma_ts(tD, tB + 8 * k + (k >= 4 ? 32 : 0),
