@@ -299,10 +299,82 @@ DECODE_WORKLOADS = {
 }
 
 
+DECODE_METRIC = ("decode attention HBM GB/s (1 query token per row and "
+                 "head against the cache)")
+
+
+def decode_oracle_sample(cfg, seed, budget_s):
+    """Time the fp64 oracle on one decode query (batch row 0, head 0) against
+    a prefix of the cache, sized so one run takes about budget_s. The
+    metric counts the key and value rows read, as on the device. Returns
+    (GB/s, info)."""
+    import oracle
+    from threadpoolctl import threadpool_info
+    D = 128
+
+    def run(L):
+        scale = 1.0 / math.sqrt(D)
+        k = wl.random_tensor((1, L, 1, D), seed * 16 + 2, scale,
+                             torch.bfloat16, "cpu")
+        v = wl.random_tensor((1, L, 1, D), seed * 16 + 3, scale,
+                             torch.bfloat16, "cpu")
+        # only the last row is the query; the others are never read
+        q = wl.random_tensor((1, 1, 1, D), seed * 16 + 1, scale,
+                             torch.bfloat16, "cpu").expand(1, L, 1, D)
+        seg = torch.zeros((1, L), dtype=torch.int32)
+        pos = torch.arange(L, dtype=torch.int32)[None]
+        t0 = time.perf_counter()
+        oracle.attn_fwd_rows(q, k, v, seg, pos, cfg["theta"], 0, 0, [L - 1])
+        return time.perf_counter() - t0
+
+    L = min(1 << 15, cfg["L"])
+    dt = run(L)
+    L = int(min(cfg["L"], max(4096, (L * max(budget_s, 0.05) / max(dt, 1e-4))
+                              // 4096 * 4096)))
+    dt = run(L)
+    threads = max((i.get("num_threads", 1) for i in threadpool_info()),
+                  default=1)
+    info = {"sample": f"oracle decode (fp64) of batch row 0, head 0 against "
+                      f"the first {L} cached keys; key and value bytes read "
+                      f"/ wall time",
+            "cores": int(threads), "host_cores": os.cpu_count(),
+            "seconds": dt}
+    return L * D * 2 * 2 / dt / 1e9, info
+
+
+def decode_reference(args):
+    """The oracle's decode as the reference arm (rank 0, host cores)."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    cfg = DECODE_WORKLOADS[args.workload]
+    vals, secs, info = [], [], None
+    for i in range(args.warmup + args.steps):
+        gbs, info = decode_oracle_sample(cfg, args.seed, args.ref_budget)
+        if i >= args.warmup:
+            vals.append(gbs)
+            secs.append(info["seconds"])
+    value = float(np.mean(vals))
+    print(json.dumps({
+        "impl": "reference", "metric": DECODE_METRIC, "value": value,
+        "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": float(np.mean(secs)) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "B": cfg["B"], "L": cfg["L"],
+                   "H": cfg["H"], "D": 128},
+        "cpu_baseline": {"kind": "oracle", "value": value, "unit": "GB/s",
+                         "cores": info["cores"], "sample": info["sample"]},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0}}), flush=True)
+
+
 def bench_decode(args):
     """Decode attention: HBM-bound (every visible key and value row is read
     once). Prints one JSON line with GB/s against the measured copy
     bandwidth."""
+    if args.impl == "reference":
+        decode_reference(args)
+        return
     from long_context_blockwise_causal_b200 import ops
     cfg = DECODE_WORKLOADS[args.workload]
     B, L, H, D = cfg["B"], cfg["L"], cfg["H"], 128
@@ -347,8 +419,7 @@ def bench_decode(args):
     nbytes = B * H * L * D * 2 * 2 + B * H * D * 4  # K, V rows + q, out
     gbs = nbytes / (ms / 1e3) / 1e9
     pk = peaks()
-    line = {"metric": "decode attention HBM GB/s (1 query token per row and "
-                      "head against the cache)",
+    line = {"metric": DECODE_METRIC,
             "value": gbs, "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak",
@@ -363,6 +434,44 @@ def bench_decode(args):
                          "peak_kind": f"copy bandwidth ({pk['source']})"},
             "gpu_launches": int(launches), "device_status": ops.last_status(),
             "clocks": clk}
+    if not args.no_e2e:
+        # through the public call with host buffers: each step's query
+        # tokens and their positions in, the outputs and lse out; the cache
+        # is serving state resident in HBM
+        qh = q.cpu().pin_memory()
+        ph = q_pos.cpu().pin_memory()
+        h_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory(),
+                 torch.empty(lse.shape, dtype=lse.dtype).pin_memory()]
+
+        def make_set():
+            # the workspace is used by the compute stream only: shared
+            return {"q": torch.empty_like(q), "q_pos": torch.empty_like(q_pos),
+                    "out": torch.empty_like(out),
+                    "lse": torch.empty_like(lse)}
+
+        def run(d):
+            ops.decode(d["q"], k_rot, v, kv_start, kv_len, d["q_pos"], table,
+                       out=d["out"], lse=d["lse"], workspace=ws)
+
+        h_in = {"q": qh, "q_pos": ph}
+        outs = lambda d: [d["out"], d["lse"]]
+        pipelined_e2e(dev, h_in, make_set, run, outs, h_out, 2)
+        ems = pipelined_e2e(dev, h_in, make_set, run, outs, h_out,
+                            max(2, args.steps))
+        nbytes_in = qh.numel() * qh.element_size() + ph.numel() * 4
+        nbytes_out = sum(x.numel() * x.element_size() for x in h_out)
+        line["e2e"] = {"value": nbytes / (ems / 1e3) / 1e9, "unit": "GB/s",
+                       "ms_per_step": ems, "h2d_bytes_per_step": nbytes_in,
+                       "d2h_bytes_per_step": nbytes_out,
+                       "note": "query tokens and positions in, out and lse "
+                               "back per step (copy streams overlapped with "
+                               "the neighbouring steps' compute); the "
+                               "rotated key cache and the values stay in "
+                               "HBM"}
+    if not args.no_cpu_baseline:
+        gbs_cpu, info = decode_oracle_sample(cfg, args.seed, args.cpu_budget)
+        line["cpu_baseline"] = {"value": gbs_cpu, "unit": "GB/s",
+                                "kind": "oracle", **info}
     print(json.dumps(line), flush=True)
 
 
@@ -570,8 +679,7 @@ def main():
     args.warmup = max(args.warmup, 3)
 
     if args.workload in DECODE_WORKLOADS:
-        if args.impl != "reference":
-            bench_decode(args)
+        bench_decode(args)
         return
     if args.workload in wl.FFN_WORKLOADS:
         bench_ffn(args)
