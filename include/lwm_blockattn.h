@@ -279,7 +279,8 @@ LWM_API size_t lwm_blockffn_bwd_workspace_size(int chunk, int F);
  *   dw_down = dy^T act ([Dm][F] fp32), all three written (zeroed first).
  * dy [T][Dm] bf16. dact, dh, dg and act are rounded to bf16 once; the
  * products accumulate in fp32. Dm, F multiples of 64; bf16 only. Async on
- * stream. */
+ * stream; every argument is checked before the first launch, so a rejected
+ * call writes nothing (T = 0 only zeroes the three weight gradients). */
 LWM_API int lwm_blockffn_bwd(const void* x, const void* w_gate,
                              const void* w_up, const void* w_down,
                              const void* dy, int T, int Dm, int F, int chunk,

@@ -647,20 +647,24 @@ int lwm_blockffn_bwd(const void* x, const void* w_gate, const void* w_up,
     if (!p || !aligned16(p)) return LWM_ERR_INVALID_ARG;
   if (int64_t(T) * std::max(Dm, F) >= (int64_t(1) << 40))
     return LWM_ERR_INVALID_ARG;
+  // every check before the first launch: a rejected call writes nothing
+  const int c = std::max(1, std::min(chunk, T));
+  int* status = nullptr;
+  if (T > 0) {
+    const void* ptrs2[] = {x, dy, dx, workspace};
+    for (const void* p : ptrs2)
+      if (!p || !aligned16(p)) return LWM_ERR_INVALID_ARG;
+    if (workspace_bytes < lwm_blockffn_bwd_workspace_size(c, F))
+      return LWM_ERR_WORKSPACE;
+    status = status_word();
+    if (!status) return LWM_ERR_CUDA;
+  }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // the weight gradients are sums over every token: start from zero
   LWM_TRY(cudaMemsetAsync(dw_gate, 0, size_t(F) * Dm * 4, st));
   LWM_TRY(cudaMemsetAsync(dw_up, 0, size_t(F) * Dm * 4, st));
   LWM_TRY(cudaMemsetAsync(dw_down, 0, size_t(F) * Dm * 4, st));
   if (T == 0) return LWM_OK;
-  const void* ptrs2[] = {x, dy, dx, workspace};
-  for (const void* p : ptrs2)
-    if (!p || !aligned16(p)) return LWM_ERR_INVALID_ARG;
-  const int c = std::min(chunk, T);
-  if (workspace_bytes < lwm_blockffn_bwd_workspace_size(c, F))
-    return LWM_ERR_WORKSPACE;
-  int* status = status_word();
-  if (!status) return LWM_ERR_CUDA;
   char* ws = static_cast<char*>(workspace);
   const size_t one = align_up(size_t(c) * F * 2);
   void* dact = ws;

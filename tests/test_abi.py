@@ -172,3 +172,41 @@ def test_ring_and_layout_entry_points_reject_bad_arguments():
     assert L.lwm_blockattn_bwd_block(None, None, None, None, None, None, None,
                                      None, 0, 0, 1, 16, 0, 1, 128, None, None,
                                      None, None, 0, None) == ops.OK
+
+
+def test_ffn_entry_points_reject_bad_arguments_before_any_launch():
+    L = ops.lib()
+    v = ctypes.c_void_p
+    p = v(1 << 20)
+    big = 1 << 40
+    T, Dm, F, c = 256, 128, 192, 128
+    # forward: null input, unsupported width / dtype, small workspace
+    assert L.lwm_blockffn_fwd(None, p, p, p, T, Dm, F, c, 0, p, p, big,
+                              None) == ops.ERR_INVALID_ARG
+    assert L.lwm_blockffn_fwd(p, p, p, p, T, 100, F, c, 0, p, p, big,
+                              None) == ops.ERR_UNSUPPORTED
+    assert L.lwm_blockffn_fwd(p, p, p, p, T, Dm, F, c, 1, p, p, big,
+                              None) == ops.ERR_UNSUPPORTED
+    assert L.lwm_blockffn_fwd(p, p, p, p, T, Dm, F, 0, 0, p, p, big,
+                              None) == ops.ERR_INVALID_ARG
+    need = L.lwm_blockffn_workspace_size(c, F)
+    assert need >= c * F * 2
+    assert L.lwm_blockffn_fwd(p, p, p, p, T, Dm, F, c, 0, p, p, need - 1,
+                              None) == ops.ERR_WORKSPACE
+    assert L.lwm_blockffn_fwd(None, None, None, None, 0, Dm, F, c, 0, None,
+                              None, 0, None) == ops.OK
+    # backward: every check happens before the weight gradients are zeroed,
+    # so these return their own code (a launch here, with no GPU, would
+    # turn into LWM_ERR_CUDA)
+    need_b = L.lwm_blockffn_bwd_workspace_size(c, F)
+    assert need_b >= 4 * c * F * 2
+    assert L.lwm_blockffn_bwd(p, p, p, p, p, T, Dm, F, c, 0, p, p, p, p, p,
+                              need_b - 1, None) == ops.ERR_WORKSPACE
+    assert L.lwm_blockffn_bwd(p, p, p, p, None, T, Dm, F, c, 0, p, p, p, p,
+                              p, big, None) == ops.ERR_INVALID_ARG
+    assert L.lwm_blockffn_bwd(p, p, p, p, p, T, Dm, F, c, 0, None, p, p, p,
+                              p, big, None) == ops.ERR_INVALID_ARG
+    assert L.lwm_blockffn_bwd(p, p, p, p, p, T, Dm, F, c, 0, p, None, p, p,
+                              p, big, None) == ops.ERR_INVALID_ARG
+    assert L.lwm_blockffn_bwd(p, p, p, p, p, T, Dm, 96, c, 0, p, p, p, p, p,
+                              big, None) == ops.ERR_UNSUPPORTED
