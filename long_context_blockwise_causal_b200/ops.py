@@ -157,6 +157,47 @@ def _layout_code(rope_layout) -> int:
     raise ValueError(f"rope_layout {rope_layout!r}")
 
 
+def _expect(where, name, t, shape, dtype=None):
+    """Shapes and dtypes are checked here, before any pointer reaches the
+    library: the C calls take sizes from q (or x) and trust every other
+    buffer to match them."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape) or (dtype is not None
+                                          and t.dtype != dtype):
+        raise LwmError(ERR_INVALID_ARG,
+                       f"{where}: {name} is {tuple(t.shape)} {t.dtype}, "
+                       f"expected {tuple(shape)}"
+                       + ("" if dtype is None else f" {dtype}"))
+
+
+def _expect_dims(where, name, t, dims):
+    if t.dim() != dims:
+        raise LwmError(ERR_INVALID_ARG,
+                       f"{where}: {name} must have {dims} dimensions")
+
+
+def _same_device(where, *ts):
+    devs = {t.device for t in ts if t is not None}
+    if len(devs) > 1:
+        raise LwmError(ERR_INVALID_ARG, f"{where}: tensors on {sorted(map(str, devs))}")
+
+
+def _check_attn(where, q, k, v, segment_ids, positions, lse=None,
+                like_q=()):
+    """q, k, v (and like_q) [B,N,H,D] of one dtype; ids and positions
+    [B,N] int32; lse [B,H,N] fp32."""
+    _expect_dims(where, "q", q, 4)
+    B, N, H, _ = q.shape
+    for name, t in (("k", k), ("v", v)) + tuple(like_q):
+        _expect(where, name, t, q.shape, q.dtype)
+    _expect(where, "segment_ids", segment_ids, (B, N), torch.int32)
+    _expect(where, "positions", positions, (B, N), torch.int32)
+    _expect(where, "lse", lse, (B, H, N), torch.float32)
+    _same_device(where, q, k, v, segment_ids, positions, lse,
+                 *(t for _, t in like_q))
+
+
 def _need_cuda(*ts):
     for t in ts:
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
@@ -193,6 +234,8 @@ def fwd(q, k, v, segment_ids, positions, theta, max_pos=None,
     """Forward pass. Returns (out [B,N,H,D] in q's dtype, lse [B,H,N] fp32).
     ``rope_layout``: "interleaved" pairs (2k, 2k+1) or "half" (k, k+D/2),
     the rotate-half layout of Hugging Face Llama checkpoints."""
+    _check_attn("fwd", q, k, v, segment_ids, positions, lse,
+                like_q=(("out", out),))
     _need_cuda(q, k, v, segment_ids, positions, out, lse, workspace)
     B, N, H, D = q.shape
     if max_pos is None:
@@ -219,6 +262,8 @@ def fwd_noalloc(q, k, v, segment_ids, positions, theta, max_pos,
     """Forward through lwm_blockattn_fwd_noalloc: the library's own fixed
     scratch array replaces the workspace (see the header for its limits).
     ``out``/``lse`` are allocated here only if the caller passes none."""
+    _check_attn("fwd_noalloc", q, k, v, segment_ids, positions, lse,
+                like_q=(("out", out),))
     _need_cuda(q, k, v, segment_ids, positions, out, lse)
     B, N, H, D = q.shape
     if out is None:
@@ -240,6 +285,9 @@ def bwd(q, k, v, out, dout, lse, segment_ids, positions, theta,
         rope_layout="interleaved"):
     """Backward pass. Returns (dq, dk, dv) in q's dtype (dq, dk in the
     layout q and k came in)."""
+    _check_attn("bwd", q, k, v, segment_ids, positions, lse,
+                like_q=(("out", out), ("dout", dout), ("dq", dq), ("dk", dk),
+                        ("dv", dv)))
     _need_cuda(q, k, v, out, dout, lse, segment_ids, positions, dq, dk, dv,
                workspace)
     B, N, H, D = q.shape
@@ -358,6 +406,24 @@ def grad_finish(acc, positions=None, table=None, out=None, stream=None,
     return out
 
 
+def _check_ffn(where, x, w_gate, w_up, w_down, like_x=(), grads=()):
+    """x (and like_x) [T, Dm]; Wg, Wu [F, Dm] and Wd [Dm, F] of x's dtype;
+    grads: (name, tensor, shape) in fp32."""
+    _expect_dims(where, "x", x, 2)
+    _expect_dims(where, "w_gate", w_gate, 2)
+    T, Dm = x.shape
+    F = w_gate.shape[0]
+    _expect(where, "w_gate", w_gate, (F, Dm), x.dtype)
+    _expect(where, "w_up", w_up, (F, Dm), x.dtype)
+    _expect(where, "w_down", w_down, (Dm, F), x.dtype)
+    for name, t in like_x:
+        _expect(where, name, t, (T, Dm), x.dtype)
+    for name, t, shape in grads:
+        _expect(where, name, t, shape, torch.float32)
+    _same_device(where, x, w_gate, w_up, w_down, *(t for _, t in like_x),
+                 *(t for _, t, _ in grads))
+
+
 def ffn_workspace_size(chunk, F) -> int:
     return int(lib().lwm_blockffn_workspace_size(chunk, F))
 
@@ -366,6 +432,7 @@ def ffn_fwd(x, w_gate, w_up, w_down, chunk=8192, y=None, workspace=None,
             stream=None):
     """Blockwise SwiGLU MLP: y = (silu(x Wg^T) * (x Wu^T)) Wd^T, `chunk`
     tokens at a time. x [T, Dm]; Wg, Wu [F, Dm]; Wd [Dm, F]; bf16."""
+    _check_ffn("ffn_fwd", x, w_gate, w_up, w_down, like_x=(("y", y),))
     _need_cuda(x, w_gate, w_up, w_down, y, workspace)
     T, Dm = x.shape
     F = w_gate.shape[0]
@@ -387,6 +454,15 @@ def ffn_bwd(x, w_gate, w_up, w_down, dy, chunk=8192, dx=None, dw_gate=None,
             dw_up=None, dw_down=None, workspace=None, stream=None):
     """Backward of ffn_fwd: returns (dx bf16 [T, Dm], dWg, dWu fp32 [F, Dm],
     dWd fp32 [Dm, F]); h and g are recomputed chunk by chunk."""
+    if x.dim() == 2 and w_gate.dim() == 2:
+        Fg, Dmx = w_gate.shape[0], x.shape[1]
+        _check_ffn("ffn_bwd", x, w_gate, w_up, w_down,
+                   like_x=(("dy", dy), ("dx", dx)),
+                   grads=(("dw_gate", dw_gate, (Fg, Dmx)),
+                          ("dw_up", dw_up, (Fg, Dmx)),
+                          ("dw_down", dw_down, (Dmx, Fg))))
+    else:
+        _check_ffn("ffn_bwd", x, w_gate, w_up, w_down)
     _need_cuda(x, w_gate, w_up, w_down, dy, dx, dw_gate, dw_up, dw_down,
                workspace)
     T, Dm = x.shape
@@ -457,6 +533,22 @@ def decode(q, k_rot, v, kv_start, kv_len, q_pos, table, out=None, lse=None,
            workspace=None, stream=None, rope_layout="interleaved"):
     """One query token per (b, h) [B,H,D] against a cache of rotated keys
     and values [B,L,H,D]; returns (out [B,H,D], lse [B,H])."""
+    _expect_dims("decode", "q", q, 3)
+    _expect_dims("decode", "k_rot", k_rot, 4)
+    _expect_dims("decode", "table", table, 3)
+    Bq, Hq, Dq = q.shape
+    kshape = (Bq, k_rot.shape[1], Hq, Dq)
+    _expect("decode", "k_rot", k_rot, kshape, q.dtype)
+    _expect("decode", "v", v, kshape, q.dtype)
+    for name, t in (("kv_start", kv_start), ("kv_len", kv_len),
+                    ("q_pos", q_pos)):
+        _expect("decode", name, t, (Bq,), torch.int32)
+    _expect("decode", "table", table, (table.shape[0], Dq // 2, 2),
+            torch.float32)
+    _expect("decode", "out", out, q.shape, q.dtype)
+    _expect("decode", "lse", lse, (Bq, Hq), torch.float32)
+    _same_device("decode", q, k_rot, v, kv_start, kv_len, q_pos, table, out,
+                 lse)
     _need_cuda(q, k_rot, v, kv_start, kv_len, q_pos, table, out, lse,
                workspace)
     B, H, D = q.shape

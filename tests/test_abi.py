@@ -210,3 +210,87 @@ def test_ffn_entry_points_reject_bad_arguments_before_any_launch():
                               p, big, None) == ops.ERR_INVALID_ARG
     assert L.lwm_blockffn_bwd(p, p, p, p, p, T, Dm, 96, c, 0, p, p, p, p, p,
                               big, None) == ops.ERR_UNSUPPORTED
+
+
+def _attn_cpu(B=1, N=8, H=2, D=128, dtype=torch.bfloat16):
+    q = torch.zeros(B, N, H, D, dtype=dtype)
+    seg = torch.zeros(B, N, dtype=torch.int32)
+    pos = torch.arange(N, dtype=torch.int32)[None].repeat(B, 1)
+    return q, q.clone(), q.clone(), seg, pos
+
+
+def _invalid(fn, *a, **kw):
+    with pytest.raises(ops.LwmError) as e:
+        fn(*a, **kw)
+    assert e.value.status == ops.ERR_INVALID_ARG
+    return str(e.value)
+
+
+def test_bindings_check_shapes_and_dtypes_before_the_library():
+    """The C calls take their sizes from q (or x) and trust every other
+    buffer; the bindings refuse mismatched tensors before any pointer is
+    passed (on CPU tensors the shape check fires before the device one)."""
+    q, k, v, seg, pos = _attn_cpu()
+    assert "k is" in _invalid(ops.fwd, q, k[:, :4], v, seg, pos, 1e4)
+    assert "v is" in _invalid(ops.fwd, q, k, v.float(), seg, pos, 1e4)
+    _invalid(ops.fwd, q, k, v, seg.long(), pos, 1e4)
+    _invalid(ops.fwd, q, k, v, seg, pos[:, :4], 1e4)
+    _invalid(ops.fwd, q[0], k, v, seg, pos, 1e4)
+    _invalid(ops.fwd, q, k, v, seg, pos, 1e4,
+             lse=torch.zeros(1, 8, 2))                 # [B,N,H]: transposed
+    _invalid(ops.fwd, q, k, v, seg, pos, 1e4, out=torch.zeros_like(q).float())
+    _invalid(ops.fwd_noalloc, q, k, v, seg, pos, 1e4, 8, out=q[:, :2])
+    lse = torch.zeros(1, 2, 8)
+    _invalid(ops.bwd, q, k, v, q, q.float(), lse, seg, pos, 1e4)   # dout
+    _invalid(ops.bwd, q, k, v, q, q, lse, seg, pos, 1e4, dk=q[:, :3])
+    # consistent shapes: only the device check is left
+    with pytest.raises(ValueError, match="CUDA"):
+        ops.fwd(q, k, v, seg, pos, 1e4)
+    with pytest.raises(ValueError, match="CUDA"):
+        ops.bwd(q, k, v, q, q, lse, seg, pos, 1e4)
+
+    T, Dm, F = 16, 64, 128
+    x = torch.zeros(T, Dm, dtype=torch.bfloat16)
+    wg = torch.zeros(F, Dm, dtype=torch.bfloat16)
+    wd = torch.zeros(Dm, F, dtype=torch.bfloat16)
+    _invalid(ops.ffn_fwd, x, wg, wg, wg)                 # w_down [F, Dm]
+    _invalid(ops.ffn_fwd, x, wg, wg[:, :32], wd)
+    _invalid(ops.ffn_fwd, x, wg, wg, wd, y=x[:8])
+    _invalid(ops.ffn_bwd, x, wg, wg, wd, x[:8])          # dy
+    _invalid(ops.ffn_bwd, x, wg, wg, wd, x, dw_gate=wg)  # bf16 gradient
+    _invalid(ops.ffn_bwd, x, wg, wg, wd, x,
+             dw_down=torch.zeros(F, Dm))                # transposed
+    with pytest.raises(ValueError, match="CUDA"):
+        ops.ffn_bwd(x, wg, wg, wd, x)
+
+    B, L, H = 2, 64, 2
+    qd = torch.zeros(B, H, 128, dtype=torch.bfloat16)
+    kc = torch.zeros(B, L, H, 128, dtype=torch.bfloat16)
+    i32 = torch.zeros(B, dtype=torch.int32)
+    table = torch.zeros(L, 64, 2)
+    _invalid(ops.decode, qd, kc, kc, i32, i32.long(), i32, table)
+    _invalid(ops.decode, qd, kc, kc[:, :, :1], i32, i32, i32, table)
+    _invalid(ops.decode, qd, kc, kc, i32, i32, i32, torch.zeros(L, 128))
+    _invalid(ops.decode, qd, kc, kc, i32, i32, i32, table.double())
+    _invalid(ops.decode, qd, kc, kc, i32, i32, i32, table,
+             lse=torch.zeros(B, H, 1))
+    with pytest.raises(ValueError, match="CUDA"):
+        ops.decode(qd, kc, kc, i32, i32, i32, table)
+
+
+def test_binding_checks_accept_the_workloads_tensors():
+    from long_context_blockwise_causal_b200 import workloads as wl
+    for name, w in wl.WORKLOADS.items():
+        t = wl.make_inputs(w, 0, device="cpu", N=min(w.N, 512), with_dout=True)
+        B, N, H, D = t["q"].shape
+        lse = torch.empty(B, H, N)
+        ops._check_attn("fwd", t["q"], t["k"], t["v"], t["segment_ids"],
+                        t["positions"], lse,
+                        like_q=(("out", torch.empty_like(t["q"])),
+                                ("dout", t["dout"])))
+    for name, w in wl.FFN_WORKLOADS.items():
+        t = wl.make_ffn_inputs(256, w.Dm, w.F, 0, device="cpu")
+        ops._check_ffn("ffn_bwd", t["x"], t["w_gate"], t["w_up"], t["w_down"],
+                       like_x=(("dy", t["x"]), ("dx", t["x"])),
+                       grads=(("dw_gate", torch.empty(w.F, w.Dm), (w.F, w.Dm)),
+                              ("dw_down", torch.empty(w.Dm, w.F), (w.Dm, w.F))))
