@@ -294,3 +294,25 @@ def test_binding_checks_accept_the_workloads_tensors():
                        like_x=(("dy", t["x"]), ("dx", t["x"])),
                        grads=(("dw_gate", torch.empty(w.F, w.Dm), (w.F, w.Dm)),
                               ("dw_down", torch.empty(w.Dm, w.F), (w.Dm, w.F))))
+
+
+def test_plain_c_client_links_and_runs(tmp_path):
+    """The boundary is a C ABI: a C99 program that includes only the header
+    and links only the library builds with -Werror and runs (no Python, no
+    torch; the calls it makes need no GPU)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    libdir = os.path.dirname(ops._LIB_PATH)
+    exe = tmp_path / "c_abi_client"
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror",
+                    "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c_abi_client.c"),
+                    "-o", str(exe), "-L", libdir, "-l:liblwm_blockattn.so",
+                    f"-Wl,-rpath,{libdir}"], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True,
+                       timeout=60)
+    assert r.returncode == 0, r.stderr
+    assert "c client ok" in r.stdout
