@@ -58,5 +58,6 @@ from .ffn import (  # noqa: F401
     swiglu_mlp_bwd,
 )
 from .classify import (  # noqa: F401
-    classify_bruteforce, classify_count, TILE_EMPTY, TILE_PARTIAL, TILE_FULL,
+    classify_bruteforce, classify_count, classify_cross, visible_key_ranges,
+    visible_query_ranges, TILE_EMPTY, TILE_PARTIAL, TILE_FULL,
 )

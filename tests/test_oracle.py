@@ -362,6 +362,102 @@ def test_ragged_tail_tile_is_never_full():
     assert cls[0, 1, 0] == oracle.TILE_FULL
 
 
+def test_cross_classification_of_the_whole_row_is_the_square_one():
+    L = wl.segment_lengths("uniform", 700, 5, lo=1, hi=250)
+    seg, _ = wl.segments_from_lengths(L)
+    seg = np.stack([seg, np.repeat(np.arange(3, dtype=np.int32),
+                                   [100, 300, 300])])
+    a = oracle.classify_bruteforce(seg, 128, 128)
+    c = oracle.classify_cross(seg, 0, 700, 0, 700, 128, 128)
+    for x, y in zip(a, c):
+        np.testing.assert_array_equal(x, y)
+
+
+@pytest.mark.parametrize("q_off,Nq,k_off,Nk", [(300, 500, 0, 300),
+                                               (256, 384, 256, 384),
+                                               (0, 200, 500, 300),
+                                               (130, 333, 7, 250)])
+def test_cross_classification_single_segment_closed_form(q_off, Nq, k_off,
+                                                         Nk):
+    # one causal segment: key c visible to row r iff c <= r
+    N = 1000
+    seg = np.zeros((1, N), np.int32)
+    lo, hi, cls = oracle.classify_cross(seg, q_off, Nq, k_off, Nk, 128, 128)
+    for t in range(-(-Nq // 128)):
+        r0, r1 = q_off + 128 * t, q_off + min(128 * (t + 1), Nq) - 1
+        for s in range(-(-Nk // 128)):
+            c0, c1 = k_off + 128 * s, k_off + min(128 * (s + 1), Nk) - 1
+            whole = (r1 - r0 == 127) and (c1 - c0 == 127)
+            want = (oracle.TILE_EMPTY if c0 > r1 else
+                    oracle.TILE_FULL if whole and c1 <= r0 else
+                    oracle.TILE_PARTIAL)
+            assert cls[0, t, s] == want, (t, s)
+
+
+def test_visible_ranges_closed_forms():
+    N = 600
+    one = np.zeros(N, np.int32)
+    rows = np.arange(N)
+    lo, hi = oracle.visible_key_ranges(one, rows, 200, 250)
+    seen = rows >= 200
+    np.testing.assert_array_equal(lo[seen], 200)
+    np.testing.assert_array_equal(hi[seen], np.minimum(rows[seen], 449))
+    assert (lo[~seen] == -1).all() and (hi[~seen] == -2).all()
+    ql, qh = oracle.visible_query_ranges(one, rows, 100, 300)
+    seen = rows <= 399
+    np.testing.assert_array_equal(ql[seen], np.maximum(rows[seen], 100))
+    np.testing.assert_array_equal(qh[seen], 399)
+    assert (ql[~seen] == -1).all()
+    alone = np.arange(N, dtype=np.int32)
+    lo, hi = oracle.visible_key_ranges(alone, rows, 0, N)
+    np.testing.assert_array_equal(lo, rows)
+    np.testing.assert_array_equal(hi, rows)
+
+
+@pytest.mark.parametrize("P", [1, 3, 4])
+def test_visible_ranges_over_ring_chunks_count_every_pair_once(P):
+    # summed over the P key chunks of a ring, the row ranges (and the
+    # key-side ranges) cover exactly the sum over examples of L(L+1)/2
+    L = wl.segment_lengths("uniform", 900, 11, lo=1, hi=300)
+    seg, _ = wl.segments_from_lengths(L)
+    bounds = np.linspace(0, 900, P + 1).astype(int)
+    rows = np.arange(900)
+    tot_r = tot_c = 0
+    for a, z in zip(bounds[:-1], bounds[1:]):
+        lo, hi = oracle.visible_key_ranges(seg, rows, a, z - a)
+        tot_r += int(np.maximum(hi - lo + 1, 0).sum())
+        ql, qh = oracle.visible_query_ranges(seg, rows, a, z - a)
+        tot_c += int(np.maximum(qh - ql + 1, 0).sum())
+    want = int((L * (L + 1) // 2).sum())
+    assert tot_r == want and tot_c == want
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_cross_classification_agrees_with_row_ranges(seed):
+    # a tile is EMPTY iff no row range meets its key block, FULL iff the
+    # block is whole and every row range covers its key block
+    N = 1100
+    L = wl.segment_lengths("uniform", N, 20 + seed, lo=1, hi=400)
+    seg, _ = wl.segments_from_lengths(L)
+    q_off, Nq, k_off, Nk = [(0, N, 0, N), (400, 700, 100, 500),
+                            (520, 580, 390, 260)][seed]
+    lo_, hi_, cls = oracle.classify_cross(seg[None], q_off, Nq, k_off, Nk,
+                                          128, 128)
+    lo, hi = oracle.visible_key_ranges(seg, np.arange(q_off, q_off + Nq),
+                                       k_off, Nk)
+    for t in range(cls.shape[1]):
+        r = slice(128 * t, min(128 * (t + 1), Nq))
+        for s in range(cls.shape[2]):
+            c0, c1 = k_off + 128 * s, k_off + min(128 * (s + 1), Nk) - 1
+            meet = (lo[r] <= c1) & (hi[r] >= c0) & (lo[r] <= hi[r])
+            cover = (lo[r] <= c0) & (hi[r] >= c1)
+            whole = (r.stop - r.start == 128) and (c1 - c0 == 127)
+            want = (oracle.TILE_EMPTY if not meet.any() else
+                    oracle.TILE_FULL if whole and cover.all() else
+                    oracle.TILE_PARTIAL)
+            assert cls[0, t, s] == want, (t, s)
+
+
 # ------------------------------------------------- workloads and page facts
 
 def test_workloads_use_page_facts():
@@ -452,3 +548,20 @@ def test_attention_in_rotate_half_layout_equals_permuted_interleaved():
     ref_out = np.exp(s - ref_lse[:, None]) @ v[b, :, h]
     np.testing.assert_allclose(out[b, :, h], ref_out, atol=1e-12)
     np.testing.assert_allclose(lse[b, h], ref_lse, atol=1e-12)
+
+
+def test_input_prefix_draw_equals_full_draw_prefix():
+    # the generator's prefix mode (used to time the oracle on a sample) must
+    # give exactly the first tokens of the full draw, across chunk borders
+    w = wl.Workload("t", 2, 300, 3, 16, 1e4, "uniform", 0.5, True,
+                    seg_args={"lo": 1, "hi": 50})
+    full = wl.make_inputs(w, 4)
+    for n in (1, 77, 300):
+        part = wl.make_inputs(w, 4, prefix=n)
+        for k in ("q", "k", "v", "dout", "segment_ids", "positions"):
+            assert torch.equal(part[k], full[k][:, :n]), (k, n)
+    x = wl.random_tensor((1, 50, 2, 8), 9, 1.0, torch.float32, "cpu",
+                         chunk_elems=64)
+    y = wl.random_tensor((1, 50, 2, 8), 9, 1.0, torch.float32, "cpu",
+                         chunk_elems=64, n_tokens=13)
+    assert torch.equal(x[:, :13], y)
