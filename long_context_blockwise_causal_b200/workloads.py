@@ -129,35 +129,44 @@ def visible_pairs(lengths_per_row) -> int:
 
 
 def random_tensor(shape, seed: int, scale: float, dtype, device,
-                  chunk_elems: int = 1 << 26):
+                  chunk_elems: int = 1 << 26, n_tokens: int | None = None):
     """N(0,1)*scale rounded to ``dtype``, drawn in chunks along dim 1.
 
     Chunking bounds the fp32 scratch for the 1M-token case; the values are
-    a deterministic function of (shape, seed, chunk_elems).
+    a deterministic function of (shape, seed, chunk_elems). ``n_tokens``
+    returns only the first n_tokens along dim 1 (the same values as that
+    prefix of the full tensor, drawing only the chunks it needs).
     """
     import torch
 
     g = torch.Generator(device=device)
     g.manual_seed(int(seed))
-    out = torch.empty(shape, dtype=dtype, device=device)
+    n = shape[1] if n_tokens is None else min(int(n_tokens), shape[1])
+    out = torch.empty((shape[0], n) + tuple(shape[2:]), dtype=dtype,
+                      device=device)
     if out.numel() == 0:
         return out
     per_tok = int(np.prod(shape[2:])) * shape[0]
     step = max(1, chunk_elems // max(1, per_tok))
-    for s in range(0, shape[1], step):
+    for s in range(0, n, step):
         e = min(shape[1], s + step)
         sub = (shape[0], e - s) + tuple(shape[2:])
         x = torch.randn(sub, generator=g, device=device, dtype=torch.float32)
         if scale != 1.0:
             x.mul_(scale)
-        out[:, s:e].copy_(x.to(dtype))
+        e = min(e, n)
+        out[:, s:e].copy_(x[:, :e - s].to(dtype))
     return out
 
 
 def make_inputs(w: Workload, seed: int, device="cpu", dtype=None,
                 N: int | None = None, B: int | None = None, H: int | None = None,
-                with_dout: bool | None = None):
-    """All inputs of one workload as torch tensors on ``device``."""
+                with_dout: bool | None = None, prefix: int | None = None):
+    """All inputs of one workload as torch tensors on ``device``.
+
+    ``prefix`` keeps only the first ``prefix`` tokens of every row (the
+    same values as the full draw; "lengths" still describes the full
+    rows)."""
     import torch
 
     dtype = torch.bfloat16 if dtype is None else dtype
@@ -166,18 +175,22 @@ def make_inputs(w: Workload, seed: int, device="cpu", dtype=None,
     H = w.H if H is None else H
     seg, pos, lens = make_segments(w, seed, N=N, B=B)
     shape = (B, N, H, w.D)
+    n = N if prefix is None else min(N, int(prefix))
+    draw = lambda k: random_tensor(shape, seed * 16 + k, w.scale, dtype,
+                                   device, n_tokens=n)
     t = {
-        "q": random_tensor(shape, seed * 16 + 1, w.scale, dtype, device),
-        "k": random_tensor(shape, seed * 16 + 2, w.scale, dtype, device),
-        "v": random_tensor(shape, seed * 16 + 3, w.scale, dtype, device),
-        "segment_ids": torch.from_numpy(seg).to(device),
-        "positions": torch.from_numpy(pos).to(device),
+        "q": draw(1),
+        "k": draw(2),
+        "v": draw(3),
+        "segment_ids": torch.from_numpy(np.ascontiguousarray(seg[:, :n])).to(
+            device),
+        "positions": torch.from_numpy(np.ascontiguousarray(pos[:, :n])).to(
+            device),
         "lengths": lens,
         "theta": w.theta,
     }
     if w.backward if with_dout is None else with_dout:
-        t["dout"] = random_tensor(shape, seed * 16 + 4, w.scale, dtype,
-                                  device)
+        t["dout"] = draw(4)
     return t
 
 
