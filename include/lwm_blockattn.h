@@ -288,8 +288,10 @@ LWM_API int lwm_blockffn_bwd(const void* x, const void* w_gate,
                              float* dw_up, float* dw_down, void* workspace,
                              size_t workspace_bytes, void* stream);
 
-/* Tile classifier (exported so it can be checked bit-exactly). For each
- * batch row b and query block t (Tq = ceil(N/block_q) blocks), key blocks
+/* General tile classifier, for any block sizes: a planning and reporting
+ * tool (how many tiles a packing leaves EMPTY / PARTIAL / FULL). The
+ * attention kernels themselves classify from the metadata that
+ * lwm_blockattn_visibility exports. For each batch row b and query block t (Tq = ceil(N/block_q) blocks), key blocks
  * j (Tk = ceil(N/block_k)):
  *   kv_lo[b][t] = (start of the packed example holding row t*block_q)
  *                 / block_k,
@@ -306,6 +308,47 @@ LWM_API int lwm_blockattn_classify(const int32_t* segment_ids, int B, int N,
                            int block_q, int block_k, int32_t* kv_lo,
                            int32_t* kv_hi, uint8_t* tile_class,
                            void* stream);
+
+/* The visibility metadata the attention kernels actually run on, exported
+ * so that their segment/causal tile classification can be checked
+ * bit-exactly (the mask: a query sees the keys of its own packed example
+ * at or before it, "LWM：突破 100 万 Token 的开源大模型", 概述 (b); tiles:
+ * the query/key chunks of 配置参数). Makes exactly the launches that
+ * lwm_blockattn_fwd / _fwd_block (query view) and lwm_blockattn_bwd /
+ * _bwd_block (key view) make before their attention kernels.
+ * Queries are the global token indices [q_off, q_off + Nq) with ids seg_q
+ * [B][Nq]; keys [k_off, k_off + Nk) with ids seg_k [B][Nk] (self-attention:
+ * the same array, offsets 0, Nq == Nk). Only block_q == block_k == 128.
+ * Query view (all six pointers or none):
+ *   row_lo, row_hi [B][Nq]: global indices of the first / last key the row
+ *     sees (none: row_lo > row_hi);
+ *   kv_lo, kv_hi [B][Tq]: the key blocks (counted from k_off) holding any
+ *     key the query block sees (none: kv_lo > kv_hi); the kernel visits
+ *     exactly these, every other tile is EMPTY;
+ *   lo_max, hi_min [B][Tq]: max row_lo and min row_hi over the block's
+ *     rows (INT_MAX / -INT_MAX when a row lies past Nq or sees nothing);
+ *     key block j (first key k0 = k_off + 128 j) is FULL, and takes the
+ *     mask-free path, iff lo_max <= k0 and hi_min >= k0 + 127; other
+ *     visited tiles are PARTIAL.
+ * Key view (all six or none), the same with queries and keys swapped:
+ *   col_lo, col_hi [B][Nk]: first / last query that sees the key;
+ *   q_lo, q_hi [B][Tk]: the query blocks the key block is visited with;
+ *   klo_max, khi_min [B][Tk]: the FULL test for query block t (first query
+ *     q0 = q_off + 128 t): klo_max <= q0 and khi_min >= q0 + 127.
+ * Caller-owned device buffers; async on stream. Returns LWM_ERR_INVALID_ARG
+ * for a partly given view or bad sizes, LWM_ERR_UNSUPPORTED for other
+ * block sizes; nothing is launched on error. */
+LWM_API int lwm_blockattn_visibility(const int32_t* seg_q,
+                                     const int32_t* seg_k, int B, int Nq,
+                                     int Nk, int q_off, int k_off,
+                                     int block_q, int block_k,
+                                     int32_t* row_lo, int32_t* row_hi,
+                                     int32_t* kv_lo, int32_t* kv_hi,
+                                     int32_t* lo_max, int32_t* hi_min,
+                                     int32_t* col_lo, int32_t* col_hi,
+                                     int32_t* q_lo, int32_t* q_hi,
+                                     int32_t* klo_max, int32_t* khi_min,
+                                     void* stream);
 
 /* RoPE table the kernels use: table[p][k] = (cos a, sin a) as float32 with
  * a = p * theta^(-2k/D) evaluated in fp64, p in [0, max_pos),
@@ -402,8 +445,10 @@ LWM_API uint64_t lwm_blockattn_kernel_launches(void);
  * only for such callers.
  * Arguments and results are those of lwm_blockattn_fwd without the
  * workspace: the scratch lives in a fixed device array inside the library
- * (LWM_NOALLOC_SCRATCH_BYTES). Sizes whose lwm_blockattn_fwd_workspace_size
- * exceeds it return LWM_ERR_WORKSPACE and launch nothing. The call never
+ * (LWM_NOALLOC_SCRATCH_BYTES). Every argument is first checked as
+ * lwm_blockattn_fwd checks it (same status codes); a valid, supported call
+ * whose lwm_blockattn_fwd_workspace_size exceeds the array returns
+ * LWM_ERR_WORKSPACE. Nothing is launched on error. The call never
  * allocates or frees memory.
  * The first call on each device looks up that device's scratch address
  * (cudaGetSymbolAddress with the device current); make it before any stream

@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstring>
 
+#include "api_checks.cuh"
 #include "aux_kernels.cuh"
 #include "decode.cuh"
 #include "mlp.cuh"
@@ -216,6 +217,30 @@ int run_forward(const void* q, const void* k_rot, const void* k_rot_lo,
 }
 
 }  // namespace
+
+int check_fwd_args(const void* q, const void* k, const void* v,
+                   const int32_t* segment_ids, const int32_t* positions,
+                   double theta, int block_q, int block_k, int max_pos, int B,
+                   int N, int H, int D, int dtype, int qk_precision,
+                   int rope_layout, const void* out, const float* lse) {
+  if (!sizes_ok(B, N, H, D, block_q, block_k, max_pos))
+    return LWM_ERR_INVALID_ARG;
+  if (!layout_ok(rope_layout)) return LWM_ERR_INVALID_ARG;
+  if (!(theta > 0.0) || !std::isfinite(theta)) return LWM_ERR_INVALID_ARG;
+  if (dtype != LWM_DTYPE_BF16 && dtype != LWM_DTYPE_FP32)
+    return LWM_ERR_INVALID_ARG;
+  if (qk_precision != LWM_QK_BF16 && qk_precision != LWM_QK_BF16X3)
+    return LWM_ERR_INVALID_ARG;
+  const int s = shape_status(D, block_q, block_k);
+  if (s != LWM_OK) return s;
+  if (int64_t(B) * N * H == 0) return kFwdNothingToDo;
+  if (max_pos < 1) return LWM_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, segment_ids, positions, out, lse};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return LWM_ERR_INVALID_ARG;
+  return LWM_OK;
+}
+
 }  // namespace lwm
 
 using namespace lwm;
@@ -339,22 +364,13 @@ int lwm_blockattn_fwd(const void* q, const void* k, const void* v,
                       int B, int N, int H, int D, int dtype, int qk_precision,
                       int rope_layout, void* out, float* lse, void* workspace,
                       size_t workspace_bytes, void* stream) {
-  if (!sizes_ok(B, N, H, D, block_q, block_k, max_pos))
-    return LWM_ERR_INVALID_ARG;
-  if (!layout_ok(rope_layout)) return LWM_ERR_INVALID_ARG;
+  const int c = check_fwd_args(q, k, v, segment_ids, positions, theta,
+                               block_q, block_k, max_pos, B, N, H, D, dtype,
+                               qk_precision, rope_layout, out, lse);
+  if (c == kFwdNothingToDo) return LWM_OK;
+  if (c != LWM_OK) return c;
+  if (!workspace || !aligned16(workspace)) return LWM_ERR_INVALID_ARG;
   const bool half = rope_layout == LWM_ROPE_HALF;
-  if (!(theta > 0.0) || !std::isfinite(theta)) return LWM_ERR_INVALID_ARG;
-  if (dtype != LWM_DTYPE_BF16 && dtype != LWM_DTYPE_FP32)
-    return LWM_ERR_INVALID_ARG;
-  if (qk_precision != LWM_QK_BF16 && qk_precision != LWM_QK_BF16X3)
-    return LWM_ERR_INVALID_ARG;
-  int s = shape_status(D, block_q, block_k);
-  if (s != LWM_OK) return s;
-  if (int64_t(B) * N * H == 0) return LWM_OK;
-  if (max_pos < 1) return LWM_ERR_INVALID_ARG;
-  const void* ptrs[] = {q, k, v, segment_ids, positions, out, lse, workspace};
-  for (const void* p : ptrs)
-    if (!p || !aligned16(p)) return LWM_ERR_INVALID_ARG;
   Workspace w = carve(workspace, B, N, N, H, D, max_pos, Pass::kFwd, dtype,
                       qk_precision);
   if (workspace_bytes < w.bytes) return LWM_ERR_WORKSPACE;
@@ -700,6 +716,44 @@ int lwm_blockattn_classify(const int32_t* segment_ids, int B, int N,
   if (tile_class)
     LWM_TRY(launch_tile_class(segment_ids, B, N, block_q, block_k, kv_lo,
                               kv_hi, tile_class, st));
+  return LWM_OK;
+}
+
+int lwm_blockattn_visibility(const int32_t* seg_q, const int32_t* seg_k,
+                             int B, int Nq, int Nk, int q_off, int k_off,
+                             int block_q, int block_k, int32_t* row_lo,
+                             int32_t* row_hi, int32_t* kv_lo, int32_t* kv_hi,
+                             int32_t* lo_max, int32_t* hi_min,
+                             int32_t* col_lo, int32_t* col_hi, int32_t* q_lo,
+                             int32_t* q_hi, int32_t* klo_max,
+                             int32_t* khi_min, void* stream) {
+  if (B < 0 || Nq < 0 || Nk < 0 || q_off < 0 || k_off < 0 ||
+      (int64_t(B) * Nq) >= (int64_t(1) << 31) ||
+      (int64_t(B) * Nk) >= (int64_t(1) << 31))
+    return LWM_ERR_INVALID_ARG;
+  if (block_q != kBlock || block_k != kBlock) return LWM_ERR_UNSUPPORTED;
+  int32_t* qside[] = {row_lo, row_hi, kv_lo, kv_hi, lo_max, hi_min};
+  int32_t* kside[] = {col_lo, col_hi, q_lo, q_hi, klo_max, khi_min};
+  // each view is written whole or not at all
+  auto group = [](int32_t* const (&g)[6]) {
+    int n = 0;
+    for (int32_t* p : g) n += p != nullptr;
+    return n;
+  };
+  const int nq = group(qside), nk = group(kside);
+  if ((nq != 0 && nq != 6) || (nk != 0 && nk != 6)) return LWM_ERR_INVALID_ARG;
+  if (int64_t(B) * Nq * Nk == 0 || (nq == 0 && nk == 0)) return LWM_OK;
+  if (!seg_q || !seg_k) return LWM_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the very launches lwm_blockattn_fwd / _fwd_block and lwm_blockattn_bwd /
+  // _bwd_block make before their attention kernels
+  if (nq)
+    LWM_TRY(launch_cross_meta(seg_q, seg_k, B, Nq, Nk, q_off, k_off, row_lo,
+                              row_hi, kv_lo, kv_hi, lo_max, hi_min, st));
+  if (nk)
+    LWM_TRY(launch_cross_meta_keys(seg_q, seg_k, B, Nq, Nk, q_off, k_off,
+                                   col_lo, col_hi, q_lo, q_hi, klo_max,
+                                   khi_min, st));
   return LWM_OK;
 }
 

@@ -44,6 +44,8 @@ _SIGS = {
     "lwm_blockattn_classify": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp,
                                     _vp]),
     "lwm_blockattn_rope_table": (_i, [_d, _i, _i, _vp, _vp]),
+    "lwm_blockattn_visibility": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _i]
+                                 + [_vp] * 13),
     "lwm_blockattn_check_inputs": (_i, [_vp, _vp, _i, _i, _i,
                                         ctypes.POINTER(_i), _vp]),
     "lwm_blockattn_last_status": (_i, [_vp]),
@@ -270,11 +272,15 @@ def fwd_noalloc(q, k, v, segment_ids, positions, theta, max_pos,
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    st = lib().lwm_blockattn_fwd_noalloc(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(segment_ids), _ptr(positions),
-        float(theta), block_q, block_k, int(max_pos), B, N, H, D,
-        _dtype_code(q), _qk_code(qk_precision), _layout_code(rope_layout),
-        _ptr(out), _ptr(lse), _stream(stream))
+    # the library uses the scratch array of the current device: make it the
+    # tensors' device (and take that device's stream by default)
+    with torch.cuda.device(q.device):
+        st = lib().lwm_blockattn_fwd_noalloc(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(segment_ids), _ptr(positions),
+            float(theta), block_q, block_k, int(max_pos), B, N, H, D,
+            _dtype_code(q), _qk_code(qk_precision),
+            _layout_code(rope_layout), _ptr(out), _ptr(lse),
+            _stream(stream))
     _check(st, "lwm_blockattn_fwd_noalloc")
     return out, lse
 
@@ -500,6 +506,47 @@ def classify(segment_ids, block_q=BLOCK, block_k=BLOCK, with_class=True,
                                       _stream(stream))
     _check(st, "lwm_blockattn_classify")
     return lo, hi, cls
+
+
+VISIBILITY_QUERY_VIEW = ("row_lo", "row_hi", "kv_lo", "kv_hi", "lo_max",
+                         "hi_min")
+VISIBILITY_KEY_VIEW = ("col_lo", "col_hi", "q_lo", "q_hi", "klo_max",
+                       "khi_min")
+
+
+def visibility(seg_q, seg_k=None, q_off=0, k_off=0, query_view=True,
+               key_view=True, block_q=BLOCK, block_k=BLOCK, stream=None):
+    """The metadata the attention kernels classify tiles with (see
+    lwm_blockattn_visibility). seg_q [B,Nq] int32 ids of queries
+    [q_off, q_off+Nq); seg_k [B,Nk] of keys [k_off, k_off+Nk) (default:
+    seg_q, self-attention). Returns a dict of int32 tensors: per query row
+    and per query block (query view), per key and per key block (key
+    view)."""
+    seg_k = seg_q if seg_k is None else seg_k
+    _need_cuda(seg_q, seg_k)
+    _expect_dims("visibility", "seg_q", seg_q, 2)
+    _expect_dims("visibility", "seg_k", seg_k, 2)
+    B, Nq = seg_q.shape
+    Nk = seg_k.shape[1]
+    _expect("visibility", "seg_q", seg_q, (B, Nq), torch.int32)
+    _expect("visibility", "seg_k", seg_k, (B, Nk), torch.int32)
+    _same_device("visibility", seg_q, seg_k)
+    dev = seg_q.device
+    tq, tk = -(-Nq // block_q), -(-Nk // block_k)
+    shapes = dict(zip(VISIBILITY_QUERY_VIEW,
+                      [(B, Nq)] * 2 + [(B, tq)] * 4))
+    shapes.update(zip(VISIBILITY_KEY_VIEW, [(B, Nk)] * 2 + [(B, tk)] * 4))
+    want = (VISIBILITY_QUERY_VIEW if query_view else ()) + \
+        (VISIBILITY_KEY_VIEW if key_view else ())
+    res = {n: torch.empty(shapes[n], dtype=torch.int32, device=dev)
+           for n in want}
+    ptrs = [_ptr(res.get(n)) for n in VISIBILITY_QUERY_VIEW +
+            VISIBILITY_KEY_VIEW]
+    st = lib().lwm_blockattn_visibility(_ptr(seg_q), _ptr(seg_k), B, Nq, Nk,
+                                        int(q_off), int(k_off), block_q,
+                                        block_k, *ptrs, _stream(stream))
+    _check(st, "lwm_blockattn_visibility")
+    return res
 
 
 def rope_table(theta, max_pos, D=HEAD_DIM, device="cuda", stream=None):

@@ -101,6 +101,56 @@ def test_fwd_rejects_bad_arguments_before_launch(kw, status):
     assert _fwd_raw(**kw) == status
 
 
+def test_visibility_rejects_bad_arguments_before_launch():
+    L = ops.lib()
+    p = ctypes.c_void_p(1 << 20)
+    six = [p] * 6
+    none6 = [None] * 6
+
+    def call(*views, B=1, Nq=16, Nk=16, q_off=0, k_off=0, bq=128, bk=128,
+             seg=p):
+        ptrs = [x for view in views for x in view]
+        return L.lwm_blockattn_visibility(seg, seg, B, Nq, Nk, q_off, k_off,
+                                          bq, bk, *ptrs, None)
+
+    # a view given in part is refused (it would leave the rest unwritten)
+    assert call([p, None] + [p] * 4, none6) == ops.ERR_INVALID_ARG
+    assert call(none6, [p] * 5 + [None]) == ops.ERR_INVALID_ARG
+    assert call(six, six, bk=64) == ops.ERR_UNSUPPORTED
+    assert call(six, six, q_off=-1) == ops.ERR_INVALID_ARG
+    assert call(six, six, Nk=-3) == ops.ERR_INVALID_ARG
+    assert call(six, six, seg=None) == ops.ERR_INVALID_ARG
+    # nothing to do: no launch, no pointer touched
+    assert call(none6, none6) == ops.OK
+    assert call(six, six, Nq=0) == ops.OK
+    assert call(six, six, B=0) == ops.OK
+
+
+def test_noalloc_checks_arguments_before_its_scratch_size():
+    # an invalid or unsupported call too large for the fixed scratch must
+    # report what is wrong with it, not the scratch size (no CUDA call is
+    # made on any of these paths)
+    L = ops.lib()
+    p = ctypes.c_void_p(1 << 20)
+
+    def call(N=262144, H=32, D=128, dtype=0, qkp=0, layout=0, bk=128,
+             theta=5e7, q=p):
+        return L.lwm_blockattn_fwd_noalloc(q, p, p, p, p, theta, 128, bk,
+                                           N, 1, N, H, D, dtype, qkp, layout,
+                                           p, p, None)
+
+    assert call() == ops.ERR_WORKSPACE              # valid, too large
+    assert call(D=64) == ops.ERR_UNSUPPORTED
+    assert call(bk=64) == ops.ERR_UNSUPPORTED
+    assert call(dtype=9) == ops.ERR_INVALID_ARG
+    assert call(qkp=4) == ops.ERR_INVALID_ARG
+    assert call(layout=3) == ops.ERR_INVALID_ARG
+    assert call(theta=0.0) == ops.ERR_INVALID_ARG
+    assert call(q=None) == ops.ERR_INVALID_ARG
+    assert call(q=ctypes.c_void_p((1 << 20) + 4)) == ops.ERR_INVALID_ARG
+    assert call(H=0) == ops.OK                      # nothing to do
+
+
 def test_bwd_and_classify_reject_bad_arguments():
     L = ops.lib()
     v = ctypes.c_void_p
