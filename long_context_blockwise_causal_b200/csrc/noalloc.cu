@@ -22,6 +22,7 @@
 // ordering between them) race on the array: serialise them.
 #include <mutex>
 
+#include "api_checks.cuh"
 #include "aux_kernels.cuh"
 
 namespace lwm {
@@ -63,6 +64,14 @@ int lwm_blockattn_fwd_noalloc(const void* q, const void* k, const void* v,
                               int N, int H, int D, int dtype,
                               int qk_precision, int rope_layout, void* out,
                               float* lse, void* stream) {
+  // the forward's own checks first: an invalid or unsupported call reports
+  // that, not the size of the scratch
+  const int c = lwm::check_fwd_args(q, k, v, segment_ids, positions, theta,
+                                    block_q, block_k, max_pos, B, N, H, D,
+                                    dtype, qk_precision, rope_layout, out,
+                                    lse);
+  if (c == lwm::kFwdNothingToDo) return LWM_OK;
+  if (c != LWM_OK) return c;
   const size_t need = lwm_blockattn_fwd_workspace_size(
       B, N, H, D, block_q, block_k, max_pos, dtype, qk_precision);
   if (need == 0) return LWM_ERR_INVALID_ARG;
