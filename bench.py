@@ -181,10 +181,11 @@ def oracle_sample(w, t_host, budget_s, backward):
         flop = (14 if backward else 4) * w.D * pairs
         return dt, flop
 
-    L = min(1024, w.N)
+    avail = t_host["q"].shape[1]   # the host copy may be a prefix
+    L = min(1024, avail)
     dt, _ = run(L)
     scale = math.sqrt(max(budget_s, 0.1) / max(dt, 1e-3))
-    L = int(min(w.N, max(128, (L * scale) // 128 * 128)))
+    L = int(min(avail, max(128, (L * scale) // 128 * 128)))
     dt, flop = run(L)
     threads = max((i.get("num_threads", 1) for i in threadpool_info()),
                   default=1)
@@ -262,13 +263,18 @@ def max_over_ranks(x, ws, dev):
     return dist.max_over_ranks(x, ws, dev)
 
 
+REF_PREFIX_TOKENS = 32768
+
+
 def reference_arm(args, ws, rank):
     """The oracle, timed as it stands on the host cores (rank 0 only)."""
     if rank != 0:
         return
     w = wl.WORKLOADS[args.workload]
+    # the oracle runs on a prefix of row 0: draw only that much of the
+    # inputs (the same values as the full draw)
     t_host = wl.make_inputs(w, args.seed, device="cpu",
-                            with_dout=w.backward)
+                            with_dout=w.backward, prefix=REF_PREFIX_TOKENS)
     times, flops, info = [], [], None
     for i in range(args.warmup + args.steps):
         tf, info = oracle_sample(w, t_host, args.ref_budget, w.backward)
@@ -655,10 +661,10 @@ def bench_ffn(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="text32k",
+    ap.add_argument("--workload", default="packed128k",
                     choices=sorted(wl.WORKLOADS) + sorted(DECODE_WORKLOADS)
                     + sorted(wl.FFN_WORKLOADS))
     ap.add_argument("--seed", type=int, default=0)
@@ -689,6 +695,64 @@ def main():
         rank = int(os.environ.get("RANK", "0"))
         reference_arm(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
         return
+    bench_attention(args)
+
+
+L2_BYTES = 126e6
+
+
+def tile_counts(ops, segment_ids):
+    """Tiles the forward kernel visits and, of those, the ones it takes
+    mask-free, from the very metadata it runs on (lwm_blockattn_visibility:
+    key blocks [kv_lo, kv_hi] per query block, FULL iff every row's key
+    range covers the block)."""
+    v = ops.visibility(segment_ids, key_view=False)
+    lo, hi = v["kv_lo"].long(), v["kv_hi"].long()
+    lo_max, hi_min = v["lo_max"].long(), v["hi_min"].long()
+    visited = (hi - lo + 1).clamp(min=0)
+    blk = ops.BLOCK
+    first_full = torch.maximum(lo, (lo_max + blk - 1).div(blk,
+                                                          rounding_mode="floor"))
+    last_full = torch.minimum(hi, (hi_min - (blk - 1)).div(
+        blk, rounding_mode="floor"))
+    full = (last_full - first_full + 1).clamp(min=0)
+    full = torch.where(lo_max > hi_min, torch.zeros_like(full), full)
+    return int(visited.sum().item()), int(full.sum().item())
+
+
+def copy_floor(dev, h_in, d_in, h_out, d_out):
+    """Host<->device copy time of one step's bytes over this box's link:
+    uploads alone, downloads alone and both at once on two streams (ms,
+    CUDA events, after one untimed round)."""
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def once(do_up, do_down):
+        comp = torch.cuda.current_stream(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(comp)
+        up.wait_stream(comp)
+        down.wait_stream(comp)
+        if do_up:
+            with torch.cuda.stream(up):
+                for n, hb in h_in.items():
+                    d_in[n].copy_(hb, non_blocking=True)
+        if do_down:
+            with torch.cuda.stream(down):
+                for hb, db in zip(h_out, d_out):
+                    hb.copy_(db, non_blocking=True)
+        comp.wait_stream(up)
+        comp.wait_stream(down)
+        e1.record(comp)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1)
+
+    once(True, True)
+    return {"h2d_ms": once(True, False), "d2h_ms": once(False, True),
+            "both_ms": once(True, True)}
+
+
+def bench_attention(args):
     ws, rank, local = init_dist(args.impl)
 
     from long_context_blockwise_causal_b200 import ops
@@ -712,13 +776,13 @@ def main():
                            with_dout=w.backward)
     B, N, H, D = t["q"].shape
     pairs_per_head = wl.visible_pairs(t["lengths"])
-    # tile pairs the kernels execute (key blocks in each query block's
-    # [kv_lo, kv_hi], 128 x 128 pairs each) over the visible pairs
-    lo_, hi_, _ = ops.classify(t["segment_ids"], with_class=False)
-    executed_ratio = float(((hi_ - lo_ + 1).clamp(min=0).sum().item())
-                           * 128 * 128 / max(1, pairs_per_head))
+    tiles_visited, tiles_full = tile_counts(ops, t["segment_ids"])
     fwd_flop = 4.0 * D * pairs_per_head * H
     bwd_flop = 10.0 * D * pairs_per_head * H if w.backward else 0.0
+    elem = t["q"].element_size()
+    # forward algorithmic bytes: q, k, v in, out and lse out, ids and
+    # positions in
+    fwd_bytes = 4 * B * N * H * D * elem + B * H * N * 4 + 8 * B * N
     strong = args.shard == "heads" and ws > 1
     # whole-job work: replicas multiply it by the rank count, a head-sharded
     # job is one workload split across the ranks
@@ -735,6 +799,11 @@ def main():
     grads = [torch.empty_like(t["q"]) for _ in range(3)] if w.backward \
         else None
     stream = torch.cuda.current_stream(dev)
+    # inputs smaller than L2 would be re-read from it: flush it (a write
+    # larger than L2) before every timed step, outside the step's events
+    small = 3 * t["q"].numel() * elem < L2_BYTES
+    flush = torch.empty(int(2 * L2_BYTES), dtype=torch.uint8, device=dev) \
+        if small else None
 
     def step(ev=None):
         if ev is not None:
@@ -750,10 +819,12 @@ def main():
                     max_pos=max_pos, qk_precision=qkp, dq=grads[0],
                     dk=grads[1], dv=grads[2], workspace=workspace,
                     stream=stream)
-            if ev is not None:
-                ev[2].record(stream)
+        if ev is not None:
+            ev[2].record(stream)
 
     for _ in range(args.warmup):
+        if small:
+            flush.zero_()
         step()
     torch.cuda.synchronize(dev)
     if ops.last_status() != ops.OK:
@@ -772,6 +843,8 @@ def main():
     end = torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for i in range(args.steps):
+        if small:
+            flush.zero_()
         step(evs[i])
     end.record(stream)
     torch.cuda.synchronize(dev)
@@ -779,11 +852,14 @@ def main():
     barrier(ws)
     clk = clocks.stop() if clocks else None
     status = ops.last_status()
-    ms = start.elapsed_time(end) / args.steps
-    ms = max_over_ranks(ms, ws, dev)
     fwd_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
     bwd_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs])) \
         if w.backward else 0.0
+    # with flushes in between, a step is its own events; else the whole
+    # bracketed interval over the steps
+    ms = (fwd_ms + bwd_ms) if small else \
+        start.elapsed_time(end) / args.steps
+    ms = max_over_ranks(ms, ws, dev)
 
     # end to end through the public API with pinned host buffers
     e2e = None
@@ -822,19 +898,31 @@ def main():
             return [d["out"], d["lse"]] + (d["grads"] if w.backward else [])
 
         pipelined_e2e(dev, hin, make_set, run, outputs, hout, 2)  # warm-up
+        s0 = make_set()
+        link = copy_floor(dev, hin, s0, hout, outputs(s0))
+        del s0
         barrier(ws)
-        ksteps = max(2, min(args.steps, 6))
         ems = max_over_ranks(pipelined_e2e(dev, hin, make_set, run, outputs,
-                                           hout, ksteps), ws, dev)
+                                           hout, max(2, args.steps)), ws,
+                             dev)
+        compute_ms = fwd_ms + bwd_ms
         e2e = {"value": (fwd_flop + bwd_flop) * job_scale / (ems / 1e3) / 1e12,
                "unit": "TFLOP/s", "ms_per_step": ems,
+               "steps": max(2, args.steps),
                "tokens_per_s": B * N * (1 if strong else ws) / (ems / 1e3),
                "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h),
+               "link": {**link,
+                        "h2d_gbs": h2d / link["h2d_ms"] / 1e6,
+                        "d2h_gbs": d2h / link["d2h_ms"] / 1e6},
+               "floor_ms": max(link["both_ms"], compute_ms),
+               "over_floor": ems / max(link["both_ms"], compute_ms),
                "copies": "every step uploads its inputs and downloads its "
                          "results through pinned host buffers, on copy "
                          "streams overlapped with the neighbouring steps' "
-                         "compute (two device buffer sets)"}
+                         "compute (two device buffer sets); floor = the "
+                         "slower of one step's uploads and downloads run "
+                         "together on this link and the step's compute"}
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -858,8 +946,30 @@ def main():
         peak_sus = pk.get("bf16_tflops_sustained", peak_burst)
         fwd_tf = fwd_flop / (fwd_ms / 1e3) / 1e12
         bwd_tf = bwd_flop / (bwd_ms / 1e3) / 1e12 if w.backward else None
+        fwd_gbs = fwd_bytes / (fwd_ms / 1e3) / 1e9
         dom = "bwd" if w.backward and bwd_ms > fwd_ms else "fwd"
         ach = bwd_tf if dom == "bwd" else fwd_tf
+        kernel = f"{dom}_tc_kernel"
+        if small:
+            # a few MB per call: launch- and memory-latency-bound, reported
+            # against HBM bandwidth
+            roof = {"bound": "hbm", "kernel": "forward call (all kernels)",
+                    "achieved": fwd_gbs, "peak": pk["hbm_gbs"],
+                    "unit": "GB/s", "frac": fwd_gbs / pk["hbm_gbs"],
+                    "peak_kind": f"copy bandwidth ({pk['source']})",
+                    "algorithmic_bytes": fwd_bytes, "traffic": None,
+                    "us_per_call": fwd_ms * 1e3}
+        else:
+            # the timed region is well under a second of back-to-back
+            # launches: the burst peak applies
+            roof = {"bound": "tensor", "kernel": kernel, "achieved": ach,
+                    "peak": peak_burst,
+                    "peak_kind": f"bf16 burst ({pk['source']})",
+                    "unit": "TFLOP/s", "frac": ach / peak_burst,
+                    "frac_of_sustained_peak": ach / peak_sus,
+                    "traffic": recorded_traffic(w.name, kernel),
+                    "traffic_unit": "bytes per launch (ncu, dram "
+                                    "read+write)"}
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s",
             "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
@@ -870,26 +980,29 @@ def main():
                        "heads_per_rank": H, "D": D,
                        "theta": w.theta, "qk_precision": qkp,
                        "segments": w.segments,
+                       "passes": "fwd+bwd" if w.backward else "fwd",
                        "visible_pairs_per_head": pairs_per_head,
-                       "executed_tile_pairs_over_visible": executed_ratio,
-                       "l2": "inputs larger than L2 (no flush)"
-                       if 3 * t["q"].numel() * 2 > 126e6 else
-                       "inputs smaller than L2 (re-read from L2)",
+                       "tiles_visited_per_head": tiles_visited // B,
+                       "tiles_full_per_head": tiles_full // B,
+                       "executed_tile_pairs_over_visible":
+                           tiles_visited * 128 * 128 / max(1, B *
+                                                          pairs_per_head),
+                       "l2": "inputs smaller than L2: L2 flushed (256 MB "
+                             "write) before every timed step" if small else
+                             "inputs larger than L2 (no flush)",
                        "parallelism": (f"heads split over {ws} GPUs" if strong
                                        else f"replicas x{ws}")},
             "tokens_per_s": B * N * (1 if strong else ws) / (ms / 1e3),
             "fwd": {"ms": fwd_ms, "tflops": fwd_tf,
-                    "frac_of_burst_peak": fwd_tf / peak_burst},
+                    "frac_of_burst_peak": fwd_tf / peak_burst,
+                    "frac_of_sustained_peak": fwd_tf / peak_sus,
+                    "hbm_gbs_algorithmic": fwd_gbs,
+                    "tokens_per_s": B * N / (fwd_ms / 1e3)},
             "bwd": ({"ms": bwd_ms, "tflops": bwd_tf,
-                     "frac_of_burst_peak": bwd_tf / peak_burst}
+                     "frac_of_burst_peak": bwd_tf / peak_burst,
+                     "frac_of_sustained_peak": bwd_tf / peak_sus}
                     if w.backward else None),
-            "roofline": {"bound": "tensor", "kernel": f"{dom}_tc_kernel",
-                         "achieved": ach, "peak": peak_sus,
-                         "peak_kind": f"bf16 sustained ({pk['source']})",
-                         "unit": "TFLOP/s", "frac": ach / peak_sus,
-                         "frac_of_burst_peak": ach / peak_burst,
-                         "traffic": recorded_traffic(w.name, f"{dom}_tc_kernel"),
-                         "traffic_unit": "bytes per launch (ncu, dram read+write)"},
+            "roofline": roof,
             "gpu_launches": int(launches),
             "device_status": status,
             "clocks": clk,
