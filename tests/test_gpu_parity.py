@@ -263,25 +263,74 @@ def test_bwd_bf16_split_qk_tiny(cuda_dev):
     check_bwd_full(t, run_bwd(t, "bf16x3"), BWD_REL_BF16, 0.0)
 
 
+def check_bwd_rows(h, t, dq, rows, heads):
+    idx = torch.from_numpy(rows).to(dq.device)
+    gq = dq[0, idx].float().cpu().numpy()
+    for hh in heads:
+        r = oracle.attn_bwd_rows(h["q"], h["k"], h["v"], h["dout"],
+                                 h["segment_ids"], h["positions"],
+                                 t["theta"], 0, hh, rows)
+        err = np.abs(gq[:, hh] - r).max()
+        assert err <= BWD_REL_BF16 * np.abs(r).max(), (hh, err)
+
+
+def check_bwd_cols(h, t, dk, dv, a, z, cols, heads):
+    """dk, dv at keys ``cols`` (global indices in [a, z)) against the oracle
+    run on tokens [a, z). With a, z the bounds of the packed example that
+    holds the keys (or the whole row) nothing outside [a, z) sees them or
+    is seen by the rows that do, so the oracle on that slice is the oracle
+    on the whole row."""
+    sl = {k_: h[k_][:, a:z] for k_ in ("q", "k", "v", "dout", "segment_ids",
+                                       "positions")}
+    idx = torch.from_numpy(cols).to(dk.device)
+    gk = dk[0, idx].float().cpu().numpy()
+    gv = dv[0, idx].float().cpu().numpy()
+    for hh in heads:
+        rk, rv = oracle.attn_bwd_cols(sl["q"], sl["k"], sl["v"], sl["dout"],
+                                      sl["segment_ids"], sl["positions"],
+                                      t["theta"], 0, hh, cols - a,
+                                      row_block=1024)
+        ek = np.abs(gk[:, hh] - rk).max()
+        ev = np.abs(gv[:, hh] - rv).max()
+        assert ek <= BWD_REL_BF16 * np.abs(rk).max(), (hh, ek)
+        assert ev <= BWD_REL_BF16 * np.abs(rv).max(), (hh, ev)
+
+
 def test_bwd_text32k_full_size_sampled(cuda_dev):
-    # the benchmark's workload and launch configuration
+    # the 32K workload at full size: dq on 64 rows of 2 heads, dk and dv on
+    # 64 keys of 4 heads (each key column needs the whole head's forward)
     t = inputs("text32k", 0, cuda_dev, dout=True)
     dq, dk, dv = run_bwd(t)
     h = host(t)
     N = t["q"].shape[1]
     rng = np.random.default_rng(21)
     rows = np.unique(np.r_[0, N - 1, rng.integers(0, N, 62)])
-    idx = torch.from_numpy(rows).to(dq.device)
-    gq = dq[0, idx].float().cpu().numpy()
-    gk = dk[0, idx].float().cpu().numpy()
-    gv = dv[0, idx].float().cpu().numpy()
-    for hh in (0, 17):
-        r = oracle.attn_bwd_rows(h["q"], h["k"], h["v"], h["dout"],
-                                 h["segment_ids"], h["positions"],
-                                 t["theta"], 0, hh, rows)
-        assert np.abs(gq[:, hh] - r).max() <= BWD_REL_BF16 * np.abs(r).max()
-    rk, rv = oracle.attn_bwd_cols(h["q"], h["k"], h["v"], h["dout"],
-                                  h["segment_ids"], h["positions"],
-                                  t["theta"], 0, 5, rows, row_block=1024)
-    assert np.abs(gk[:, 5] - rk).max() <= BWD_REL_BF16 * np.abs(rk).max()
-    assert np.abs(gv[:, 5] - rv).max() <= BWD_REL_BF16 * np.abs(rv).max()
+    check_bwd_rows(h, t, dq, rows, (0, 17))
+    check_bwd_cols(h, t, dk, dv, 0, N, rows, (5, 12, 20, 31))
+
+
+def test_bwd_packed128k_full_size_sampled(cuda_dev):
+    # the 128K packed workload (seed 0) in the benchmark's launch
+    # configuration: dq on the first and last token of every example plus
+    # random rows; dk, dv on the first and last key and random keys of six
+    # examples (short to 22.8K tokens); four heads each
+    t = inputs("packed128k", 0, cuda_dev, dout=True)
+    dq, dk, dv = run_bwd(t)
+    h = host(t)
+    L = t["lengths"][0]
+    starts = np.r_[0, np.cumsum(L)[:-1]]
+    ends = starts + L - 1
+    rng = np.random.default_rng(31)
+    N = t["q"].shape[1]
+    rows = np.unique(np.r_[starts, ends, rng.integers(0, N, 40)])
+    assert len(rows) >= 64
+    check_bwd_rows(h, t, dq, rows, (0, 9, 22, 31))
+    picked = [i for i in np.argsort(L) if L[i] <= 23000]
+    docs = picked[:4] + picked[-2:]  # the four shortest and two long ones
+    ncols = 0
+    for i in docs:
+        a, z = int(starts[i]), int(ends[i]) + 1
+        cols = np.unique(np.r_[a, z - 1, rng.integers(a, z, 10)])
+        check_bwd_cols(h, t, dk, dv, a, z, cols, (0, 9, 22, 31))
+        ncols += len(cols)
+    assert ncols >= 64
