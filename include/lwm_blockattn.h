@@ -51,9 +51,13 @@
  *   - Preconditions the kernels trust (lwm_blockattn_check_inputs verifies
  *     them): segment_ids non-decreasing along each batch row (packed
  *     examples are contiguous runs); 0 <= positions < max_pos.
- *   - Supported shapes: D == 128; block_q == block_k == 128; any N >= 0
- *     (a ragged last block is masked); B, H >= 0 (0 => no work); every
- *     tensor pointer 16-byte aligned.
+ *   - Supported shapes: D == 128; block_q == 128; block_k == 128 or 64
+ *     (the forward sweeps key tiles of block_k keys; with 64 the first key
+ *     tile a query block visits leaves half of its rows with no visible
+ *     key yet, which the online softmax handles; the key-major backward
+ *     visits 128-key units either way, an exact reorganisation with the
+ *     same gradients); any N >= 0 (a ragged last block is masked);
+ *     B, H >= 0 (0 => no work); every tensor pointer 16-byte aligned.
  */
 #ifndef LWM_BLOCKATTN_H
 #define LWM_BLOCKATTN_H
@@ -291,8 +295,8 @@ LWM_API int lwm_blockffn_bwd(const void* x, const void* w_gate,
 /* General tile classifier, for any block sizes: a planning and reporting
  * tool (how many tiles a packing leaves EMPTY / PARTIAL / FULL). The
  * attention kernels themselves classify from the metadata that
- * lwm_blockattn_visibility exports. For each batch row b and query block t (Tq = ceil(N/block_q) blocks), key blocks
- * j (Tk = ceil(N/block_k)):
+ * lwm_blockattn_visibility exports. For each batch row b and query block
+ * t (Tq = ceil(N/block_q) blocks), key blocks j (Tk = ceil(N/block_k)):
  *   kv_lo[b][t] = (start of the packed example holding row t*block_q)
  *                 / block_k,
  *   kv_hi[b][t] = (last valid row of block t) / block_k,
@@ -318,7 +322,9 @@ LWM_API int lwm_blockattn_classify(const int32_t* segment_ids, int B, int N,
  * _bwd_block (key view) make before their attention kernels.
  * Queries are the global token indices [q_off, q_off + Nq) with ids seg_q
  * [B][Nq]; keys [k_off, k_off + Nk) with ids seg_k [B][Nk] (self-attention:
- * the same array, offsets 0, Nq == Nk). Only block_q == block_k == 128.
+ * the same array, offsets 0, Nq == Nk). block_q == 128; block_k == 128,
+ * or 64 for the query view alone (the forward's 64-key tiles; the
+ * backward's key view is always in 128-key units).
  * Query view (all six pointers or none):
  *   row_lo, row_hi [B][Nq]: global indices of the first / last key the row
  *     sees (none: row_lo > row_hi);
@@ -327,9 +333,9 @@ LWM_API int lwm_blockattn_classify(const int32_t* segment_ids, int B, int N,
  *     exactly these, every other tile is EMPTY;
  *   lo_max, hi_min [B][Tq]: max row_lo and min row_hi over the block's
  *     rows (INT_MAX / -INT_MAX when a row lies past Nq or sees nothing);
- *     key block j (first key k0 = k_off + 128 j) is FULL, and takes the
- *     mask-free path, iff lo_max <= k0 and hi_min >= k0 + 127; other
- *     visited tiles are PARTIAL.
+ *     key block j (first key k0 = k_off + block_k j) is FULL, and takes
+ *     the mask-free path, iff lo_max <= k0 and hi_min >= k0 + block_k - 1;
+ *     other visited tiles are PARTIAL.
  * Key view (all six or none), the same with queries and keys swapped:
  *   col_lo, col_hi [B][Nk]: first / last query that sees the key;
  *   q_lo, q_hi [B][Tk]: the query blocks the key block is visited with;

@@ -141,8 +141,12 @@ bool sizes_ok(int B, int N, int H, int D, int block_q, int block_k,
          max_pos >= 0 && (int64_t(B) * N) < (int64_t(1) << 31);
 }
 
+// Query blocks of 128 rows; key blocks of 128 or 64 keys (the forward
+// sweeps key tiles of that height; the key-major backward visits 128-key
+// units either way, which gives the same gradients).
 int shape_status(int D, int block_q, int block_k) {
-  if (D != kHeadDim || block_q != kBlock || block_k != kBlock)
+  if (D != kHeadDim || block_q != kBlock ||
+      (block_k != kBlock && block_k != kBlock / 2))
     return LWM_ERR_UNSUPPORTED;
   return LWM_OK;
 }
@@ -194,11 +198,11 @@ int run_backward(BwdArgs a, const int32_t* seg_q, const int32_t* seg_k,
 int run_forward(const void* q, const void* k_rot, const void* k_rot_lo,
                 const void* v, const int32_t* seg_q, const int32_t* pos_q,
                 const int32_t* seg_k, int q_off, int k_off, int B, int Nq,
-                int Nk, int H, bool x3, bool half, void* out, float* lse,
-                const Workspace& w, cudaStream_t st) {
-  LWM_TRY(launch_cross_meta(seg_q, seg_k, B, Nq, Nk, q_off, k_off, w.row_lo,
-                            w.row_hi, w.kv_lo, w.kv_hi, w.lo_max, w.hi_min,
-                            st));
+                int Nk, int H, int block_k, bool x3, bool half, void* out,
+                float* lse, const Workspace& w, cudaStream_t st) {
+  LWM_TRY(launch_cross_meta(seg_q, seg_k, B, Nq, Nk, q_off, k_off, block_k,
+                            w.row_lo, w.row_hi, w.kv_lo, w.kv_hi, w.lo_max,
+                            w.hi_min, st));
   LWM_TRY(launch_lpt_order(B, (Nq + kBlock - 1) / kBlock, kFwdBlocksPerUnit,
                            w.kv_lo, w.kv_hi, w.sort_keys, w.order_fwd,
                            w.counter, st));
@@ -209,6 +213,7 @@ int run_forward(const void* q, const void* k_rot, const void* k_rot_lo,
   a.row_hi = w.row_hi; a.lo_max = w.lo_max; a.hi_min = w.hi_min;
   a.order = w.order_fwd; a.counter = w.counter;
   a.B = B; a.Nq = Nq; a.Nk = Nk; a.H = H; a.k_off = k_off;
+  a.block_k = block_k;
   a.qk_x3 = x3;
   a.rope_half = half;
   a.status = status_word();
@@ -388,7 +393,7 @@ int lwm_blockattn_fwd(const void* q, const void* k, const void* v,
   LWM_TRY(launch_rope_apply(k, positions, w.table, B, N, H, half, w.k_rot,
                             w.k_rot_lo, st));
   return run_forward(q, w.k_rot, w.k_rot_lo, v, segment_ids, positions,
-                     segment_ids, 0, 0, B, N, N, H,
+                     segment_ids, 0, 0, B, N, N, H, block_k,
                      qk_precision == LWM_QK_BF16X3, half, out, lse, w, st);
 }
 
@@ -440,8 +445,8 @@ int lwm_blockattn_fwd_block(const void* q, const void* k_rot, const void* v,
     LWM_TRY(launch_rope_table(theta, D, max_pos, w.table, st));
   }
   return run_forward(q, k_rot, nullptr, v, seg_q, pos_q, seg_k, q_off, k_off,
-                     B, Nq, Nk, H, false, rope_layout == LWM_ROPE_HALF, out,
-                     lse, w, st);
+                     B, Nq, Nk, H, kBlock, false, rope_layout == LWM_ROPE_HALF,
+                     out, lse, w, st);
 }
 
 int lwm_blockattn_merge(void* out, float* lse, const void* out_part,
@@ -731,7 +736,8 @@ int lwm_blockattn_visibility(const int32_t* seg_q, const int32_t* seg_k,
       (int64_t(B) * Nq) >= (int64_t(1) << 31) ||
       (int64_t(B) * Nk) >= (int64_t(1) << 31))
     return LWM_ERR_INVALID_ARG;
-  if (block_q != kBlock || block_k != kBlock) return LWM_ERR_UNSUPPORTED;
+  if (shape_status(kHeadDim, block_q, block_k) != LWM_OK)
+    return LWM_ERR_UNSUPPORTED;
   int32_t* qside[] = {row_lo, row_hi, kv_lo, kv_hi, lo_max, hi_min};
   int32_t* kside[] = {col_lo, col_hi, q_lo, q_hi, klo_max, khi_min};
   // each view is written whole or not at all
@@ -742,14 +748,18 @@ int lwm_blockattn_visibility(const int32_t* seg_q, const int32_t* seg_k,
   };
   const int nq = group(qside), nk = group(kside);
   if ((nq != 0 && nq != 6) || (nk != 0 && nk != 6)) return LWM_ERR_INVALID_ARG;
+  // the backward's key view is in 128-key units whatever the forward's key
+  // block height
+  if (nk && block_k != kBlock) return LWM_ERR_UNSUPPORTED;
   if (int64_t(B) * Nq * Nk == 0 || (nq == 0 && nk == 0)) return LWM_OK;
   if (!seg_q || !seg_k) return LWM_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // the very launches lwm_blockattn_fwd / _fwd_block and lwm_blockattn_bwd /
   // _bwd_block make before their attention kernels
   if (nq)
-    LWM_TRY(launch_cross_meta(seg_q, seg_k, B, Nq, Nk, q_off, k_off, row_lo,
-                              row_hi, kv_lo, kv_hi, lo_max, hi_min, st));
+    LWM_TRY(launch_cross_meta(seg_q, seg_k, B, Nq, Nk, q_off, k_off, block_k,
+                              row_lo, row_hi, kv_lo, kv_hi, lo_max, hi_min,
+                              st));
   if (nk)
     LWM_TRY(launch_cross_meta_keys(seg_q, seg_k, B, Nq, Nk, q_off, k_off,
                                    col_lo, col_hi, q_lo, q_hi, klo_max,

@@ -620,8 +620,9 @@ cudaError_t launch_rope_apply(const void* x, const int32_t* pos,
 
 cudaError_t launch_cross_meta(const int32_t* seg_q, const int32_t* seg_k,
                               int B, int Nq, int Nk, int q_off, int k_off,
-                              int32_t* row_lo, int32_t* row_hi, int32_t* kv_lo,
-                              int32_t* kv_hi, int32_t* lo_max, int32_t* hi_min,
+                              int bk, int32_t* row_lo, int32_t* row_hi,
+                              int32_t* kv_lo, int32_t* kv_hi,
+                              int32_t* lo_max, int32_t* hi_min,
                               cudaStream_t st) {
   const int64_t n = int64_t(B) * Nq;
   if (n == 0) return cudaSuccess;
@@ -630,7 +631,7 @@ cudaError_t launch_cross_meta(const int32_t* seg_q, const int32_t* seg_k,
   note_launch();
   const int Tq = (Nq + kBlock - 1) / kBlock;
   cross_tiles_kernel<<<(B * Tq + 127) / 128, 128, 0, st>>>(
-      row_lo, row_hi, B, Nq, Nk, k_off, kBlock, kBlock, Tq, kv_lo, kv_hi,
+      row_lo, row_hi, B, Nq, Nk, k_off, kBlock, bk, Tq, kv_lo, kv_hi,
       lo_max, hi_min);
   note_launch();
   return cudaGetLastError();

@@ -19,10 +19,13 @@ cudaError_t launch_rope_apply(const void* x, const int32_t* pos,
 // Per-row visible key ranges of queries [q_off, q_off+Nq) against keys
 // [k_off, k_off+Nk) (global indices), and per query block the key-block
 // range plus the shared row range used for the all-visible test.
+// kv_lo / kv_hi count key blocks of bk keys (128 or 64); query blocks are
+// 128 rows.
 cudaError_t launch_cross_meta(const int32_t* seg_q, const int32_t* seg_k,
                               int B, int Nq, int Nk, int q_off, int k_off,
-                              int32_t* row_lo, int32_t* row_hi, int32_t* kv_lo,
-                              int32_t* kv_hi, int32_t* lo_max, int32_t* hi_min,
+                              int bk, int32_t* row_lo, int32_t* row_hi,
+                              int32_t* kv_lo, int32_t* kv_hi,
+                              int32_t* lo_max, int32_t* hi_min,
                               cudaStream_t st);
 // Key-side metadata of the same pair of ranges for the key-major backward:
 // per key the queries that see it (global indices), per key block the query

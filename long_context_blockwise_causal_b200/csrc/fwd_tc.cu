@@ -43,16 +43,20 @@ constexpr int kHalfTileBytes = kTileBytes / 2;          // one 64-wide d chunk
 constexpr uint64_t kWaitLimitNs = 4000000000ull;        // 4 s per wait
 constexpr float kRescaleThreshold = 8.0f;               // log2 units
 
-template <bool X3>
+// BK: keys per key block (the key tile the forward sweeps), 128 or 64.
+template <bool X3, int BK>
 struct FwdCfg {
-  static constexpr int KS = X3 ? 1 : 2;   // K stages
-  static constexpr int VS = X3 ? 1 : 2;   // V stages
+  static_assert(BK == 128 || BK == 64, "key blocks of 128 or 64 keys");
+  static constexpr int kKVTile = BK * kHeadDim * 2;   // one K or V tile
+  static constexpr int kKVHalf = kKVTile / 2;         // one 64-wide d chunk
+  static constexpr int KS = BK == 128 ? (X3 ? 1 : 2) : (X3 ? 2 : 4);
+  static constexpr int VS = KS;
   static constexpr int kQ = 0;
   static constexpr int kQlo = kQ + 2 * kTileBytes;
   static constexpr int kK = kQlo + (X3 ? 2 * kTileBytes : 0);
-  static constexpr int kKlo = kK + KS * kTileBytes;
-  static constexpr int kV = kKlo + (X3 ? KS * kTileBytes : 0);
-  static constexpr int kBars = kV + VS * kTileBytes;
+  static constexpr int kKlo = kK + KS * kKVTile;
+  static constexpr int kV = kKlo + (X3 ? KS * kKVTile : 0);
+  static constexpr int kBars = kV + VS * kKVTile;
   // barrier slots
   static constexpr int bQFull = 0, bQReady = 2, bQEmpty = 4, bSFull = 6,
                        bPFull = 8, bOFull = 10, bOEmpty = 12, bEpi = 14,
@@ -62,6 +66,7 @@ struct FwdCfg {
                        kNumBars = bVEmpty + VS;
   static constexpr int kMisc = kBars + kNumBars * 8;
   static constexpr int kSmem = kMisc + 32 + 1024;  // + alignment slack
+  static_assert(kSmem <= 232448, "shared memory per CTA");
 };
 
 struct FwdParams {
@@ -267,7 +272,7 @@ __device__ __forceinline__ const float4* rope_prefetch(
   return trow;
 }
 
-template <bool X3>
+template <bool X3, int BK>
 __global__ void __launch_bounds__(kThreadsFwd, 1)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
               const __grid_constant__ CUtensorMap tm_k,
@@ -275,7 +280,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
               const __grid_constant__ CUtensorMap tm_o,
               const __grid_constant__ CUtensorMap tm_klo,
               const FwdParams p) {
-  using C = FwdCfg<X3>;
+  using C = FwdCfg<X3, BK>;
+  constexpr int NC = BK / 32;   // 32-column chunks of an S row
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -382,27 +388,27 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (!ok) break;
         sc++;
         tc_fence_after();
-        const int k0 = p.k_off + j * kBlock;  // global index of key 0
+        const int k0 = p.k_off + j * BK;  // global index of key 0
         // every pair of the tile allowed: every row of the block sees the
         // whole key block
-        const bool full = lo_max <= k0 && hi_min >= k0 + kBlock - 1;
-        // the whole 128-column S row of this thread in registers
-        uint32_t v[4][32];
+        const bool full = lo_max <= k0 && hi_min >= k0 + BK - 1;
+        // the whole S row of this thread (BK columns) in registers
+        uint32_t v[NC][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, v[c]);
+        for (int c = 0; c < NC; ++c) tmem_ld32(tS + c * 32, v[c]);
         tmem_wait_ld();
         if (!full) {  // mask: keep lo_i <= key <= hi_i
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
+          for (int c = 0; c < NC; ++c) {
             const int lo = lo_i - (k0 + c * 32), hi = hi_i - (k0 + c * 32);
 #pragma unroll
             for (int x = 0; x < 32; ++x)
               v[c][x] = (x >= lo && x <= hi) ? v[c][x] : 0xff800000u;
           }
         }
-        float mc[4];
+        float mc[NC];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < NC; ++c) {
           mc[c] = __uint_as_float(v[c][0]);
 #pragma unroll
           for (int x = 1; x < 31; x += 2)
@@ -410,7 +416,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                          __uint_as_float(v[c][x + 1]));
           mc[c] = fmaxf(mc[c], __uint_as_float(v[c][31]));
         }
-        const float mx = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
+        float mx = mc[0];
+#pragma unroll
+        for (int c = 1; c < NC; ++c) mx = fmaxf(mx, mc[c]);
         const float m_tile = mx * p.scale_log2;
         float m_new = m_used;
         bool rescale = false;
@@ -421,12 +429,14 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         const float alpha = rescale ? ex2(m_used - m_new) : 1.f;
         l *= alpha;
         const float sub = m_new == -INFINITY ? 0.f : m_new;
-        // P = 2^(S*c - m) (bf16, over S columns [0, 64)), row sum in fp32
+        // P = 2^(S*c - m) (bf16, over S columns [0, BK/2)), row sum in
+        // fp32; a row that has seen no key yet keeps m = -inf and gets
+        // P = 0 (the subtrahend is 0, its scores are -inf)
         const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
         const float2 nsub2 = make_float2(-sub, -sub);
         float2 lsum = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < NC; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int x = 0; x < 32; x += 2) {
@@ -598,19 +608,18 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             ok = mbar_wait(bar(C::bKEmpty + ks), ((kfill / C::KS) - 1) & 1,
                            abort_flag, p.status, kWaitLimitNs);
           if (!ok) break;
-          uint32_t kd = sbase + C::kK + ks * kTileBytes;
+          uint32_t kd = sbase + C::kK + ks * C::kKVTile;
           mbar_arrive_expect_tx(bar(C::bKFull + ks),
-                                X3 ? 2 * kTileBytes : kTileBytes);
-          tma_load_4d(kd, &tm_k, bar(C::bKFull + ks), 0, m.h, j * kBlock,
-                      m.b);
-          tma_load_4d(kd + kHalfTileBytes, &tm_k, bar(C::bKFull + ks), 64,
-                      m.h, j * kBlock, m.b);
+                                X3 ? 2 * C::kKVTile : C::kKVTile);
+          tma_load_4d(kd, &tm_k, bar(C::bKFull + ks), 0, m.h, j * BK, m.b);
+          tma_load_4d(kd + C::kKVHalf, &tm_k, bar(C::bKFull + ks), 64, m.h,
+                      j * BK, m.b);
           if (X3) {
-            uint32_t kl = sbase + C::kKlo + ks * kTileBytes;
-            tma_load_4d(kl, &tm_klo, bar(C::bKFull + ks), 0, m.h,
-                        j * kBlock, m.b);
-            tma_load_4d(kl + kHalfTileBytes, &tm_klo, bar(C::bKFull + ks),
-                        64, m.h, j * kBlock, m.b);
+            uint32_t kl = sbase + C::kKlo + ks * C::kKVTile;
+            tma_load_4d(kl, &tm_klo, bar(C::bKFull + ks), 0, m.h, j * BK,
+                        m.b);
+            tma_load_4d(kl + C::kKVHalf, &tm_klo, bar(C::bKFull + ks), 64,
+                        m.h, j * BK, m.b);
           }
           kfill++;
           int vs = vfill % C::VS;
@@ -618,12 +627,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             ok = mbar_wait(bar(C::bVEmpty + vs), ((vfill / C::VS) - 1) & 1,
                            abort_flag, p.status, kWaitLimitNs);
           if (!ok) break;
-          uint32_t vd = sbase + C::kV + vs * kTileBytes;
-          mbar_arrive_expect_tx(bar(C::bVFull + vs), kTileBytes);
-          tma_load_4d(vd, &tm_v, bar(C::bVFull + vs), 0, m.h, j * kBlock,
-                      m.b);
-          tma_load_4d(vd + kHalfTileBytes, &tm_v, bar(C::bVFull + vs), 64,
-                      m.h, j * kBlock, m.b);
+          uint32_t vd = sbase + C::kV + vs * C::kKVTile;
+          mbar_arrive_expect_tx(bar(C::bVFull + vs), C::kKVTile);
+          tma_load_4d(vd, &tm_v, bar(C::bVFull + vs), 0, m.h, j * BK, m.b);
+          tma_load_4d(vd + C::kKVHalf, &tm_v, bar(C::bVFull + vs), 64, m.h,
+                      j * BK, m.b);
           vfill++;
         }
       }
@@ -643,12 +651,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     } else if (warp == 13) {
     // ------------------------------------------------ tcgen05 issuer
     if (lane == 0) {
-      const uint32_t idS = idesc_bf16(128, 128, 0, 0);
+      const uint32_t idS = idesc_bf16(128, BK, 0, 0);
       const uint32_t idPV = idesc_bf16(128, 128, 0, 1);
       // SW128 descriptors at shared-memory offset 0: K-major (Q, K tiles)
-      // and MN-major with the 64-wide d chunks 16 KB apart (V tiles)
+      // and MN-major with the 64-wide d chunks BK * 128 bytes apart (V)
       const uint64_t kdesc0 = sdesc_sw128(sbase, 16, 1024);
-      const uint64_t vdesc0 = sdesc_sw128(sbase + C::kV, kHalfTileBytes, 1024);
+      const uint64_t vdesc0 = sdesc_sw128(sbase + C::kV, C::kKVHalf, 1024);
       int kc = 0, vc = 0;
       int qc[2] = {0, 0}, pc[2] = {0, 0}, oc[2] = {0, 0};
       bool ok = true;
@@ -665,14 +673,14 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         int prev = -1;
         for (int j = m.jhi; j >= m.jlo - 1 && ok; --j) {
           const bool has_j = j >= m.jlo;
-          int ks = kc % C::KS;
+          const int ks = kc % C::KS;
+          const int vs = vc % C::VS;
           if (has_j) {
             ok = mbar_wait(bar(C::bKFull + ks), (kc / C::KS) & 1, abort_flag,
                            p.status, kWaitLimitNs);
             if (!ok) break;
             tc_fence_after();
           }
-          int vs = vc % C::VS;
           if (prev >= 0) {
             ok = mbar_wait(bar(C::bVFull + vs), (vc / C::VS) & 1, abort_flag,
                            p.status, kWaitLimitNs);
@@ -695,11 +703,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
               // descriptor start fields are addr >> 4 in the low 14 bits;
               // offsets inside shared memory never carry out of them
               const uint64_t vdesc =
-                  vdesc0 + uint64_t((vs * kTileBytes) >> 4);
+                  vdesc0 + uint64_t((vs * C::kKVTile) >> 4);
               const uint32_t a_tm = tmem + s * 128;        // P over S_s
               const uint32_t d_tm = tmem + 256 + s * 128;  // O_s
 #pragma unroll
-              for (int k = 0; k < 8; ++k)
+              for (int k = 0; k < BK / 16; ++k)
                 mma_ts(d_tm, a_tm + k * 8, vdesc + uint64_t(k * (2048 >> 4)),
                        idPV, (pv_started[s] || k > 0) ? 1u : 0u);
               pv_started[s] = true;
@@ -714,7 +722,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 tc_fence_after();
               }
               const uint64_t qd = kdesc0 + uint64_t((C::kQ + s * kTileBytes) >> 4);
-              const uint64_t kd = kdesc0 + uint64_t((C::kK + ks * kTileBytes) >> 4);
+              const uint64_t kd = kdesc0 + uint64_t((C::kK + ks * C::kKVTile) >> 4);
               const uint32_t d_tm = tmem + s * 128;
               const int npass = X3 ? 3 : 1;
 #pragma unroll
@@ -726,9 +734,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                     kd + uint64_t(pass == 1 ? (C::kKlo - C::kK) >> 4 : 0);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                  const uint64_t off =
+                  // 16 of d: the 32-byte step inside a 128-byte row, the
+                  // 64-wide d chunks a tile apart (Q: 128 rows, K: BK rows)
+                  const uint64_t qo =
                       uint64_t(((k >> 2) * kHalfTileBytes + (k & 3) * 32) >> 4);
-                  mma_ss(d_tm, qa + off, ka + off, idS,
+                  const uint64_t ko =
+                      uint64_t(((k >> 2) * C::kKVHalf + (k & 3) * 32) >> 4);
+                  mma_ss(d_tm, qa + qo, ka + ko, idS,
                          (pass > 0 || k > 0) ? 1u : 0u);
                 }
               }
@@ -805,9 +817,10 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-// [B][N][H][D] bf16 tensor as a 4-D map {D, H, N, B}; box 64 x 1 x 128 x 1
-// with the 128-byte swizzle (one 64-wide d chunk of 128 rows per copy).
-bool make_bnhd_map(CUtensorMap* m, const void* base, int B, int N, int H) {
+// [B][N][H][D] bf16 tensor as a 4-D map {D, H, N, B}; box 64 x 1 x rows x 1
+// with the 128-byte swizzle (one 64-wide d chunk of `rows` rows per copy).
+bool make_bnhd_map(CUtensorMap* m, const void* base, int B, int N, int H,
+                   int rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[4] = {cuuint64_t(kHeadDim), cuuint64_t(H), cuuint64_t(N),
@@ -815,7 +828,7 @@ bool make_bnhd_map(CUtensorMap* m, const void* base, int B, int N, int H) {
   cuuint64_t strides[3] = {cuuint64_t(kHeadDim) * 2,
                            cuuint64_t(H) * kHeadDim * 2,
                            cuuint64_t(N) * H * kHeadDim * 2};
-  cuuint32_t box[4] = {64, 1, cuuint32_t(kBlock), 1};
+  cuuint32_t box[4] = {64, 1, cuuint32_t(rows), 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
                    const_cast<void*>(base), dims, strides, box, estr,
@@ -880,14 +893,14 @@ int sm_count() {
   return n;
 }
 
-template <bool X3>
+template <bool X3, int BK>
 static cudaError_t launch_fwd_impl(const FwdArgs& a, cudaStream_t st) {
   CUtensorMap mq, mk, mv, mo, mklo;
   if (!make_bnhd_map(&mq, a.q, a.B, a.Nq, a.H) ||
-      !make_bnhd_map(&mk, a.k_rot, a.B, a.Nk, a.H) ||
-      !make_bnhd_map(&mv, a.v, a.B, a.Nk, a.H) ||
       !make_bnhd_map(&mo, a.out, a.B, a.Nq, a.H) ||
-      !make_bnhd_map(&mklo, X3 ? a.k_rot_lo : a.k_rot, a.B, a.Nk, a.H))
+      !make_bnhd_map(&mk, a.k_rot, a.B, a.Nk, a.H, BK) ||
+      !make_bnhd_map(&mv, a.v, a.B, a.Nk, a.H, BK) ||
+      !make_bnhd_map(&mklo, X3 ? a.k_rot_lo : a.k_rot, a.B, a.Nk, a.H, BK))
     return cudaErrorInvalidValue;
   FwdParams p{};
   p.counter = a.counter;
@@ -917,27 +930,32 @@ static cudaError_t launch_fwd_impl(const FwdArgs& a, cudaStream_t st) {
     if (a.H % g == 0) { p.G = g; break; }
   p.total_items = a.B * p.U * a.H;
   p.scale_log2 = kLog2e / sqrtf(float(kHeadDim));
-  constexpr int smem = FwdCfg<X3>::kSmem;
+  constexpr int smem = FwdCfg<X3, BK>::kSmem;
   // setmaxnreg hands out exactly the registers the block was launched with;
   // refuse to launch a build whose allocation differs (it could wait
   // forever for registers that do not exist).
   cudaFuncAttributes fa;
-  cudaError_t e = cudaFuncGetAttributes(&fa, fwd_tc_kernel<X3>);
+  cudaError_t e = cudaFuncGetAttributes(&fa, fwd_tc_kernel<X3, BK>);
   if (e != cudaSuccess) return e;
   if (fa.numRegs != 128) return cudaErrorInvalidConfiguration;
-  e = cudaFuncSetAttribute(
-      fwd_tc_kernel<X3>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  e = cudaFuncSetAttribute(fwd_tc_kernel<X3, BK>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int grid = std::min(sm_count(), p.total_items);
-  fwd_tc_kernel<X3><<<grid, kThreadsFwd, smem, st>>>(mq, mk, mv, mo, mklo,
-                                                      p);
+  fwd_tc_kernel<X3, BK><<<grid, kThreadsFwd, smem, st>>>(mq, mk, mv, mo, mklo,
+                                                          p);
   note_launch();
   return cudaGetLastError();
 }
 
 cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t st) {
   if (a.B == 0 || a.Nq == 0 || a.Nk == 0 || a.H == 0) return cudaSuccess;
-  return a.qk_x3 ? launch_fwd_impl<true>(a, st) : launch_fwd_impl<false>(a, st);
+  if (a.block_k == 64)
+    return a.qk_x3 ? launch_fwd_impl<true, 64>(a, st)
+                   : launch_fwd_impl<false, 64>(a, st);
+  if (a.block_k != kBlock) return cudaErrorInvalidValue;
+  return a.qk_x3 ? launch_fwd_impl<true, 128>(a, st)
+                 : launch_fwd_impl<false, 128>(a, st);
 }
 
 }  // namespace lwm

@@ -35,6 +35,8 @@ struct FwdArgs {
   const int32_t* order;
   int32_t* counter;        // zeroed work counter (units handed out in order)
   int B, Nq, Nk, H, k_off;
+  int block_k;             // keys per key block: 128 or 64 (kv_lo / kv_hi
+                           // count key blocks of this height)
   bool qk_x3;
   bool rope_half;          // q (and k_rot) in the rotate-half layout
   int* status;
@@ -77,9 +79,10 @@ struct BwdArgs {
 };
 
 cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t st);
-// 4-D TMA map over a bf16 [B][N][H][128] tensor, box 64 x 1 x 128 x 1,
+// 4-D TMA map over a bf16 [B][N][H][128] tensor, box 64 x 1 x rows x 1,
 // 128-byte swizzle. False if the driver's encoder is unavailable/refuses.
-bool make_bnhd_map(CUtensorMap* m, const void* base, int B, int N, int H);
+bool make_bnhd_map(CUtensorMap* m, const void* base, int B, int N, int H,
+                   int rows = kBlock);
 // 4-D TMA map over an fp32 [B][N][H][128] tensor, box 32 x 1 x 32 x 1,
 // 128-byte swizzle (used for the dQ reduce-add).
 bool make_bnhd_f32_map(CUtensorMap* m, const void* base, int B, int N,

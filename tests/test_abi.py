@@ -91,7 +91,8 @@ def _fwd_raw(**kw):
     ({"max_pos": 0}, ops.ERR_INVALID_ARG),
     ({"D": 64}, ops.ERR_UNSUPPORTED),
     ({"bq": 64}, ops.ERR_UNSUPPORTED),
-    ({"bk": 64}, ops.ERR_UNSUPPORTED),
+    ({"bk": 32}, ops.ERR_UNSUPPORTED),
+    ({"bk": 256}, ops.ERR_UNSUPPORTED),
     ({"wsb": 100}, ops.ERR_WORKSPACE),
     ({"N": 0, "q": None}, ops.OK),                    # empty: no work
     ({"H": 0}, ops.OK),
@@ -116,6 +117,8 @@ def test_visibility_rejects_bad_arguments_before_launch():
     # a view given in part is refused (it would leave the rest unwritten)
     assert call([p, None] + [p] * 4, none6) == ops.ERR_INVALID_ARG
     assert call(none6, [p] * 5 + [None]) == ops.ERR_INVALID_ARG
+    assert call(six, six, bk=32) == ops.ERR_UNSUPPORTED
+    # 64-key blocks: the forward's query view only
     assert call(six, six, bk=64) == ops.ERR_UNSUPPORTED
     assert call(six, six, q_off=-1) == ops.ERR_INVALID_ARG
     assert call(six, six, Nk=-3) == ops.ERR_INVALID_ARG
@@ -140,8 +143,9 @@ def test_noalloc_checks_arguments_before_its_scratch_size():
                                            p, p, None)
 
     assert call() == ops.ERR_WORKSPACE              # valid, too large
+    assert call(bk=64) == ops.ERR_WORKSPACE         # 64-key blocks: valid
     assert call(D=64) == ops.ERR_UNSUPPORTED
-    assert call(bk=64) == ops.ERR_UNSUPPORTED
+    assert call(bk=32) == ops.ERR_UNSUPPORTED
     assert call(dtype=9) == ops.ERR_INVALID_ARG
     assert call(qkp=4) == ops.ERR_INVALID_ARG
     assert call(layout=3) == ops.ERR_INVALID_ARG
