@@ -321,10 +321,12 @@ int lwm_blockattn_decode(const void* q, const void* k_rot, const void* v,
   float* part_l = reinterpret_cast<float*>(ws + align_up(slots * sizeof(float)));
   float* part_acc =
       reinterpret_cast<float*>(ws + 2 * align_up(slots * sizeof(float)));
+  int* st = status_word();
+  if (!st) return LWM_ERR_CUDA;
   return cuda_status(launch_decode(q, k_rot, v, kv_start, kv_len, q_pos,
                                    rope_table, max_pos, B, L, H,
                                    rope_layout == LWM_ROPE_HALF, out, lse,
-                                   part_m, part_l, part_acc,
+                                   part_m, part_l, part_acc, st,
                                    static_cast<cudaStream_t>(stream)));
 }
 

@@ -80,6 +80,14 @@ def test_decode_short_and_single_key(cuda_dev):
     _decode_check(t, [300, 1])           # every token its own example
 
 
+def test_decode_several_chunks_ragged(cuda_dev):
+    # caches of 20000 keys: three chunks per (row, head), each streamed in
+    # 128-key steps with a ragged last step; the rows' examples start at
+    # different offsets, so chunks of one row begin mid-step
+    t = _case(20000, 3, 3, 6, lo=1, hi=14000)
+    _decode_check(t, [20000, 16385, 9001])
+
+
 def test_decode_empty_range(cuda_dev):
     t = _case(256, 2, 1, 4, seg_kind="single")
     mp = 256
