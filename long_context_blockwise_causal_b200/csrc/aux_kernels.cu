@@ -147,6 +147,41 @@ __global__ void row_start_kernel(const int32_t* __restrict__ seg, int B, int N,
 // token indices: row i (global q_off + ii) sees the keys of the block whose
 // segment id equals its own and whose index is <= i. With non-decreasing
 // ids those keys are contiguous: [row_lo, row_hi] (empty when lo > hi).
+// Range summary of one 128-row block (rows or keys), one warp per block:
+// each lane folds every 32nd entry, then the warp combines. mn / mx: union
+// of the non-empty ranges; lmax / hmin: their intersection; all: every
+// entry exists and is non-empty.
+struct RangeFold {
+  int mn, mx, lmax, hmin;
+  bool all;
+};
+
+__device__ __forceinline__ RangeFold fold_ranges(const int32_t* __restrict__ lo_v,
+                                                 const int32_t* __restrict__ hi_v,
+                                                 int first, int count, int n,
+                                                 int lane) {
+  RangeFold f{0x7fffffff, -1, -0x7fffffff, 0x7fffffff, true};
+  for (int r = lane; r < count; r += 32) {
+    const int ii = first + r;
+    if (ii >= n) { f.all = false; continue; }
+    const int lo = lo_v[ii], hi = hi_v[ii];
+    if (lo > hi) { f.all = false; continue; }
+    f.mn = min(f.mn, lo);
+    f.mx = max(f.mx, hi);
+    f.lmax = max(f.lmax, lo);
+    f.hmin = min(f.hmin, hi);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    f.mn = min(f.mn, __shfl_xor_sync(0xffffffffu, f.mn, o));
+    f.mx = max(f.mx, __shfl_xor_sync(0xffffffffu, f.mx, o));
+    f.lmax = max(f.lmax, __shfl_xor_sync(0xffffffffu, f.lmax, o));
+    f.hmin = min(f.hmin, __shfl_xor_sync(0xffffffffu, f.hmin, o));
+  }
+  f.all = __all_sync(0xffffffffu, f.all);
+  return f;
+}
+
 __global__ void cross_rows_kernel(const int32_t* __restrict__ seg_q,
                                   const int32_t* __restrict__ seg_k, int B,
                                   int Nq, int Nk, int q_off, int k_off,
@@ -181,30 +216,24 @@ __global__ void cross_tiles_kernel(const int32_t* __restrict__ row_lo,
                                    int32_t* __restrict__ kv_hi,
                                    int32_t* __restrict__ lo_max,
                                    int32_t* __restrict__ hi_min) {
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  // one warp per query block (the whole warp leaves together)
+  const int e = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
   if (e >= B * Tq) return;
   const int b = e / Tq, t = e - b * Tq;
-  int mn = 0x7fffffff, mx = -1, lmax = -0x7fffffff, hmin = 0x7fffffff;
-  bool all = true;
-  for (int r = 0; r < bq; ++r) {
-    const int ii = t * bq + r;
-    if (ii >= Nq) { all = false; break; }
-    const int lo = row_lo[int64_t(b) * Nq + ii], hi = row_hi[int64_t(b) * Nq + ii];
-    if (lo > hi) { all = false; continue; }
-    mn = min(mn, lo);
-    mx = max(mx, hi);
-    lmax = max(lmax, lo);
-    hmin = min(hmin, hi);
-  }
-  if (mx < 0 || mn > mx) {
+  const RangeFold f = fold_ranges(row_lo + int64_t(b) * Nq,
+                                  row_hi + int64_t(b) * Nq, t * bq, bq, Nq,
+                                  lane);
+  if (lane != 0) return;
+  if (f.mx < 0 || f.mn > f.mx) {
     kv_lo[e] = 1;
     kv_hi[e] = 0;
   } else {
-    kv_lo[e] = (mn - k_off) / bk;
-    kv_hi[e] = min((mx - k_off) / bk, (Nk - 1) / bk);
+    kv_lo[e] = (f.mn - k_off) / bk;
+    kv_hi[e] = min((f.mx - k_off) / bk, (Nk - 1) / bk);
   }
-  lo_max[e] = all ? lmax : 0x7fffffff;
-  hi_min[e] = all ? hmin : -0x7fffffff;
+  lo_max[e] = f.all ? f.lmax : 0x7fffffff;
+  hi_min[e] = f.all ? f.hmin : -0x7fffffff;
 }
 
 // Key-side view of the same rule, for the key-major backward: key k
@@ -243,30 +272,24 @@ __global__ void cross_kblocks_kernel(const int32_t* __restrict__ col_lo,
                                      int32_t* __restrict__ q_hi,
                                      int32_t* __restrict__ klo_max,
                                      int32_t* __restrict__ khi_min) {
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  // one warp per key block (the whole warp leaves together)
+  const int e = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
   if (e >= B * Tk) return;
   const int b = e / Tk, j = e - b * Tk;
-  int mn = 0x7fffffff, mx = -1, lmax = -0x7fffffff, hmin = 0x7fffffff;
-  bool all = true;
-  for (int r = 0; r < kBlock; ++r) {
-    const int jj = j * kBlock + r;
-    if (jj >= Nk) { all = false; break; }
-    const int lo = col_lo[int64_t(b) * Nk + jj], hi = col_hi[int64_t(b) * Nk + jj];
-    if (lo > hi) { all = false; continue; }
-    mn = min(mn, lo);
-    mx = max(mx, hi);
-    lmax = max(lmax, lo);
-    hmin = min(hmin, hi);
-  }
-  if (mx < 0 || mn > mx) {
+  const RangeFold f = fold_ranges(col_lo + int64_t(b) * Nk,
+                                  col_hi + int64_t(b) * Nk, j * kBlock,
+                                  kBlock, Nk, lane);
+  if (lane != 0) return;
+  if (f.mx < 0 || f.mn > f.mx) {
     q_lo[e] = 1;
     q_hi[e] = 0;
   } else {
-    q_lo[e] = (mn - q_off) / kBlock;
-    q_hi[e] = min((mx - q_off) / kBlock, (Nq - 1) / kBlock);
+    q_lo[e] = (f.mn - q_off) / kBlock;
+    q_hi[e] = min((f.mx - q_off) / kBlock, (Nq - 1) / kBlock);
   }
-  klo_max[e] = all ? lmax : 0x7fffffff;
-  khi_min[e] = all ? hmin : -0x7fffffff;
+  klo_max[e] = f.all ? f.lmax : 0x7fffffff;
+  khi_min[e] = f.all ? f.hmin : -0x7fffffff;
 }
 
 // out, lse <- the softmax-weighted combination of (out, lse) and
@@ -630,7 +653,7 @@ cudaError_t launch_cross_meta(const int32_t* seg_q, const int32_t* seg_k,
       seg_q, seg_k, B, Nq, Nk, q_off, k_off, row_lo, row_hi);
   note_launch();
   const int Tq = (Nq + kBlock - 1) / kBlock;
-  cross_tiles_kernel<<<(B * Tq + 127) / 128, 128, 0, st>>>(
+  cross_tiles_kernel<<<(B * Tq + 3) / 4, 128, 0, st>>>(
       row_lo, row_hi, B, Nq, Nk, k_off, kBlock, bk, Tq, kv_lo, kv_hi,
       lo_max, hi_min);
   note_launch();
@@ -649,7 +672,7 @@ cudaError_t launch_cross_meta_keys(const int32_t* seg_q, const int32_t* seg_k,
       seg_q, seg_k, B, Nq, Nk, q_off, k_off, col_lo, col_hi);
   note_launch();
   const int Tk = (Nk + kBlock - 1) / kBlock;
-  cross_kblocks_kernel<<<(B * Tk + 127) / 128, 128, 0, st>>>(
+  cross_kblocks_kernel<<<(B * Tk + 3) / 4, 128, 0, st>>>(
       col_lo, col_hi, B, Nq, Nk, q_off, Tk, q_lo, q_hi, klo_max, khi_min);
   note_launch();
   return cudaGetLastError();
