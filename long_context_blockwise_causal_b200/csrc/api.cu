@@ -78,7 +78,6 @@ struct Workspace {
   int32_t* col_lo;       // [B][Nk]
   int32_t* col_hi;
   int32_t* order_bwd;    // [B*Tk]
-  uint64_t* sort_keys;   // [B*Uq] or [B*Tk]
   int32_t* counter;      // work counter of the attention kernel
   float* delta;          // [B][H][N]
   float* dq_acc;         // [B][N][H][D]
@@ -107,7 +106,6 @@ Workspace carve(void* base, int B, int Nq, int Nk, int H, int D, int max_pos,
     w.row_lo = c.take<int32_t>(size_t(B) * Nq);
     w.row_hi = c.take<int32_t>(size_t(B) * Nq);
     w.order_fwd = c.take<int32_t>(size_t(B) * Uq);
-    w.sort_keys = c.take<uint64_t>(size_t(B) * Uq);
   } else {
     w.q_lo = c.take<int32_t>(size_t(B) * Tk);
     w.q_hi = c.take<int32_t>(size_t(B) * Tk);
@@ -116,7 +114,6 @@ Workspace carve(void* base, int B, int Nq, int Nk, int H, int D, int max_pos,
     w.col_lo = c.take<int32_t>(size_t(B) * Nk);
     w.col_hi = c.take<int32_t>(size_t(B) * Nk);
     w.order_bwd = c.take<int32_t>(size_t(B) * Tk);
-    w.sort_keys = c.take<uint64_t>(size_t(B) * Tk);
   }
   w.counter = c.take<int32_t>(64);
   if (pass == Pass::kBwd) {
@@ -182,7 +179,7 @@ int run_backward(BwdArgs a, const int32_t* seg_q, const int32_t* seg_k,
                                  k_off, w.col_lo, w.col_hi, w.q_lo, w.q_hi,
                                  w.klo_max, w.khi_min, st));
   LWM_TRY(launch_lpt_order(a.B, (a.Nk + kBlock - 1) / kBlock,
-                           kBwdBlocksPerUnit, w.q_lo, w.q_hi, w.sort_keys,
+                           kBwdBlocksPerUnit, w.q_lo, w.q_hi,
                            w.order_bwd, w.counter, st));
   a.q_lo = w.q_lo; a.q_hi = w.q_hi; a.col_lo = w.col_lo; a.col_hi = w.col_hi;
   a.klo_max = w.klo_max; a.khi_min = w.khi_min;
@@ -204,7 +201,7 @@ int run_forward(const void* q, const void* k_rot, const void* k_rot_lo,
                             w.row_lo, w.row_hi, w.kv_lo, w.kv_hi, w.lo_max,
                             w.hi_min, st));
   LWM_TRY(launch_lpt_order(B, (Nq + kBlock - 1) / kBlock, kFwdBlocksPerUnit,
-                           w.kv_lo, w.kv_hi, w.sort_keys, w.order_fwd,
+                           w.kv_lo, w.kv_hi, w.order_fwd,
                            w.counter, st));
   FwdArgs a{};
   a.q = q; a.k_rot = k_rot; a.k_rot_lo = k_rot_lo; a.v = v;

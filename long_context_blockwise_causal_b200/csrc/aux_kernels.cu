@@ -147,84 +147,79 @@ __global__ void row_start_kernel(const int32_t* __restrict__ seg, int B, int N,
 // token indices: row i (global q_off + ii) sees the keys of the block whose
 // segment id equals its own and whose index is <= i. With non-decreasing
 // ids those keys are contiguous: [row_lo, row_hi] (empty when lo > hi).
-// Range summary of one 128-row block (rows or keys), one warp per block:
-// each lane folds every 32nd entry, then the warp combines. mn / mx: union
+// Range summary of one 128-row block (query rows or keys): mn / mx: union
 // of the non-empty ranges; lmax / hmin: their intersection; all: every
 // entry exists and is non-empty.
 struct RangeFold {
   int mn, mx, lmax, hmin;
   bool all;
+  __device__ __forceinline__ void add(int lo, int hi) {
+    if (lo > hi) { all = false; return; }
+    mn = min(mn, lo);
+    mx = max(mx, hi);
+    lmax = max(lmax, lo);
+    hmin = min(hmin, hi);
+  }
+  __device__ __forceinline__ void merge(const RangeFold& o) {
+    mn = min(mn, o.mn);
+    mx = max(mx, o.mx);
+    lmax = max(lmax, o.lmax);
+    hmin = min(hmin, o.hmin);
+    all = all && o.all;
+  }
+  __device__ __forceinline__ void warp_reduce() {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      lmax = max(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+      hmin = min(hmin, __shfl_xor_sync(0xffffffffu, hmin, o));
+    }
+    all = __all_sync(0xffffffffu, all);
+  }
 };
 
-__device__ __forceinline__ RangeFold fold_ranges(const int32_t* __restrict__ lo_v,
-                                                 const int32_t* __restrict__ hi_v,
-                                                 int first, int count, int n,
-                                                 int lane) {
+// Per query row i (global q_off + ii): the visible keys are those of its
+// segment up to the row itself, as a global index range [row_lo, row_hi]
+// (empty when lo > hi); and per query block t (one CTA of 128 threads, a
+// thread per row): the key blocks [kv_lo, kv_hi] (block-local) holding any
+// visible key (empty: lo = 1, hi = 0), and the tightest row range the
+// block shares (lo_max, hi_min; lo_max = INT_MAX if some row is past Nq or
+// sees nothing) for the all-visible test of a key block.
+__global__ void __launch_bounds__(kBlock)
+cross_meta_kernel(const int32_t* __restrict__ seg_q,
+                  const int32_t* __restrict__ seg_k, int B, int Nq, int Nk,
+                  int q_off, int k_off, int bk, int Tq,
+                  int32_t* __restrict__ row_lo, int32_t* __restrict__ row_hi,
+                  int32_t* __restrict__ kv_lo, int32_t* __restrict__ kv_hi,
+                  int32_t* __restrict__ lo_max, int32_t* __restrict__ hi_min) {
+  __shared__ RangeFold part[kBlock / 32];
+  const int e = blockIdx.x;
+  const int b = e / Tq, t = e - b * Tq;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int ii = t * kBlock + threadIdx.x;
   RangeFold f{0x7fffffff, -1, -0x7fffffff, 0x7fffffff, true};
-  for (int r = lane; r < count; r += 32) {
-    const int ii = first + r;
-    if (ii >= n) { f.all = false; continue; }
-    const int lo = lo_v[ii], hi = hi_v[ii];
-    if (lo > hi) { f.all = false; continue; }
-    f.mn = min(f.mn, lo);
-    f.mx = max(f.mx, hi);
-    f.lmax = max(f.lmax, lo);
-    f.hmin = min(f.hmin, hi);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    f.mn = min(f.mn, __shfl_xor_sync(0xffffffffu, f.mn, o));
-    f.mx = max(f.mx, __shfl_xor_sync(0xffffffffu, f.mx, o));
-    f.lmax = max(f.lmax, __shfl_xor_sync(0xffffffffu, f.lmax, o));
-    f.hmin = min(f.hmin, __shfl_xor_sync(0xffffffffu, f.hmin, o));
-  }
-  f.all = __all_sync(0xffffffffu, f.all);
-  return f;
-}
-
-__global__ void cross_rows_kernel(const int32_t* __restrict__ seg_q,
-                                  const int32_t* __restrict__ seg_k, int B,
-                                  int Nq, int Nk, int q_off, int k_off,
-                                  int32_t* __restrict__ row_lo,
-                                  int32_t* __restrict__ row_hi) {
-  int64_t total = int64_t(B) * Nq;
-  for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < total;
-       e += int64_t(gridDim.x) * blockDim.x) {
-    const int b = int(e / Nq);
-    const int ii = int(e - int64_t(b) * Nq);
+  if (ii < Nq) {
     const int32_t* sk = seg_k + int64_t(b) * Nk;
-    const int v = seg_q[e];
+    const int v = seg_q[int64_t(b) * Nq + ii];
     int a = 0, z = Nk;  // first key with seg >= v
     while (a < z) { int m = (a + z) >> 1; if (sk[m] < v) a = m + 1; else z = m; }
-    int lo = a;
+    const int first = a;
     z = Nk;             // first key with seg > v
     while (a < z) { int m = (a + z) >> 1; if (sk[m] <= v) a = m + 1; else z = m; }
-    const int hi_seg = a - 1;
-    row_lo[e] = k_off + lo;
-    row_hi[e] = min(k_off + hi_seg, q_off + ii);
+    const int lo = k_off + first;
+    const int hi = min(k_off + a - 1, q_off + ii);
+    row_lo[int64_t(b) * Nq + ii] = lo;
+    row_hi[int64_t(b) * Nq + ii] = hi;
+    f.add(lo, hi);
+  } else {
+    f.all = false;
   }
-}
-
-// Per query block t: the key blocks [kv_lo, kv_hi] (block-local) holding any
-// visible key (empty: lo = 1, hi = 0), and the tightest row range the block
-// shares (lo_max, hi_min; lo_max = INT_MAX if some row is past Nq or sees
-// nothing) for the all-visible test of a key block.
-__global__ void cross_tiles_kernel(const int32_t* __restrict__ row_lo,
-                                   const int32_t* __restrict__ row_hi, int B,
-                                   int Nq, int Nk, int k_off, int bq, int bk,
-                                   int Tq, int32_t* __restrict__ kv_lo,
-                                   int32_t* __restrict__ kv_hi,
-                                   int32_t* __restrict__ lo_max,
-                                   int32_t* __restrict__ hi_min) {
-  // one warp per query block (the whole warp leaves together)
-  const int e = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (e >= B * Tq) return;
-  const int b = e / Tq, t = e - b * Tq;
-  const RangeFold f = fold_ranges(row_lo + int64_t(b) * Nq,
-                                  row_hi + int64_t(b) * Nq, t * bq, bq, Nq,
-                                  lane);
-  if (lane != 0) return;
+  f.warp_reduce();
+  if (lane == 0) part[warp] = f;
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  for (int w = 1; w < kBlock / 32; ++w) f.merge(part[w]);
   if (f.mx < 0 || f.mn > f.mx) {
     kv_lo[e] = 1;
     kv_hi[e] = 0;
@@ -237,50 +232,47 @@ __global__ void cross_tiles_kernel(const int32_t* __restrict__ row_lo,
 }
 
 // Key-side view of the same rule, for the key-major backward: key k
-// (global k_off + jj) is seen by the queries col_lo[k] .. col_hi[k]
-// (global indices, empty when lo > hi): those of its segment from k on.
-__global__ void cross_cols_kernel(const int32_t* __restrict__ seg_q,
-                                  const int32_t* __restrict__ seg_k, int B,
-                                  int Nq, int Nk, int q_off, int k_off,
-                                  int32_t* __restrict__ col_lo,
-                                  int32_t* __restrict__ col_hi) {
-  int64_t total = int64_t(B) * Nk;
-  for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < total;
-       e += int64_t(gridDim.x) * blockDim.x) {
-    const int b = int(e / Nk);
-    const int jj = int(e - int64_t(b) * Nk);
+// (global k_off + jj) is seen by the queries [col_lo, col_hi] (global
+// indices, empty when lo > hi): those of its segment from k on. Per key
+// block j (one CTA of 128 threads, a thread per key): the query blocks
+// [q_lo, q_hi] (chunk-local) holding a query that sees one of its keys
+// (none: lo = 1, hi = 0), and the tightest shared query range (klo_max,
+// khi_min; klo_max = INT_MAX if some key is past Nk or seen by nobody) for
+// the all-visible test of a query block.
+__global__ void __launch_bounds__(kBlock)
+cross_keys_kernel(const int32_t* __restrict__ seg_q,
+                  const int32_t* __restrict__ seg_k, int B, int Nq, int Nk,
+                  int q_off, int k_off, int Tk, int32_t* __restrict__ col_lo,
+                  int32_t* __restrict__ col_hi, int32_t* __restrict__ q_lo,
+                  int32_t* __restrict__ q_hi, int32_t* __restrict__ klo_max,
+                  int32_t* __restrict__ khi_min) {
+  __shared__ RangeFold part[kBlock / 32];
+  const int e = blockIdx.x;
+  const int b = e / Tk, j = e - b * Tk;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int jj = j * kBlock + threadIdx.x;
+  RangeFold f{0x7fffffff, -1, -0x7fffffff, 0x7fffffff, true};
+  if (jj < Nk) {
     const int32_t* sq = seg_q + int64_t(b) * Nq;
-    const int v = seg_k[e];
+    const int v = seg_k[int64_t(b) * Nk + jj];
     int a = 0, z = Nq;  // first query with seg >= v
     while (a < z) { int m = (a + z) >> 1; if (sq[m] < v) a = m + 1; else z = m; }
     const int first = a;
     z = Nq;             // first query with seg > v
     while (a < z) { int m = (a + z) >> 1; if (sq[m] <= v) a = m + 1; else z = m; }
-    col_lo[e] = max(q_off + first, k_off + jj);
-    col_hi[e] = q_off + a - 1;
+    const int lo = max(q_off + first, k_off + jj);
+    const int hi = q_off + a - 1;
+    col_lo[int64_t(b) * Nk + jj] = lo;
+    col_hi[int64_t(b) * Nk + jj] = hi;
+    f.add(lo, hi);
+  } else {
+    f.all = false;
   }
-}
-
-// Per key block j: the query blocks [q_lo, q_hi] (chunk-local) holding a
-// query that sees one of its keys (none: lo = 1, hi = 0), and the tightest
-// shared query range (klo_max, khi_min; klo_max = INT_MAX if some key is
-// past Nk or seen by nobody) for the all-visible test of a query block.
-__global__ void cross_kblocks_kernel(const int32_t* __restrict__ col_lo,
-                                     const int32_t* __restrict__ col_hi,
-                                     int B, int Nq, int Nk, int q_off, int Tk,
-                                     int32_t* __restrict__ q_lo,
-                                     int32_t* __restrict__ q_hi,
-                                     int32_t* __restrict__ klo_max,
-                                     int32_t* __restrict__ khi_min) {
-  // one warp per key block (the whole warp leaves together)
-  const int e = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (e >= B * Tk) return;
-  const int b = e / Tk, j = e - b * Tk;
-  const RangeFold f = fold_ranges(col_lo + int64_t(b) * Nk,
-                                  col_hi + int64_t(b) * Nk, j * kBlock,
-                                  kBlock, Nk, lane);
-  if (lane != 0) return;
+  f.warp_reduce();
+  if (lane == 0) part[warp] = f;
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  for (int w = 1; w < kBlock / 32; ++w) f.merge(part[w]);
   if (f.mx < 0 || f.mn > f.mx) {
     q_lo[e] = 1;
     q_hi[e] = 0;
@@ -416,38 +408,37 @@ __global__ void kv_meta_kernel(int B, int Tq, int Tk,
   q_hi[e] = last;
 }
 
-// Cost of each unit (b, u): units are groups of `rows_per_unit` blocks of
-// the "outer" dimension whose inner ranges [lo, hi] are unioned.
-__global__ void unit_cost_kernel(int B, int T, int group,
-                                 const int32_t* __restrict__ lo,
-                                 const int32_t* __restrict__ hi, int U,
-                                 uint64_t* __restrict__ keys) {
-  int e = blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= B * U) return;
-  int b = e / U, u = e - b * U;
-  int t0 = u * group, t1 = min(t0 + group, T) - 1;
-  int l = 0x7fffffff, h = -1;
-  for (int t = t0; t <= t1; ++t) {
-    if (lo[b * T + t] > hi[b * T + t]) continue;  // no visible key block
-    l = min(l, lo[b * T + t]);
-    h = max(h, hi[b * T + t]);
-  }
-  int cost = h >= l ? h - l + 1 : 0;
-  // ascending key order == descending cost, then ascending unit id
-  keys[e] = (uint64_t(0x7FFFFFFF - cost) << 32) | uint32_t(e);
-}
-
-// Longest-first order: one CTA bitonic-sorts up to kSortMax keys in shared
-// memory; the sorted unit ids are written to order[].
+// Longest-first order: one CTA forms the sort key of every unit (b, u)
+// (units are groups of `group` blocks of the outer dimension whose inner
+// ranges [lo, hi] are unioned; key = descending cost, then ascending unit
+// id) and bitonic-sorts up to kSortMax keys in shared memory; the sorted
+// unit ids are written to order[].
 __global__ void __launch_bounds__(1024)
-lpt_sort_kernel(const uint64_t* __restrict__ keys, int n,
+lpt_sort_kernel(int B, int T, int group, const int32_t* __restrict__ lo,
+                const int32_t* __restrict__ hi, int U,
                 int32_t* __restrict__ order, int32_t* __restrict__ counter) {
   extern __shared__ uint64_t sk[];
   if (threadIdx.x == 0) *counter = 0;  // work counter of the next launch
+  const int n = B * U;
   int p2 = 1;
   while (p2 < n) p2 <<= 1;
-  for (int i = threadIdx.x; i < p2; i += blockDim.x)
-    sk[i] = i < n ? keys[i] : ~0ull;
+  for (int i = threadIdx.x; i < p2; i += blockDim.x) {
+    uint64_t key = ~0ull;
+    if (i < n) {
+      const int b = i / U, u = i - b * U;
+      const int t0 = u * group, t1 = min(t0 + group, T) - 1;
+      int l = 0x7fffffff, h = -1;
+      for (int t = t0; t <= t1; ++t) {
+        const int tl = lo[b * T + t], th = hi[b * T + t];
+        if (tl > th) continue;  // no visible block
+        l = min(l, tl);
+        h = max(h, th);
+      }
+      const int cost = h >= l ? h - l + 1 : 0;
+      key = (uint64_t(0x7FFFFFFF - cost) << 32) | uint32_t(i);
+    }
+    sk[i] = key;
+  }
   __syncthreads();
   for (int size = 2; size <= p2; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
@@ -649,13 +640,10 @@ cudaError_t launch_cross_meta(const int32_t* seg_q, const int32_t* seg_k,
                               cudaStream_t st) {
   const int64_t n = int64_t(B) * Nq;
   if (n == 0) return cudaSuccess;
-  cross_rows_kernel<<<grid_for(n, 256, 148 * 16), 256, 0, st>>>(
-      seg_q, seg_k, B, Nq, Nk, q_off, k_off, row_lo, row_hi);
-  note_launch();
   const int Tq = (Nq + kBlock - 1) / kBlock;
-  cross_tiles_kernel<<<(B * Tq + 3) / 4, 128, 0, st>>>(
-      row_lo, row_hi, B, Nq, Nk, k_off, kBlock, bk, Tq, kv_lo, kv_hi,
-      lo_max, hi_min);
+  cross_meta_kernel<<<B * Tq, kBlock, 0, st>>>(
+      seg_q, seg_k, B, Nq, Nk, q_off, k_off, bk, Tq, row_lo, row_hi, kv_lo,
+      kv_hi, lo_max, hi_min);
   note_launch();
   return cudaGetLastError();
 }
@@ -668,12 +656,10 @@ cudaError_t launch_cross_meta_keys(const int32_t* seg_q, const int32_t* seg_k,
                                    int32_t* khi_min, cudaStream_t st) {
   const int64_t n = int64_t(B) * Nk;
   if (n == 0) return cudaSuccess;
-  cross_cols_kernel<<<grid_for(n, 256, 148 * 16), 256, 0, st>>>(
-      seg_q, seg_k, B, Nq, Nk, q_off, k_off, col_lo, col_hi);
-  note_launch();
   const int Tk = (Nk + kBlock - 1) / kBlock;
-  cross_kblocks_kernel<<<(B * Tk + 3) / 4, 128, 0, st>>>(
-      col_lo, col_hi, B, Nq, Nk, q_off, Tk, q_lo, q_hi, klo_max, khi_min);
+  cross_keys_kernel<<<B * Tk, kBlock, 0, st>>>(
+      seg_q, seg_k, B, Nq, Nk, q_off, k_off, Tk, col_lo, col_hi, q_lo, q_hi,
+      klo_max, khi_min);
   note_launch();
   return cudaGetLastError();
 }
@@ -732,16 +718,12 @@ cudaError_t launch_kv_meta(int B, int Tq, int Tk, const int32_t* kv_lo,
 }
 
 cudaError_t launch_lpt_order(int B, int T, int group, const int32_t* lo,
-                             const int32_t* hi, uint64_t* keys,
-                             int32_t* order, int32_t* counter,
-                             cudaStream_t st) {
+                             const int32_t* hi, int32_t* order,
+                             int32_t* counter, cudaStream_t st) {
   int U = (T + group - 1) / group;
   int n = B * U;
   if (n == 0) return cudaSuccess;
   if (n <= kSortMax) {
-    unit_cost_kernel<<<(n + 255) / 256, 256, 0, st>>>(B, T, group, lo, hi, U,
-                                                       keys);
-    note_launch();
     int p2 = 1;
     while (p2 < n) p2 <<= 1;
     size_t smem = size_t(p2) * sizeof(uint64_t);
@@ -751,7 +733,8 @@ cudaError_t launch_lpt_order(int B, int T, int group, const int32_t* lo,
           int(smem));
       if (e != cudaSuccess) return e;
     }
-    lpt_sort_kernel<<<1, 1024, smem, st>>>(keys, n, order, counter);
+    lpt_sort_kernel<<<1, 1024, smem, st>>>(B, T, group, lo, hi, U, order,
+                                           counter);
     note_launch();
   } else {
     reverse_order_kernel<<<(n + 255) / 256, 256, 0, st>>>(B, U, order,
