@@ -10,6 +10,8 @@ namespace lwm {
 // RingAttention", 提出的方法: RoPE with a context-scaled theta).
 __global__ void rope_table_kernel(double theta, int half_d, int max_pos,
                                   float2* __restrict__ table) {
+  pdl_wait();
+  pdl_trigger();
   int64_t n = int64_t(max_pos) * half_d;
   for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < n;
        e += int64_t(gridDim.x) * blockDim.x) {
@@ -32,6 +34,8 @@ __global__ void rope_apply_kernel(const __nv_bfloat16* __restrict__ x,
                                   int64_t chunks, int H,
                                   __nv_bfloat16* __restrict__ hi,
                                   __nv_bfloat16* __restrict__ lo) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int kChunksPerRow = kHeadDim / 8;
   for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
        e < chunks; e += int64_t(gridDim.x) * blockDim.x) {
@@ -68,6 +72,8 @@ __global__ void rope_apply_half_kernel(const __nv_bfloat16* __restrict__ x,
                                        int64_t items, int H,
                                        __nv_bfloat16* __restrict__ hi,
                                        __nv_bfloat16* __restrict__ lo) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int kItemsPerRow = kHeadDim / 16;
   for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
        e < items; e += int64_t(gridDim.x) * blockDim.x) {
@@ -193,6 +199,8 @@ cross_meta_kernel(const int32_t* __restrict__ seg_q,
                   int32_t* __restrict__ row_lo, int32_t* __restrict__ row_hi,
                   int32_t* __restrict__ kv_lo, int32_t* __restrict__ kv_hi,
                   int32_t* __restrict__ lo_max, int32_t* __restrict__ hi_min) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ RangeFold part[kBlock / 32];
   const int e = blockIdx.x;
   const int b = e / Tq, t = e - b * Tq;
@@ -246,6 +254,8 @@ cross_keys_kernel(const int32_t* __restrict__ seg_q,
                   int32_t* __restrict__ col_hi, int32_t* __restrict__ q_lo,
                   int32_t* __restrict__ q_hi, int32_t* __restrict__ klo_max,
                   int32_t* __restrict__ khi_min) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ RangeFold part[kBlock / 32];
   const int e = blockIdx.x;
   const int b = e / Tk, j = e - b * Tk;
@@ -295,6 +305,8 @@ __global__ void merge_kernel(__nv_bfloat16* __restrict__ out,
                              const __nv_bfloat16* __restrict__ out_p,
                              const float* __restrict__ lse_p, int B, int N,
                              int H) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int kLanesPerRow = kHeadDim / 8;
   constexpr int kRowsPerWarp = 32 / kLanesPerRow;
   const int64_t rows = int64_t(B) * N * H;
@@ -417,6 +429,8 @@ __global__ void __launch_bounds__(1024)
 lpt_sort_kernel(int B, int T, int group, const int32_t* __restrict__ lo,
                 const int32_t* __restrict__ hi, int U,
                 int32_t* __restrict__ order, int32_t* __restrict__ counter) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ uint64_t sk[];
   if (threadIdx.x == 0) *counter = 0;  // work counter of the next launch
   const int n = B * U;
@@ -461,6 +475,8 @@ lpt_sort_kernel(int B, int T, int group, const int32_t* __restrict__ lo,
 // units from last to first (longest first for a causal row).
 __global__ void reverse_order_kernel(int B, int U, int32_t* __restrict__ order,
                                      int32_t* __restrict__ counter) {
+  pdl_wait();
+  pdl_trigger();
   int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e == 0) *counter = 0;
   if (e >= B * U) return;
@@ -490,6 +506,8 @@ template <typename T>
 __global__ void bwd_delta_kernel(const T* __restrict__ out,
                                  const T* __restrict__ dout, int B, int N,
                                  int H, float* __restrict__ delta) {
+  pdl_wait();
+  pdl_trigger();
   int64_t rows = int64_t(B) * N * H;
   int64_t warp = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5;
   int lane = threadIdx.x & 31;
@@ -534,6 +552,8 @@ __global__ void dq_convert_kernel(const float* __restrict__ acc,
                                   const float4* __restrict__ table, int B,
                                   int N, int H, float scale,
                                   T* __restrict__ dq) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int kQuads = kHeadDim / 8;  // groups of 4 pairs per row
   const int64_t total = int64_t(B) * N * H * kQuads;
   for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
@@ -593,8 +613,12 @@ cudaError_t launch_rope_table(double theta, int D, int max_pos, float* table,
                               cudaStream_t st) {
   if (max_pos <= 0) return cudaSuccess;
   int64_t n = int64_t(max_pos) * (D / 2);
-  rope_table_kernel<<<grid_for(n, 256, 148 * 32), 256, 0, st>>>(
-      theta, D / 2, max_pos, reinterpret_cast<float2*>(table));
+  {
+    const cudaError_t le = launch_dependent(
+        rope_table_kernel, dim3(grid_for(n, 256, 148 * 32)), dim3(256), 0, st,
+        theta, D / 2, max_pos, reinterpret_cast<float2*>(table));
+    if (le != cudaSuccess) return le;
+  }
   note_launch();
   return cudaGetLastError();
 }
@@ -617,16 +641,23 @@ cudaError_t launch_rope_apply(const void* x, const int32_t* pos,
   int64_t chunks = int64_t(B) * N * H * (kHeadDim / 8);
   if (chunks == 0) return cudaSuccess;
   if (half) {
-    rope_apply_half_kernel<<<grid_for(chunks / 2, 256, 148 * 16), 256, 0,
-                             st>>>(
-        static_cast<const __nv_bfloat16*>(x), pos,
-        reinterpret_cast<const float2*>(table), chunks / 2, H,
-        static_cast<__nv_bfloat16*>(hi), static_cast<__nv_bfloat16*>(lo));
+    {
+      const cudaError_t le = launch_dependent(
+          rope_apply_half_kernel, dim3(grid_for(chunks / 2, 256, 148 * 16)),
+          dim3(256), 0, st, static_cast<const __nv_bfloat16*>(x), pos,
+          reinterpret_cast<const float2*>(table), chunks / 2, H,
+          static_cast<__nv_bfloat16*>(hi), static_cast<__nv_bfloat16*>(lo));
+      if (le != cudaSuccess) return le;
+    }
   } else {
-    rope_apply_kernel<<<grid_for(chunks, 256, 148 * 16), 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(x), pos,
-        reinterpret_cast<const float2*>(table), chunks, H,
-        static_cast<__nv_bfloat16*>(hi), static_cast<__nv_bfloat16*>(lo));
+    {
+      const cudaError_t le = launch_dependent(
+          rope_apply_kernel, dim3(grid_for(chunks, 256, 148 * 16)), dim3(256),
+          0, st, static_cast<const __nv_bfloat16*>(x), pos,
+          reinterpret_cast<const float2*>(table), chunks, H,
+          static_cast<__nv_bfloat16*>(hi), static_cast<__nv_bfloat16*>(lo));
+      if (le != cudaSuccess) return le;
+    }
   }
   note_launch();
   return cudaGetLastError();
@@ -641,9 +672,13 @@ cudaError_t launch_cross_meta(const int32_t* seg_q, const int32_t* seg_k,
   const int64_t n = int64_t(B) * Nq;
   if (n == 0) return cudaSuccess;
   const int Tq = (Nq + kBlock - 1) / kBlock;
-  cross_meta_kernel<<<B * Tq, kBlock, 0, st>>>(
-      seg_q, seg_k, B, Nq, Nk, q_off, k_off, bk, Tq, row_lo, row_hi, kv_lo,
-      kv_hi, lo_max, hi_min);
+  {
+    const cudaError_t le = launch_dependent(
+        cross_meta_kernel, dim3(B * Tq), dim3(kBlock), 0, st, seg_q, seg_k, B,
+        Nq, Nk, q_off, k_off, bk, Tq, row_lo, row_hi, kv_lo, kv_hi, lo_max,
+        hi_min);
+    if (le != cudaSuccess) return le;
+  }
   note_launch();
   return cudaGetLastError();
 }
@@ -657,9 +692,12 @@ cudaError_t launch_cross_meta_keys(const int32_t* seg_q, const int32_t* seg_k,
   const int64_t n = int64_t(B) * Nk;
   if (n == 0) return cudaSuccess;
   const int Tk = (Nk + kBlock - 1) / kBlock;
-  cross_keys_kernel<<<B * Tk, kBlock, 0, st>>>(
-      seg_q, seg_k, B, Nq, Nk, q_off, k_off, Tk, col_lo, col_hi, q_lo, q_hi,
-      klo_max, khi_min);
+  {
+    const cudaError_t le = launch_dependent(
+        cross_keys_kernel, dim3(B * Tk), dim3(kBlock), 0, st, seg_q, seg_k, B,
+        Nq, Nk, q_off, k_off, Tk, col_lo, col_hi, q_lo, q_hi, klo_max, khi_min);
+    if (le != cudaSuccess) return le;
+  }
   note_launch();
   return cudaGetLastError();
 }
@@ -669,9 +707,13 @@ cudaError_t launch_merge(void* out, float* lse, const void* out_p,
                          cudaStream_t st) {
   const int64_t n = int64_t(B) * N * H * (kHeadDim / 8);
   if (n == 0) return cudaSuccess;
-  merge_kernel<<<grid_for(n, 256, 148 * 16), 256, 0, st>>>(
-      static_cast<__nv_bfloat16*>(out), lse,
-      static_cast<const __nv_bfloat16*>(out_p), lse_p, B, N, H);
+  {
+    const cudaError_t le = launch_dependent(
+        merge_kernel, dim3(grid_for(n, 256, 148 * 16)), dim3(256), 0, st,
+        static_cast<__nv_bfloat16*>(out), lse,
+        static_cast<const __nv_bfloat16*>(out_p), lse_p, B, N, H);
+    if (le != cudaSuccess) return le;
+  }
   note_launch();
   return cudaGetLastError();
 }
@@ -733,12 +775,20 @@ cudaError_t launch_lpt_order(int B, int T, int group, const int32_t* lo,
           int(smem));
       if (e != cudaSuccess) return e;
     }
-    lpt_sort_kernel<<<1, 1024, smem, st>>>(B, T, group, lo, hi, U, order,
-                                           counter);
+    {
+      const cudaError_t le = launch_dependent(
+          lpt_sort_kernel, dim3(1), dim3(1024), smem, st, B, T, group, lo, hi,
+          U, order, counter);
+      if (le != cudaSuccess) return le;
+    }
     note_launch();
   } else {
-    reverse_order_kernel<<<(n + 255) / 256, 256, 0, st>>>(B, U, order,
-                                                           counter);
+    {
+      const cudaError_t le = launch_dependent(
+          reverse_order_kernel, dim3((n + 255) / 256), dim3(256), 0, st, B, U,
+          order, counter);
+      if (le != cudaSuccess) return le;
+    }
     note_launch();
   }
   return cudaGetLastError();
@@ -761,8 +811,12 @@ cudaError_t launch_bwd_delta(const T* out, const T* dout, int B, int N, int H,
   int64_t rows = int64_t(B) * N * H;
   if (rows == 0) return cudaSuccess;
   int64_t threads = rows * 32;
-  bwd_delta_kernel<T><<<int((threads + 255) / 256), 256, 0, st>>>(
-      out, dout, B, N, H, delta);
+  {
+    const cudaError_t le = launch_dependent(
+        bwd_delta_kernel<T>, dim3(int((threads + 255) / 256)), dim3(256), 0, st,
+        out, dout, B, N, H, delta);
+    if (le != cudaSuccess) return le;
+  }
   note_launch();
   return cudaGetLastError();
 }
@@ -775,11 +829,19 @@ cudaError_t launch_dq_convert(const float* acc, const int32_t* pos,
   if (n == 0) return cudaSuccess;
   const float4* t4 = reinterpret_cast<const float4*>(table);
   if (half)
-    dq_convert_kernel<T, true><<<grid_for(n, 256, 148 * 32), 256, 0, st>>>(
-        acc, pos, t4, B, N, H, scale, dq);
+    {
+      const cudaError_t le = launch_dependent(
+          dq_convert_kernel<T, true>, dim3(grid_for(n, 256, 148 * 32)),
+          dim3(256), 0, st, acc, pos, t4, B, N, H, scale, dq);
+      if (le != cudaSuccess) return le;
+    }
   else
-    dq_convert_kernel<T, false><<<grid_for(n, 256, 148 * 32), 256, 0, st>>>(
-        acc, pos, t4, B, N, H, scale, dq);
+    {
+      const cudaError_t le = launch_dependent(
+          dq_convert_kernel<T, false>, dim3(grid_for(n, 256, 148 * 32)),
+          dim3(256), 0, st, acc, pos, t4, B, N, H, scale, dq);
+      if (le != cudaSuccess) return le;
+    }
   note_launch();
   return cudaGetLastError();
 }

@@ -106,6 +106,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
               const __grid_constant__ CUtensorMap tm_do,
               const __grid_constant__ CUtensorMap tm_dq,
               const BwdParams p) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   auto bar = [&](int i) { return sbase + kSBars + 8u * i; };
@@ -765,8 +767,12 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t st) {
                            kSmemBwd);
   if (e != cudaSuccess) return e;
   const int grid = std::min(sm_count(), p.total_items);
-  bwd_tc_kernel<<<grid, kThreadsBwd, kSmemBwd, st>>>(mq, mk, mv, mdo, mdq,
-                                                      p);
+  {
+    const cudaError_t le = launch_dependent(
+        bwd_tc_kernel, dim3(grid), dim3(kThreadsBwd), kSmemBwd, st, mq, mk, mv,
+        mdo, mdq, p);
+    if (le != cudaSuccess) return le;
+  }
   note_launch();
   return cudaGetLastError();
 }

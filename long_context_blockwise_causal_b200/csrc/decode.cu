@@ -91,6 +91,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
                     float scale_log2, float* __restrict__ part_m,
                     float* __restrict__ part_l, float* __restrict__ part_acc,
                     int* status) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ uint8_t dsmem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
@@ -287,6 +289,8 @@ decode_combine_kernel(const float* __restrict__ part_m,
                       const float* __restrict__ part_acc, int H, int splits,
                       __nv_bfloat16* __restrict__ out,
                       float* __restrict__ lse) {
+  pdl_wait();
+  pdl_trigger();
   const int h = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
   const int64_t base = (int64_t(b) * H + h) * splits;
   float M = -INFINITY;
@@ -330,17 +334,24 @@ cudaError_t launch_decode(const void* q, const void* k_rot, const void* v,
       kDecSmem);
   if (e != cudaSuccess) return e;
   const int grid = std::min(n_items, sm_count());
-  decode_split_kernel<<<grid, kDecThreads, kDecSmem, st>>>(
-      mk, mv, static_cast<const __nv_bfloat16*>(q), kv_start, kv_len, q_pos,
-      reinterpret_cast<const float2*>(table), max_pos, L, H, splits, n_items,
-      half, kLog2e / sqrtf(float(kHeadDim)), part_m, part_l, part_acc,
-      status);
+  {
+    const cudaError_t le = launch_dependent(
+        decode_split_kernel, dim3(grid), dim3(kDecThreads), kDecSmem, st, mk,
+        mv, static_cast<const __nv_bfloat16*>(q), kv_start, kv_len, q_pos,
+        reinterpret_cast<const float2*>(table), max_pos, L, H, splits, n_items,
+        half, kLog2e / sqrtf(float(kHeadDim)), part_m, part_l, part_acc,
+        status);
+    if (le != cudaSuccess) return le;
+  }
   note_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  decode_combine_kernel<<<dim3(H, B), kHeadDim, 0, st>>>(
-      part_m, part_l, part_acc, H, splits,
-      static_cast<__nv_bfloat16*>(out), lse);
+  {
+    const cudaError_t le = launch_dependent(
+        decode_combine_kernel, dim3(H, B), dim3(kHeadDim), 0, st, part_m,
+        part_l, part_acc, H, splits, static_cast<__nv_bfloat16*>(out), lse);
+    if (le != cudaSuccess) return le;
+  }
   note_launch();
   return cudaGetLastError();
 }

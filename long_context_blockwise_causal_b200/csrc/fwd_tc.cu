@@ -280,6 +280,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
               const __grid_constant__ CUtensorMap tm_o,
               const __grid_constant__ CUtensorMap tm_klo,
               const FwdParams p) {
+  pdl_wait();
+  pdl_trigger();
   using C = FwdCfg<X3, BK>;
   constexpr int NC = BK / 32;   // 32-column chunks of an S row
   extern __shared__ uint8_t smem_raw[];
@@ -942,8 +944,12 @@ static cudaError_t launch_fwd_impl(const FwdArgs& a, cudaStream_t st) {
                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int grid = std::min(sm_count(), p.total_items);
-  fwd_tc_kernel<X3, BK><<<grid, kThreadsFwd, smem, st>>>(mq, mk, mv, mo, mklo,
-                                                          p);
+  {
+    const cudaError_t le = launch_dependent(
+        fwd_tc_kernel<X3, BK>, dim3(grid), dim3(kThreadsFwd), smem, st, mq, mk,
+        mv, mo, mklo, p);
+    if (le != cudaSuccess) return le;
+  }
   note_launch();
   return cudaGetLastError();
 }
