@@ -508,26 +508,46 @@ __global__ void bwd_delta_kernel(const T* __restrict__ out,
                                  int H, float* __restrict__ delta) {
   pdl_wait();
   pdl_trigger();
-  int64_t rows = int64_t(B) * N * H;
-  int64_t warp = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5;
-  int lane = threadIdx.x & 31;
-  if (warp >= rows) return;
-  const T* o = out + warp * kHeadDim;
-  const T* g = dout + warp * kHeadDim;
-  float acc = 0.f;
+  // 16-byte loads: a row of 128 elements is 16 (bf16) or 32 (fp32) lanes,
+  // so a warp reads 2 or 1 whole rows of each tensor per step
+  constexpr int kEl = 16 / int(sizeof(T));
+  constexpr int kLanesPerRow = kHeadDim / kEl;
+  constexpr int kRowsPerWarp = 32 / kLanesPerRow;
+  const int64_t rows = int64_t(B) * N * H;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / kLanesPerRow, l = lane % kLanesPerRow;
+  const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t w = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5;
+       w * kRowsPerWarp < rows; w += nwarps) {
+    const int64_t row = w * kRowsPerWarp + sub;
+    float acc = 0.f;
+    if (row < rows) {
+      const uint4 a =
+          __ldg(reinterpret_cast<const uint4*>(out + row * kHeadDim) + l);
+      const uint4 c =
+          __ldg(reinterpret_cast<const uint4*>(dout + row * kHeadDim) + l);
+      const uint32_t wa[4] = {a.x, a.y, a.z, a.w};
+      const uint32_t wc[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-  for (int i = 0; i < kHeadDim / 32; ++i) {
-    int d = lane + 32 * i;
-    acc += float(o[d]) * float(g[d]);
-  }
+      for (int e = 0; e < 4; ++e) {
+        if (sizeof(T) == 2) {
+          acc = fmaf(bf16lo_to_f32(wa[e]), bf16lo_to_f32(wc[e]), acc);
+          acc = fmaf(bf16hi_to_f32(wa[e]), bf16hi_to_f32(wc[e]), acc);
+        } else {
+          acc = fmaf(__uint_as_float(wa[e]), __uint_as_float(wc[e]), acc);
+        }
+      }
+    }
 #pragma unroll
-  for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-  if (lane == 0) {
-    int h = int(warp % H);
-    int64_t bn = warp / H;
-    int n = int(bn % N);
-    int b = int(bn / N);
-    delta[(int64_t(b) * H + h) * N + n] = acc;
+    for (int o = kLanesPerRow / 2; o > 0; o >>= 1)
+      acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (l == 0 && row < rows) {
+      const int h = int(row % H);
+      const int64_t bn = row / H;
+      const int n = int(bn % N);
+      const int b = int(bn / N);
+      delta[(int64_t(b) * H + h) * N + n] = acc;
+    }
   }
 }
 
@@ -810,11 +830,12 @@ cudaError_t launch_bwd_delta(const T* out, const T* dout, int B, int N, int H,
                              float* delta, cudaStream_t st) {
   int64_t rows = int64_t(B) * N * H;
   if (rows == 0) return cudaSuccess;
-  int64_t threads = rows * 32;
+  // one warp per 1 (fp32) or 2 (bf16) rows per step, grid-stride
+  const int64_t threads = (rows * int64_t(sizeof(T)) + 3) / 4 * 32;
   {
     const cudaError_t le = launch_dependent(
-        bwd_delta_kernel<T>, dim3(int((threads + 255) / 256)), dim3(256), 0, st,
-        out, dout, B, N, H, delta);
+        bwd_delta_kernel<T>, dim3(grid_for(threads, 256, 148 * 16)),
+        dim3(256), 0, st, out, dout, B, N, H, delta);
     if (le != cudaSuccess) return le;
   }
   note_launch();
