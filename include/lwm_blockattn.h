@@ -415,8 +415,11 @@ LWM_API size_t lwm_blockattn_decode_workspace_size(int B, int H, int D,
  *   out      [B][H][D] bf16;  lse [B][H] fp32 natural log (-inf if the
  *            range is empty, with out = 0)
  * Split over key chunks (partials in the workspace), then merged; reads
- * each visible key and value row once. Only dtype LWM_DTYPE_BF16. Async on
- * stream. */
+ * each visible key and value row once, in 128-key boxes through a TMA
+ * shared-memory ring (k_rot and v must be 16-byte aligned, as every pointer
+ * here). Only dtype LWM_DTYPE_BF16. Async on stream; a load that never
+ * lands ends the kernel after a bounded wait and records LWM_ERR_TIMEOUT
+ * for lwm_blockattn_last_status. */
 LWM_API int lwm_blockattn_decode(const void* q, const void* k_rot,
                                  const void* v, const int32_t* kv_start,
                                  const int32_t* kv_len, const int32_t* q_pos,
