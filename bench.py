@@ -68,13 +68,28 @@ def peaks():
     return d
 
 
+# sources whose change invalidates a recorded DRAM capture: the kernel's
+# own file and the metadata and scheduling kernels that decide which units
+# it runs in which order (its traffic depends on both)
+TRAFFIC_SOURCES = {"fwd_tc_kernel": ("fwd_tc.cu", "aux_kernels.cu"),
+                   "bwd_tc_kernel": ("bwd_tc.cu", "aux_kernels.cu")}
+
+
+def traffic_source_hash(kernel):
+    import hashlib
+    h = hashlib.sha256()
+    for src in TRAFFIC_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "long_context_blockwise_causal_b200",
+                               "csrc", src), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def recorded_traffic(workload, kernel):
     """DRAM bytes per launch of `kernel` from the committed one-pass ncu
     capture (profiles/traffic_<workload>.json), or None when there is no
-    capture for this workload or the kernel's source changed since."""
-    import hashlib
+    capture for this workload or the sources it depends on changed since."""
     p = os.path.join(ROOT, "profiles", f"traffic_{workload}.json")
-    src = {"fwd_tc_kernel": "fwd_tc.cu", "bwd_tc_kernel": "bwd_tc.cu"}[kernel]
     if not os.path.exists(p):
         return None
     with open(p) as f:
@@ -82,10 +97,7 @@ def recorded_traffic(workload, kernel):
     rec = d.get(kernel)
     if not rec:
         return None
-    with open(os.path.join(ROOT, "long_context_blockwise_causal_b200",
-                           "csrc", src), "rb") as f:
-        h = hashlib.sha256(f.read()).hexdigest()[:16]
-    if h != rec.get("source_sha256_16"):
+    if traffic_source_hash(kernel) != rec.get("source_sha256_16"):
         return None
     return rec["dram_read_bytes"] + rec["dram_write_bytes"]
 

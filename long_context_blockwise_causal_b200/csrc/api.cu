@@ -179,7 +179,7 @@ int run_backward(BwdArgs a, const int32_t* seg_q, const int32_t* seg_k,
                                  k_off, w.col_lo, w.col_hi, w.q_lo, w.q_hi,
                                  w.klo_max, w.khi_min, st));
   LWM_TRY(launch_lpt_order(a.B, (a.Nk + kBlock - 1) / kBlock,
-                           kBwdBlocksPerUnit, w.q_lo, w.q_hi,
+                           kBwdBlocksPerUnit, w.q_lo, w.q_hi, 2,
                            w.order_bwd, w.counter, st));
   a.q_lo = w.q_lo; a.q_hi = w.q_hi; a.col_lo = w.col_lo; a.col_hi = w.col_hi;
   a.klo_max = w.klo_max; a.khi_min = w.khi_min;
@@ -201,7 +201,7 @@ int run_forward(const void* q, const void* k_rot, const void* k_rot_lo,
                             w.row_lo, w.row_hi, w.kv_lo, w.kv_hi, w.lo_max,
                             w.hi_min, st));
   LWM_TRY(launch_lpt_order(B, (Nq + kBlock - 1) / kBlock, kFwdBlocksPerUnit,
-                           w.kv_lo, w.kv_hi, w.order_fwd,
+                           w.kv_lo, w.kv_hi, 1, w.order_fwd,
                            w.counter, st));
   FwdArgs a{};
   a.q = q; a.k_rot = k_rot; a.k_rot_lo = k_rot_lo; a.v = v;

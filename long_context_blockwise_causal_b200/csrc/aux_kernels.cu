@@ -427,7 +427,7 @@ __global__ void kv_meta_kernel(int B, int Tq, int Tk,
 // unit ids are written to order[].
 __global__ void __launch_bounds__(1024)
 lpt_sort_kernel(int B, int T, int group, const int32_t* __restrict__ lo,
-                const int32_t* __restrict__ hi, int U,
+                const int32_t* __restrict__ hi, int U, int anchor,
                 int32_t* __restrict__ order, int32_t* __restrict__ counter) {
   pdl_wait();
   pdl_trigger();
@@ -448,8 +448,17 @@ lpt_sort_kernel(int B, int T, int group, const int32_t* __restrict__ lo,
         l = min(l, tl);
         h = max(h, th);
       }
-      const int cost = h >= l ? h - l + 1 : 0;
-      key = (uint64_t(0x7FFFFFFF - cost) << 32) | uint32_t(i);
+      const int cost = min(h >= l ? h - l + 1 : 0, 16383);
+      // packed examples one after another (units of one example share
+      // their range's start, or its end for the key-major backward), so
+      // the SMs work inside one or two examples at a time and their
+      // inputs stay in L2; longest first within an example
+      const int a = anchor == 0 ? 0 : (anchor == 1 ? l : h);
+      const uint64_t loc =
+          h >= l ? uint64_t(b) * uint64_t(T) + uint64_t(max(a, 0)) : 0;
+      // key: example (26 bits) | 16383 - cost (14 bits) | unit id (24 bits;
+      // n <= kSortMax), so ascending order is example, then longest first
+      key = (loc << 38) | (uint64_t(16383 - cost) << 24) | uint32_t(i);
     }
     sk[i] = key;
   }
@@ -468,7 +477,7 @@ lpt_sort_kernel(int B, int T, int group, const int32_t* __restrict__ lo,
     }
   }
   for (int i = threadIdx.x; i < n; i += blockDim.x)
-    order[i] = int32_t(sk[i] & 0xFFFFFFFFu);
+    order[i] = int32_t(sk[i] & 0xFFFFFFu);  // the unit id: the key's low 24 bits
 }
 
 // Fallback order for more units than one CTA can sort: per batch row, the
@@ -780,7 +789,7 @@ cudaError_t launch_kv_meta(int B, int Tq, int Tk, const int32_t* kv_lo,
 }
 
 cudaError_t launch_lpt_order(int B, int T, int group, const int32_t* lo,
-                             const int32_t* hi, int32_t* order,
+                             const int32_t* hi, int anchor, int32_t* order,
                              int32_t* counter, cudaStream_t st) {
   int U = (T + group - 1) / group;
   int n = B * U;
@@ -798,7 +807,7 @@ cudaError_t launch_lpt_order(int B, int T, int group, const int32_t* lo,
     {
       const cudaError_t le = launch_dependent(
           lpt_sort_kernel, dim3(1), dim3(1024), smem, st, B, T, group, lo, hi,
-          U, order, counter);
+          U, anchor, order, counter);
       if (le != cudaSuccess) return le;
     }
     note_launch();

@@ -54,8 +54,10 @@ cudaError_t launch_kv_meta(int B, int Tq, int Tk, const int32_t* kv_lo,
 // Orders the units (b, u), u covering `group` consecutive blocks, by the
 // size of the union of their [lo, hi] ranges, longest first, and zeroes
 // the work counter the following attention launch hands units out with.
+// anchor 1 (2): units are first grouped by the start (end) of that union,
+// i.e. by packed example, in ascending order; 0: longest first only.
 cudaError_t launch_lpt_order(int B, int T, int group, const int32_t* lo,
-                             const int32_t* hi, int32_t* order,
+                             const int32_t* hi, int anchor, int32_t* order,
                              int32_t* counter, cudaStream_t st);
 cudaError_t launch_check_inputs(const int32_t* seg, const int32_t* pos, int B,
                                 int N, int max_pos, int* res, cudaStream_t st);
