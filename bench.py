@@ -257,6 +257,54 @@ def pipelined_e2e(dev, h_in, make_set, run, outputs, h_out, steps):
     return start.elapsed_time(end) / steps
 
 
+def pipelined_e2e_phased(dev, h_in_phases, make_set, run_phases,
+                         output_phases, h_out_phases, steps):
+    """pipelined_e2e for a step made of phases (forward, then backward):
+    phase k's inputs (h_in_phases[k]) are uploaded in order on the upload
+    stream, its compute (run_phases[k]) waits only for them, and its
+    results (output_phases[k] -> h_out_phases[k]) leave as soon as it is
+    done, while the next phase computes. Same two device buffer sets and
+    the same events-on-the-compute-stream timing as pipelined_e2e."""
+    comp = torch.cuda.current_stream(dev)
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    sets = [make_set(), make_set()]
+    nph = len(run_phases)
+    ev = lambda: torch.cuda.Event()
+    uploaded = [[ev() for _ in range(nph)] for _ in range(2)]
+    phase_done = [[ev() for _ in range(nph)] for _ in range(2)]
+    downloaded = [ev(), ev()]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(comp)
+    up.wait_event(start)
+    for i in range(steps):
+        b = i % 2
+        ds = sets[b]
+        if i >= 2:
+            up.wait_event(phase_done[b][nph - 1])  # set b's inputs are free
+            comp.wait_event(downloaded[b])         # set b's outputs are free
+        with torch.cuda.stream(up):
+            for k in range(nph):
+                for n, hb in h_in_phases[k].items():
+                    ds[n].copy_(hb, non_blocking=True)
+                uploaded[b][k].record(up)
+        for k in range(nph):
+            comp.wait_event(uploaded[b][k])
+            run_phases[k](ds)
+            phase_done[b][k].record(comp)
+            down.wait_event(phase_done[b][k])
+            with torch.cuda.stream(down):
+                for hb, db in zip(h_out_phases[k], output_phases[k](ds)):
+                    hb.copy_(db, non_blocking=True)
+        downloaded[b].record(down)
+    comp.wait_event(downloaded[(steps - 1) % 2])
+    if steps >= 2:
+        comp.wait_event(downloaded[(steps - 2) % 2])
+    end.record(comp)
+    torch.cuda.synchronize(dev)
+    return start.elapsed_time(end) / steps
+
+
 # ------------------------------------------------------------------ main
 
 def init_dist(impl):
@@ -895,28 +943,41 @@ def bench_attention(args):
                 d["grads"] = [torch.empty_like(g) for g in grads]
             return d
 
-        def run(d):
-            ops.fwd(d["q"], d["k"], d["v"], d["segment_ids"], d["positions"],
-                    w.theta, max_pos=max_pos, qk_precision=qkp, out=d["out"],
-                    lse=d["lse"], workspace=workspace)
-            if w.backward:
-                ops.bwd(d["q"], d["k"], d["v"], d["out"], d["dout"],
-                        d["lse"], d["segment_ids"], d["positions"], w.theta,
-                        max_pos=max_pos, qk_precision=qkp, dq=d["grads"][0],
-                        dk=d["grads"][1], dv=d["grads"][2],
-                        workspace=workspace)
-
         def outputs(d):
             return [d["out"], d["lse"]] + (d["grads"] if w.backward else [])
 
-        pipelined_e2e(dev, hin, make_set, run, outputs, hout, 2)  # warm-up
+        # phases: the forward needs q, k, v, ids and positions and yields
+        # out and lse; the backward also needs dO and yields the gradients.
+        # Each phase's copies go as soon as they can: dO uploads while the
+        # forward runs, out and lse download while the backward runs.
+        fwd_names = ["q", "k", "v", "segment_ids", "positions"]
+        in_phases = [{n: hin[n] for n in fwd_names}]
+        out_phases = [hout[:2]]
+        run_phases = [lambda d: ops.fwd(
+            d["q"], d["k"], d["v"], d["segment_ids"], d["positions"],
+            w.theta, max_pos=max_pos, qk_precision=qkp, out=d["out"],
+            lse=d["lse"], workspace=workspace)]
+        res_phases = [lambda d: [d["out"], d["lse"]]]
+        if w.backward:
+            in_phases.append({"dout": hin["dout"]})
+            out_phases.append(hout[2:])
+            run_phases.append(lambda d: ops.bwd(
+                d["q"], d["k"], d["v"], d["out"], d["dout"], d["lse"],
+                d["segment_ids"], d["positions"], w.theta, max_pos=max_pos,
+                qk_precision=qkp, dq=d["grads"][0], dk=d["grads"][1],
+                dv=d["grads"][2], workspace=workspace))
+            res_phases.append(lambda d: d["grads"])
+
+        def e2e_run(nsteps):
+            return pipelined_e2e_phased(dev, in_phases, make_set, run_phases,
+                                        res_phases, out_phases, nsteps)
+
+        e2e_run(2)  # warm-up
         s0 = make_set()
         link = copy_floor(dev, hin, s0, hout, outputs(s0))
         del s0
         barrier(ws)
-        ems = max_over_ranks(pipelined_e2e(dev, hin, make_set, run, outputs,
-                                           hout, max(2, args.steps)), ws,
-                             dev)
+        ems = max_over_ranks(e2e_run(max(2, args.steps)), ws, dev)
         compute_ms = fwd_ms + bwd_ms
         e2e = {"value": (fwd_flop + bwd_flop) * job_scale / (ems / 1e3) / 1e12,
                "unit": "TFLOP/s", "ms_per_step": ems,
@@ -932,7 +993,9 @@ def bench_attention(args):
                "copies": "every step uploads its inputs and downloads its "
                          "results through pinned host buffers, on copy "
                          "streams overlapped with the neighbouring steps' "
-                         "compute (two device buffer sets); floor = the "
+                         "compute (two device buffer sets) and, within a "
+                         "step, dO uploaded during the forward and out/lse "
+                         "downloaded during the backward; floor = the "
                          "slower of one step's uploads and downloads run "
                          "together on this link and the step's compute"}
 
