@@ -921,6 +921,35 @@ def bench_attention(args):
         start.elapsed_time(end) / args.steps
     ms = max_over_ranks(ms, ws, dev)
 
+    # a small (launch-bound) forward also as a CUDA graph replay of the same
+    # call, L2 flushed before each replay like the timed calls above
+    graph_us = None
+    if small and not w.backward:
+        gs = torch.cuda.Stream(dev)
+        with torch.cuda.stream(gs):
+            step_fwd = lambda: ops.fwd(
+                t["q"], t["k"], t["v"], t["segment_ids"], t["positions"],
+                w.theta, max_pos=max_pos, qk_precision=qkp, out=out, lse=lse,
+                workspace=workspace, stream=gs)
+            step_fwd()
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=gs):
+            step_fwd()
+        torch.cuda.synchronize(dev)
+        gt = []
+        for _ in range(max(3, args.steps)):
+            flush.zero_()
+            g0 = torch.cuda.Event(enable_timing=True)
+            g1 = torch.cuda.Event(enable_timing=True)
+            g0.record(stream)
+            graph.replay()
+            g1.record(stream)
+            torch.cuda.synchronize(dev)
+            gt.append(g0.elapsed_time(g1))
+        graph_us = float(np.mean(gt)) * 1e3
+        del graph
+
     # end to end through the public API with pinned host buffers
     e2e = None
     if not args.no_e2e:
@@ -1033,7 +1062,8 @@ def bench_attention(args):
                     "unit": "GB/s", "frac": fwd_gbs / pk["hbm_gbs"],
                     "peak_kind": f"copy bandwidth ({pk['source']})",
                     "algorithmic_bytes": fwd_bytes, "traffic": None,
-                    "us_per_call": fwd_ms * 1e3}
+                    "us_per_call": fwd_ms * 1e3,
+                    "graph_replay_us_per_call": graph_us}
         else:
             # the timed region is well under a second of back-to-back
             # launches: the burst peak applies
