@@ -85,15 +85,14 @@ def test_backward_half_matches_oracle(cuda_dev, dtype):
                                 np.abs(r).max()), f"{name}: {err}"
 
 
-def test_decode_half_matches_oracle(cuda_dev):
-    t = _case("packed128k", 700, 2, 2, 4, lo=100, hi=400)
-    B = 2
+def _decode_half_check(N, lengths, lo, hi):
+    B = len(lengths)
+    t = _case("packed128k", N, 2, B, 4, lo=lo, hi=hi)
     seg = t["segment_ids"].cpu().numpy()
     pos = t["positions"].cpu().numpy()
     mp = int(pos.max()) + 1
     table = ops.rope_table(t["theta"], mp)
     k_rot = ops.rope_apply(t["k"], t["positions"], table, rope_layout="half")
-    lengths = [700, 531]
     qi = [L - 1 for L in lengths]
     q = torch.stack([t["q"][b, qi[b]] for b in range(B)])
     start = [int(np.flatnonzero(seg[b] == seg[b, qi[b]])[0]) for b in range(B)]
@@ -104,6 +103,7 @@ def test_decode_half_matches_oracle(cuda_dev):
     out, lse = ops.decode(q, k_rot, t["v"], kv_start, kv_len, q_pos, table,
                           rope_layout="half")
     torch.cuda.synchronize()
+    assert ops.last_status() == ops.OK
     h = _host(t)
     for b in range(B):
         for hh in range(2):
@@ -113,6 +113,16 @@ def test_decode_half_matches_oracle(cuda_dev):
                                          [qi[b]])
             assert np.abs(_np(out[b, hh]) - o[0]).max() <= OUT_TOL
             assert abs(float(lse[b, hh]) - l_[0]) <= LSE_TOL
+
+
+def test_decode_half_matches_oracle(cuda_dev):
+    _decode_half_check(700, [700, 531], 100, 400)
+
+
+def test_decode_half_several_chunks(cuda_dev):
+    # 20000-key caches: three chunks per (row, head), ragged last steps,
+    # examples long enough to span chunk boundaries
+    _decode_half_check(20000, [20000, 17001], 3000, 12000)
 
 
 def test_ring_half_matches_oracle(cuda_dev):
