@@ -660,7 +660,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint64_t kdesc0 = sdesc_sw128(sbase, 16, 1024);
       const uint64_t vdesc0 = sdesc_sw128(sbase + C::kV, C::kKVHalf, 1024);
       int kc = 0, vc = 0;
-      int qc[2] = {0, 0}, pc[2] = {0, 0}, oc[2] = {0, 0};
+      // per sub-tile s, as bits of one word (the issuer's registers are
+      // scarce): parity of Q tiles taken (bit s), of P tiles taken (2 + s),
+      // of O hand-overs (4 + s), any O handed over yet (6 + s); per unit:
+      // Q waited for (8 + s), P.V started (10 + s)
+      uint32_t st = 0;
+      auto bit = [&](int i) { return (st >> i) & 1u; };
+      auto flip = [&](int i) { st ^= 1u << i; };
       bool ok = true;
       for (int n = 0; ok; ++n) {
         ok = mbar_wait(bar(C::bItemFull + (n & 1)), (n >> 1) & 1, abort_flag,
@@ -670,8 +676,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_arrive(bar(C::bItemEmpty + (n & 1)));
         if (it < 0) break;
         Item m = get_item(p, it);
-        bool qwaited[2] = {false, false};
-        bool pv_started[2] = {false, false};
+        st &= 0xFFu;  // the per-unit bits start clear
         int prev = -1;
         for (int j = m.jhi; j >= m.jlo - 1 && ok; --j) {
           const bool has_j = j >= m.jlo;
@@ -692,12 +697,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           #pragma unroll
           for (int s = 0; s < 2 && ok; ++s) {
             if (prev >= 0 && active(m, s, prev)) {
-              ok = mbar_wait(bar(C::bPFull + s), pc[s] & 1, abort_flag,
+              ok = mbar_wait(bar(C::bPFull + s), bit(2 + s), abort_flag,
                              p.status, kWaitLimitNs);
               if (!ok) break;
-              pc[s]++;
-              if (!pv_started[s] && oc[s] > 0) {
-                ok = mbar_wait(bar(C::bOEmpty + s), (oc[s] - 1) & 1,
+              flip(2 + s);
+              if (!bit(10 + s) && bit(6 + s)) {
+                // the previous hand-over of O_s has parity bit(4 + s) ^ 1
+                ok = mbar_wait(bar(C::bOEmpty + s), bit(4 + s) ^ 1u,
                                abort_flag, p.status, kWaitLimitNs);
                 if (!ok) break;
               }
@@ -711,16 +717,16 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
               for (int k = 0; k < BK / 16; ++k)
                 mma_ts(d_tm, a_tm + k * 8, vdesc + uint64_t(k * (2048 >> 4)),
-                       idPV, (pv_started[s] || k > 0) ? 1u : 0u);
-              pv_started[s] = true;
+                       idPV, (bit(10 + s) || k > 0) ? 1u : 0u);
+              st |= 1u << (10 + s);
             }
             if (has_j && active(m, s, j)) {
-              if (!qwaited[s]) {
-                ok = mbar_wait(bar(C::bQReady + s), qc[s] & 1, abort_flag,
+              if (!bit(8 + s)) {
+                ok = mbar_wait(bar(C::bQReady + s), bit(s), abort_flag,
                                p.status, kWaitLimitNs);
                 if (!ok) break;
-                qc[s]++;
-                qwaited[s] = true;
+                flip(s);
+                st |= 1u << (8 + s);
                 tc_fence_after();
               }
               const uint64_t qd = kdesc0 + uint64_t((C::kQ + s * kTileBytes) >> 4);
@@ -766,17 +772,18 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         // epilogue stages the (zero) output in the same buffer
         #pragma unroll
         for (int s = 0; s < 2 && ok; ++s)
-          if (m.present[s] && !qwaited[s]) {
-            ok = mbar_wait(bar(C::bQReady + s), qc[s] & 1, abort_flag,
+          if (m.present[s] && !bit(8 + s)) {
+            ok = mbar_wait(bar(C::bQReady + s), bit(s), abort_flag,
                            p.status, kWaitLimitNs);
-            qc[s]++;
+            flip(s);
           }
         if (!ok) break;
         #pragma unroll
         for (int s = 0; s < 2; ++s)
           if (m.present[s]) {
             mma_commit(bar(C::bOFull + s));
-            oc[s]++;
+            flip(4 + s);
+            st |= 1u << (6 + s);
           }
       }
       // every issued MMA must be complete before TMEM is released
