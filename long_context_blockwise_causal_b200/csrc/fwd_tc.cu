@@ -710,8 +710,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
               tc_fence_after();
               // descriptor start fields are addr >> 4 in the low 14 bits;
               // offsets inside shared memory never carry out of them
-              const uint64_t vdesc =
-                  vdesc0 + uint64_t((vs * C::kKVTile) >> 4);
+              uint64_t vb0;
+              asm volatile("mov.b64 %0, %1;" : "=l"(vb0) : "l"(vdesc0));
+              const uint64_t vdesc = vb0 + uint64_t((vs * C::kKVTile) >> 4);
               const uint32_t a_tm = tmem + s * 128;        // P over S_s
               const uint32_t d_tm = tmem + 256 + s * 128;  // O_s
 #pragma unroll
@@ -729,8 +730,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 st |= 1u << (8 + s);
                 tc_fence_after();
               }
-              const uint64_t qd = kdesc0 + uint64_t((C::kQ + s * kTileBytes) >> 4);
-              const uint64_t kd = kdesc0 + uint64_t((C::kK + ks * C::kKVTile) >> 4);
+              // the base goes through an opaque move, so the compiler
+              // forms each MMA's descriptor here instead of keeping all
+              // of them live across the key-block loop
+              uint64_t kb0;
+              asm volatile("mov.b64 %0, %1;" : "=l"(kb0) : "l"(kdesc0));
+              const uint64_t qd = kb0 + uint64_t((C::kQ + s * kTileBytes) >> 4);
+              const uint64_t kd = kb0 + uint64_t((C::kK + ks * C::kKVTile) >> 4);
               const uint32_t d_tm = tmem + s * 128;
               const int npass = X3 ? 3 : 1;
 #pragma unroll
