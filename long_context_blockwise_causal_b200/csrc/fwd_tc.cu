@@ -35,7 +35,7 @@ namespace {
 constexpr int kThreadsFwd = 16 * 32;
 // Register budget per warpgroup after setmaxnreg (launch: 128 each). The
 // four groups share each SM sub-partition, so the sum must stay 4 x 128.
-constexpr int kRegsSoftmax = 184, kRegsRope = 64, kRegsMisc = 80;
+constexpr int kRegsSoftmax = 184, kRegsRope = 72, kRegsMisc = 72;
 static_assert(2 * kRegsSoftmax + kRegsRope + kRegsMisc == 4 * 128,
               "register split must equal the launch allocation");
 constexpr int kTileBytes = kBlock * kHeadDim * 2;       // 32 KB bf16 tile
