@@ -127,6 +127,28 @@ __device__ __forceinline__ Item get_item(const FwdParams& p, int it) {
   return m;
 }
 
+// (b, h) of work item `it` and the query block of its sub-tile s: the
+// arithmetic of get_item and its one load of the order (the softmax warps
+// recompute this after the key sweep instead of keeping it in registers
+// through it)
+struct Place {
+  int b, h, t;
+};
+
+__device__ __forceinline__ Place item_place(const FwdParams& p, int it,
+                                            int s) {
+  Place q;
+  const int per_group = p.G * p.B * p.U;
+  const int hg = it / per_group;
+  const int rem = it - hg * per_group;
+  const int r = rem / p.G;
+  q.h = hg * p.G + (rem - r * p.G);
+  const int unit = p.order[r];
+  q.b = unit / p.U;
+  q.t = 2 * (unit - q.b * p.U) + s;
+  return q;
+}
+
 __device__ __forceinline__ bool active(const Item& m, int s, int j) {
   return j >= m.lo[s] && j <= m.hi[s];
 }
@@ -476,6 +498,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       if (!ok) break;
       // ---------------------------------------------- epilogue
+      // where this sub-tile's rows go, recomputed (its load overlaps the
+      // wait for the last P.V)
+      const Place pl = item_place(p, it, s);
       ok = mbar_wait(bar(C::bOFull + s), oc & 1, abort_flag, p.status,
                      kWaitLimitNs);
       ok = __all_sync(0xffffffffu, ok);
@@ -515,14 +540,15 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           mbar_wait(bar(C::bEpi + s), (oc - 1) & 1, abort_flag, p.status,
                     kWaitLimitNs)) {
         uint32_t src = sbase + C::kQ + s * kTileBytes;
-        tma_store_4d(&tm_o, src, 0, m.h, q0, m.b);
-        tma_store_4d(&tm_o, src + kHalfTileBytes, 64, m.h, q0, m.b);
+        tma_store_4d(&tm_o, src, 0, pl.h, pl.t * kBlock, pl.b);
+        tma_store_4d(&tm_o, src + kHalfTileBytes, 64, pl.h, pl.t * kBlock,
+                     pl.b);
         bulk_commit();
         bulk_wait_read0();
         mbar_arrive(bar(C::bQEmpty + s));
       }
-      if (valid)
-        p.lse[(int64_t(m.b) * p.H + m.h) * p.Nq + i] =
+      if (pl.t * kBlock + r < p.Nq)
+        p.lse[(int64_t(pl.b) * p.H + pl.h) * p.Nq + pl.t * kBlock + r] =
             l > 0.f ? (m_used + __log2f(l)) * kLn2 : -INFINITY;
     }
     if (threadIdx.x == 0 || threadIdx.x == 128) bulk_wait0();
