@@ -458,21 +458,28 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         // P = 0 (the subtrahend is 0, its scores are -inf)
         const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
         const float2 nsub2 = make_float2(-sub, -sub);
-        float2 lsum = make_float2(0.f, 0.f);
+        // one row-sum accumulator per 32-column chunk: four short add
+        // chains instead of one through the whole row (this is also the
+        // form in which the softmax warps fit their registers unspilled)
+        float2 lsc[NC];
 #pragma unroll
         for (int c = 0; c < NC; ++c) {
           uint32_t pk[16];
+          lsc[c] = make_float2(0.f, 0.f);
 #pragma unroll
           for (int x = 0; x < 32; x += 2) {
             const float2 t = fma2(make_float2(__uint_as_float(v[c][x]),
                                               __uint_as_float(v[c][x + 1])),
                                   sc2, nsub2);
             const float p0 = ex2(t.x), p1 = ex2(t.y);
-            lsum = add2(lsum, make_float2(p0, p1));
+            lsc[c] = add2(lsc[c], make_float2(p0, p1));
             pk[x >> 1] = pack_bf16x2(p0, p1);
           }
           tmem_st16(tS + c * 16, pk);
         }
+        float2 lsum = lsc[0];
+#pragma unroll
+        for (int c = 1; c < NC; ++c) lsum = add2(lsum, lsc[c]);
         l += lsum.x + lsum.y;
         // O holds every P.V issued so far for this row (the S MMA this
         // tile waited on was issued after them); rescale it when the max
